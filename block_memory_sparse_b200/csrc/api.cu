@@ -1,0 +1,535 @@
+// C ABI of the InfLLM layer (include/infllm.h): argument and state checks, device buffers,
+// kernel sequencing on the caller's stream.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <algorithm>
+#include <numeric>
+#include <vector>
+
+#include "../../include/infllm.h"
+#include "common.cuh"
+#include "kernels.h"
+
+using namespace infllm;
+
+namespace {
+
+enum Kind { K_APPEND = 0, K_REPS, K_PREP, K_SELECT, K_ATTEND, K_DECODE, K_NKIND };
+
+struct EventPair {
+    cudaEvent_t a, b;
+    int kind;
+};
+
+}  // namespace
+
+struct infllm_ctx {
+    infllm_config cfg;
+    cudaStream_t stream = nullptr;
+    int device = 0;
+    int elt = 0;
+    Dev D{};
+    std::vector<void*> allocs;
+    void* tmaps = nullptr;      // tensor-core path descriptors (device copy)
+    bool use_tc = false;
+    int* err_host = nullptr;    // mapped pinned word
+    // stream state
+    int64_t tokens = 0;
+    int64_t units_done = 0;
+    bool pending = false;
+    int32_t pending_n = 0;
+    int64_t pending_c0 = 0;
+    int32_t last_nmem = 0, last_kk = 0;
+    int64_t last_B = 0, last_active = 0;
+    bool attended = false;
+    int64_t launches = 0;
+    // profiling
+    bool profiling = false;
+    std::vector<EventPair> events;
+    std::vector<cudaEvent_t> pool;
+    double ms[K_NKIND] = {0};
+    int64_t cnt[K_NKIND] = {0};
+    char err[512] = {0};
+};
+
+namespace {
+
+infllm_status fail(infllm_ctx* c, infllm_status s, const char* fmt, ...) {
+    if (c) {
+        va_list ap;
+        va_start(ap, fmt);
+        vsnprintf(c->err, sizeof(c->err), fmt, ap);
+        va_end(ap);
+    }
+    return s;
+}
+
+#define CK(call)                                                                                      \
+    do {                                                                                              \
+        cudaError_t e_ = (call);                                                                      \
+        if (e_ != cudaSuccess) return fail(c, INFLLM_ECUDA, "%s: %s", #call, cudaGetErrorString(e_)); \
+    } while (0)
+
+cudaEvent_t get_event(infllm_ctx* c) {
+    if (!c->pool.empty()) {
+        cudaEvent_t e = c->pool.back();
+        c->pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+}
+
+// Bracket a launch with events when profiling is on.
+struct Prof {
+    infllm_ctx* c;
+    int kind;
+    cudaEvent_t a = nullptr;
+    Prof(infllm_ctx* c_, int k) : c(c_), kind(k) {
+        if (c->profiling) {
+            a = get_event(c);
+            cudaEventRecord(a, c->stream);
+        }
+    }
+    void done() {
+        if (c->profiling && a) {
+            cudaEvent_t b = get_event(c);
+            cudaEventRecord(b, c->stream);
+            c->events.push_back({a, b, kind});
+            a = nullptr;
+        }
+    }
+};
+
+void collect_events(infllm_ctx* c) {
+    if (c->events.empty()) return;
+    cudaStreamSynchronize(c->stream);
+    for (auto& ev : c->events) {
+        float ms = 0.f;
+        if (cudaEventElapsedTime(&ms, ev.a, ev.b) == cudaSuccess) {
+            c->ms[ev.kind] += ms;
+            c->cnt[ev.kind] += 1;
+        }
+        c->pool.push_back(ev.a);
+        c->pool.push_back(ev.b);
+    }
+    c->events.clear();
+}
+
+template <typename P>
+infllm_status dalloc(infllm_ctx* c, P** p, size_t bytes) {
+    void* q = nullptr;
+    cudaError_t e = cudaMalloc(&q, bytes < 16 ? 16 : bytes);
+    if (e != cudaSuccess) return fail(c, INFLLM_ECUDA, "cudaMalloc(%zu): %s", bytes, cudaGetErrorString(e));
+    c->allocs.push_back(q);
+    *p = (P*)q;
+    return INFLLM_OK;
+}
+
+infllm_status check_device_error(infllm_ctx* c) {
+    if (c->err_host && *(volatile int*)c->err_host != 0)
+        return fail(c, INFLLM_EDEVICE, "device-side check failed (error bits 0x%x)", *(volatile int*)c->err_host);
+    return INFLLM_OK;
+}
+
+infllm_status validate(const infllm_config* g, char* msg, size_t n) {
+    auto bad = [&](const char* m) {
+        snprintf(msg, n, "invalid config: %s", m);
+        return INFLLM_EINVAL;
+    };
+    if (g->n_q_heads <= 0 || g->n_kv_heads <= 0) return bad("head counts must be positive");
+    if (g->n_q_heads % g->n_kv_heads) return bad("n_q_heads must be a multiple of n_kv_heads");
+    if (g->n_q_heads / g->n_kv_heads > 128) return bad("at most 128 q heads per kv head");
+    if (g->head_dim != 64 && g->head_dim != 128) return bad("head_dim must be 64 or 128");
+    if (g->n_sink < 0) return bad("n_sink must be >= 0");
+    if (g->window < 1) return bad("window must be >= 1");
+    if (g->unit_size < 1 || g->unit_size > 1024) return bad("unit_size must be in [1, 1024]");
+    if (g->n_reps < 1 || g->n_reps > 32 || g->n_reps > g->unit_size) return bad("n_reps must be in [1, min(32, unit_size)]");
+    if (g->top_k < 0) return bad("top_k must be >= 0");
+    if (g->max_chunk < 1) return bad("max_chunk must be >= 1");
+    if (g->max_tokens < 1 || g->max_tokens > ((int64_t)1 << 31)) return bad("max_tokens must be in [1, 2^31]");
+    if (!(g->rope_base > 1.0)) return bad("rope_base must be > 1");
+    if (g->dtype != INFLLM_F32 && g->dtype != INFLLM_BF16) return bad("dtype must be INFLLM_F32 or INFLLM_BF16");
+    if (g->score_mode != INFLLM_SCORE_REPS && g->score_mode != INFLLM_SCORE_REPSUM) return bad("unknown score_mode");
+    const int64_t units = g->max_tokens / g->unit_size + 1;
+    if (g->top_k > 32 && units > 16384) return bad("top_k > 32 supports at most 16384 memory units");
+    return INFLLM_OK;
+}
+
+template <typename T>
+infllm_status append_impl(infllm_ctx* c, const void* q, const void* k, const void* v, int32_t n) {
+    const Dev& D = c->D;
+    const int64_t c0 = c->tokens;
+    // representatives of every unit that becomes eligible at c0 (uses queries < c0 only)
+    const int64_t target = n_mem_at(c0, D.S, D.W, D.U);
+    if (target > c->units_done) {
+        Prof p(c, K_REPS);
+        CK(launch_reps<T>(D, c->units_done, target, c->stream));
+        p.done();
+        c->launches += 1;
+        c->units_done = target;
+    }
+    Prof p(c, K_APPEND);
+    CK(launch_append<T>(D, k, v, c0, n, c->stream));
+    int l = 0;
+    CK(launch_ysum<T>(D, q, c0, n, c->stream, &l));
+    p.done();
+    c->launches += 1 + l;
+    c->tokens = c0 + n;
+    c->pending = true;
+    c->pending_n = n;
+    c->pending_c0 = c0;
+    return INFLLM_OK;
+}
+
+template <typename T>
+infllm_status select_impl(infllm_ctx* c, int nm, int n_qtiles, const void* qraw) {
+    int l = 0;
+    Prof p(c, K_SELECT);
+    CK(launch_select<T>(c->D, c->cfg.score_mode, nm, n_qtiles, qraw, c->stream, &l));
+    p.done();
+    c->launches += l;
+    return INFLLM_OK;
+}
+
+void record_attend(infllm_ctx* c, int64_t c0, int n, int nm, int kk, int64_t B) {
+    c->last_nmem = nm;
+    c->last_kk = kk;
+    c->last_B = B;
+    const int64_t t = c0 + n - 1;
+    const int64_t s_eff = std::min<int64_t>(c->cfg.n_sink, t + 1);
+    c->last_active = s_eff + (int64_t)kk * c->cfg.unit_size + std::max<int64_t>(0, t - B + 1);
+    c->attended = true;
+}
+
+template <typename T>
+infllm_status attend_impl(infllm_ctx* c, const void* q, int32_t n, void* out) {
+    const Dev& D = c->D;
+    const int64_t c0 = c->pending_c0;
+    c->pending = false;
+    if (n == 0) return INFLLM_OK;
+    const int nm = (int)n_mem_at(c0, D.S, D.W, D.U);
+    const int kk = std::min(D.topk, nm);
+    const int64_t B = (int64_t)D.S + (int64_t)D.U * nm;
+    {
+        Prof p(c, K_PREP);
+        CK(launch_prep<T>(D, q, c0, n, c->stream));
+        p.done();
+        c->launches += 1;
+    }
+    const int n_qtiles = (n + D.qt - 1) / D.qt;
+    if (kk > 0) {
+        infllm_status s = select_impl<T>(c, nm, n_qtiles, nullptr);
+        if (s != INFLLM_OK) return s;
+    }
+    Prof p(c, K_ATTEND);
+    if (c->use_tc && sizeof(T) == 2) {
+        CK(launch_attend_tc(D, c0, n, kk, B, out, c->stream, c->tmaps));
+    } else {
+        CK(launch_attend_simt<T>(D, c0, n, kk, B, out, c->stream));
+    }
+    p.done();
+    c->launches += 1;
+    record_attend(c, c0, n, nm, kk, B);
+    return INFLLM_OK;
+}
+
+template <typename T>
+infllm_status decode_impl(infllm_ctx* c, const void* q, const void* k, const void* v, void* out) {
+    infllm_status s = append_impl<T>(c, q, k, v, 1);
+    if (s != INFLLM_OK) return s;
+    const Dev& D = c->D;
+    const int64_t t = c->pending_c0;
+    c->pending = false;
+    const int nm = (int)n_mem_at(t, D.S, D.W, D.U);
+    const int kk = std::min(D.topk, nm);
+    const int64_t B = (int64_t)D.S + (int64_t)D.U * nm;
+    if (D.G > 8) {  // wide groups: the chunk kernels handle a single token as well
+        c->pending = true;
+        return attend_impl<T>(c, q, 1, out);
+    }
+    if (kk > 0) {
+        s = select_impl<T>(c, nm, 1, q);
+        if (s != INFLLM_OK) return s;
+    }
+    Prof p(c, K_DECODE);
+    int n_split = 0;
+    cudaError_t e = launch_decode<T>(D, q, t, kk, B, out, c->stream, &n_split);
+    if (e != cudaSuccess) return fail(c, INFLLM_ECUDA, "decode launch (%d splits): %s", n_split, cudaGetErrorString(e));
+    p.done();
+    c->launches += 1;
+    record_attend(c, t, 1, nm, kk, B);
+    return INFLLM_OK;
+}
+
+infllm_status zero_state(infllm_ctx* c) {
+    CK(cudaMemsetAsync(c->D.Y, 0, sizeof(float) * (size_t)((c->D.T_max / c->D.gblk) + 2) * c->D.Hkv * c->D.d, c->stream));
+    CK(cudaMemsetAsync(c->D.counters, 0, sizeof(unsigned) * 2 * c->D.Hkv, c->stream));
+    CK(cudaMemsetAsync(c->D.sel, 0xff, sizeof(int32_t) * (size_t)c->D.Hkv * std::max(1, c->D.topk), c->stream));
+    c->tokens = 0;
+    c->units_done = 0;
+    c->pending = false;
+    c->pending_n = 0;
+    c->attended = false;
+    c->last_nmem = c->last_kk = 0;
+    c->last_B = c->last_active = 0;
+    return INFLLM_OK;
+}
+
+void free_all(infllm_ctx* c) {
+    for (void* p : c->allocs) cudaFree(p);
+    c->allocs.clear();
+    if (c->err_host) cudaFreeHost(c->err_host);
+    c->err_host = nullptr;
+    for (auto& ev : c->events) {
+        cudaEventDestroy(ev.a);
+        cudaEventDestroy(ev.b);
+    }
+    c->events.clear();
+    for (auto e : c->pool) cudaEventDestroy(e);
+    c->pool.clear();
+}
+
+infllm_status create_impl(infllm_ctx* c) {
+    const infllm_config& g = c->cfg;
+    Dev& D = c->D;
+    c->elt = g.dtype == INFLLM_BF16 ? 2 : 4;
+    D.Hq = g.n_q_heads;
+    D.Hkv = g.n_kv_heads;
+    D.G = g.n_q_heads / g.n_kv_heads;
+    D.d = g.head_dim;
+    D.half = g.head_dim / 2;
+    D.S = g.n_sink;
+    D.W = g.window;
+    D.U = g.unit_size;
+    D.r = g.n_reps;
+    D.topk = g.top_k;
+    D.gblk = std::gcd(g.unit_size, g.window);
+    D.T_max = g.max_tokens;
+    D.units_max = g.max_tokens / g.unit_size + 1;
+    D.inv_sqrt_d = (float)(1.0 / sqrt((double)g.head_dim));
+    D.qt = std::max(1, 128 / D.G);
+    const int rpt = D.qt * D.G;
+    D.qtiles_max = (g.max_chunk + D.qt - 1) / D.qt;
+    D.qrows_max = (int64_t)D.qtiles_max * rpt;
+    D.score_splits_max = (int)std::min<int64_t>(1024, (D.units_max + 255) / 256 + 1);
+    const int SK = decode_split_keys(c->elt);
+    D.dec_splits_max = (int)((std::min<int64_t>(g.n_sink, g.max_tokens) + (int64_t)g.top_k * g.unit_size +
+                              (int64_t)g.window + g.unit_size + 1 + SK - 1) / SK) + 1;
+    D.P_rel = std::max(g.window, g.unit_size) + 1;
+
+    CK(cudaGetDevice(&c->device));
+    const size_t store = (size_t)D.Hkv * D.T_max * D.d * c->elt;
+    infllm_status s;
+#define AL(ptr, bytes)                         \
+    if ((s = dalloc(c, &(ptr), (bytes))) != INFLLM_OK) return s;
+    AL(D.Kraw, store);
+    AL(D.Krot, store);
+    AL(D.V, store);
+    AL(D.Y, sizeof(float) * (size_t)((D.T_max / D.gblk) + 2) * D.Hkv * D.d);
+    AL(D.rep_ids, sizeof(int32_t) * (size_t)D.Hkv * D.units_max * D.r);
+    AL(D.rep_keys, (size_t)D.Hkv * D.units_max * D.r * D.d * c->elt);
+    AL(D.repsum, sizeof(float) * (size_t)D.Hkv * D.units_max * D.d);
+    AL(D.sel, sizeof(int32_t) * (size_t)D.Hkv * std::max(1, D.topk));
+    AL(D.uscore, sizeof(float) * (size_t)D.Hkv * D.units_max);
+    AL(D.qbar_part, sizeof(float) * (size_t)D.Hkv * D.qtiles_max * D.d);
+    AL(D.cand, sizeof(uint64_t) * (size_t)D.Hkv * D.score_splits_max * 32);
+    AL(D.counters, sizeof(unsigned) * 2 * D.Hkv);
+    AL(D.Qm, (size_t)D.Hkv * D.qrows_max * D.d * c->elt);
+    AL(D.Qw, (size_t)D.Hkv * D.qrows_max * D.d * c->elt);
+    AL(D.cs_chunk, sizeof(float2) * (size_t)g.max_chunk * D.half);
+    AL(D.dec_part, sizeof(float) * (size_t)D.Hkv * D.dec_splits_max * D.G * (D.d + 2));
+    double* invf = nullptr;
+    float2* cs_rel = nullptr;
+    float2* cs_w = nullptr;
+    AL(invf, sizeof(double) * D.half);
+    AL(cs_rel, sizeof(float2) * (size_t)D.P_rel * D.half);
+    AL(cs_w, sizeof(float2) * D.half);
+#undef AL
+    // position tables, fp64 on the host
+    std::vector<double> th(D.half);
+    for (int i = 0; i < D.half; ++i) th[i] = pow(g.rope_base, -2.0 * i / (double)D.d);
+    std::vector<float2> rel((size_t)D.P_rel * D.half), w(D.half);
+    for (int p = 0; p < D.P_rel; ++p)
+        for (int i = 0; i < D.half; ++i) rel[(size_t)p * D.half + i] = make_float2((float)cos(p * th[i]), (float)sin(p * th[i]));
+    for (int i = 0; i < D.half; ++i) w[i] = make_float2((float)cos(g.window * th[i]), (float)sin(g.window * th[i]));
+    CK(cudaMemcpy(invf, th.data(), sizeof(double) * D.half, cudaMemcpyHostToDevice));
+    CK(cudaMemcpy(cs_rel, rel.data(), sizeof(float2) * rel.size(), cudaMemcpyHostToDevice));
+    CK(cudaMemcpy(cs_w, w.data(), sizeof(float2) * w.size(), cudaMemcpyHostToDevice));
+    D.inv_freq = invf;
+    D.cs_rel = cs_rel;
+    D.cs_W = cs_w;
+    CK(cudaHostAlloc((void**)&c->err_host, sizeof(int), cudaHostAllocMapped));
+    *c->err_host = 0;
+    CK(cudaHostGetDevicePointer((void**)&D.err, c->err_host, 0));
+    c->use_tc = attend_tc_supported(D) && g.dtype == INFLLM_BF16 && getenv("INFLLM_FORCE_SIMT") == nullptr;
+    infllm_status zs = zero_state(c);
+    if (zs != INFLLM_OK) return zs;
+    CK(cudaStreamSynchronize(c->stream));
+    return INFLLM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* infllm_version(void) { return "infllm-b200 0.1"; }
+
+const char* infllm_last_error(infllm_ctx* ctx) { return ctx ? ctx->err : "null context"; }
+
+infllm_status infllm_create(const infllm_config* cfg, void* cuda_stream, infllm_ctx** out) {
+    if (!out) return INFLLM_EINVAL;
+    *out = nullptr;
+    if (!cfg) return INFLLM_EINVAL;
+    char msg[256];
+    infllm_status s = validate(cfg, msg, sizeof(msg));
+    if (s != INFLLM_OK) return s;
+    infllm_ctx* c = new infllm_ctx();
+    c->cfg = *cfg;
+    c->stream = (cudaStream_t)cuda_stream;
+    s = create_impl(c);
+    if (s != INFLLM_OK) {
+        fprintf(stderr, "infllm_create: %s\n", c->err);
+        free_all(c);
+        delete c;
+        return s;
+    }
+    *out = c;
+    return INFLLM_OK;
+}
+
+infllm_status infllm_destroy(infllm_ctx* c) {
+    if (!c) return INFLLM_OK;
+    cudaStreamSynchronize(c->stream);
+    free_all(c);
+    delete c;
+    return INFLLM_OK;
+}
+
+infllm_status infllm_reset(infllm_ctx* c) {
+    if (!c) return INFLLM_EINVAL;
+    return zero_state(c);
+}
+
+infllm_status infllm_append_chunk(infllm_ctx* c, const void* q, const void* k, const void* v, int32_t n) {
+    if (!c) return INFLLM_EINVAL;
+    infllm_status s = check_device_error(c);
+    if (s != INFLLM_OK) return s;
+    if (n < 0) return fail(c, INFLLM_EINVAL, "append: n = %d < 0", n);
+    if (n > c->cfg.max_chunk) return fail(c, INFLLM_EINVAL, "append: n = %d > max_chunk = %d", n, c->cfg.max_chunk);
+    if (c->tokens + n > c->cfg.max_tokens)
+        return fail(c, INFLLM_ECAPACITY, "append: %lld + %d tokens exceed max_tokens = %lld", (long long)c->tokens, n,
+                    (long long)c->cfg.max_tokens);
+    if (n == 0) {
+        c->pending = true;
+        c->pending_n = 0;
+        c->pending_c0 = c->tokens;
+        return INFLLM_OK;
+    }
+    if (!q || !k || !v) return fail(c, INFLLM_EINVAL, "append: null pointer");
+    return c->cfg.dtype == INFLLM_BF16 ? append_impl<__nv_bfloat16>(c, q, k, v, n) : append_impl<float>(c, q, k, v, n);
+}
+
+infllm_status infllm_attend_chunk(infllm_ctx* c, const void* q, int32_t n, void* out) {
+    if (!c) return INFLLM_EINVAL;
+    infllm_status s = check_device_error(c);
+    if (s != INFLLM_OK) return s;
+    if (!c->pending) return fail(c, INFLLM_ESTATE, "attend: no appended chunk is waiting");
+    if (n != c->pending_n)
+        return fail(c, INFLLM_ESTATE, "attend: n = %d does not match the appended chunk (%d)", n, c->pending_n);
+    if (n > 0 && (!q || !out)) return fail(c, INFLLM_EINVAL, "attend: null pointer");
+    return c->cfg.dtype == INFLLM_BF16 ? attend_impl<__nv_bfloat16>(c, q, n, out) : attend_impl<float>(c, q, n, out);
+}
+
+infllm_status infllm_decode_step(infllm_ctx* c, const void* q, const void* k, const void* v, void* out) {
+    if (!c) return INFLLM_EINVAL;
+    infllm_status s = check_device_error(c);
+    if (s != INFLLM_OK) return s;
+    if (!q || !k || !v || !out) return fail(c, INFLLM_EINVAL, "decode: null pointer");
+    if (c->cfg.max_chunk < 1) return fail(c, INFLLM_EINVAL, "decode: max_chunk < 1");
+    if (c->tokens + 1 > c->cfg.max_tokens)
+        return fail(c, INFLLM_ECAPACITY, "decode: max_tokens = %lld reached", (long long)c->cfg.max_tokens);
+    return c->cfg.dtype == INFLLM_BF16 ? decode_impl<__nv_bfloat16>(c, q, k, v, out) : decode_impl<float>(c, q, k, v, out);
+}
+
+infllm_status infllm_get_selection(infllm_ctx* c, int32_t* host_sel) {
+    if (!c || !host_sel) return INFLLM_EINVAL;
+    if (c->cfg.top_k == 0) return INFLLM_OK;
+    CK(cudaStreamSynchronize(c->stream));
+    CK(cudaMemcpy(host_sel, c->D.sel, sizeof(int32_t) * (size_t)c->D.Hkv * c->D.topk, cudaMemcpyDeviceToHost));
+    // entries beyond the last chunk's selection are not rewritten by the kernels
+    for (int h = 0; h < c->D.Hkv; ++h)
+        for (int i = c->last_kk; i < c->D.topk; ++i) host_sel[h * c->D.topk + i] = -1;
+    return check_device_error(c);
+}
+
+infllm_status infllm_get_unit_scores(infllm_ctx* c, float* host_scores, int32_t capacity, int32_t* n_mem_out) {
+    if (!c || !n_mem_out) return INFLLM_EINVAL;
+    *n_mem_out = c->last_nmem;
+    if (!host_scores) return INFLLM_OK;
+    if (capacity < c->last_nmem) return fail(c, INFLLM_EINVAL, "unit scores: capacity %d < n_mem %d", capacity, c->last_nmem);
+    if (c->last_nmem == 0 || c->cfg.top_k == 0) return INFLLM_OK;
+    CK(cudaStreamSynchronize(c->stream));
+    CK(cudaMemcpy2D(host_scores, sizeof(float) * c->last_nmem, c->D.uscore, sizeof(float) * c->D.units_max,
+                    sizeof(float) * c->last_nmem, c->D.Hkv, cudaMemcpyDeviceToHost));
+    return check_device_error(c);
+}
+
+infllm_status infllm_get_reps(infllm_ctx* c, int32_t unit_begin, int32_t n_units, int32_t* host_ids) {
+    if (!c || !host_ids || unit_begin < 0 || n_units < 0) return INFLLM_EINVAL;
+    if ((int64_t)unit_begin + n_units > c->units_done)
+        return fail(c, INFLLM_ESTATE, "reps: units [%d, %d) requested, %lld have representatives", unit_begin,
+                    unit_begin + n_units, (long long)c->units_done);
+    if (n_units == 0) return INFLLM_OK;
+    CK(cudaStreamSynchronize(c->stream));
+    const size_t row = sizeof(int32_t) * (size_t)n_units * c->D.r;
+    CK(cudaMemcpy2D(host_ids, row, c->D.rep_ids + (size_t)unit_begin * c->D.r, sizeof(int32_t) * (size_t)c->D.units_max * c->D.r,
+                    row, c->D.Hkv, cudaMemcpyDeviceToHost));
+    return check_device_error(c);
+}
+
+infllm_status infllm_get_stats(infllm_ctx* c, infllm_stats* o) {
+    if (!c || !o) return INFLLM_EINVAL;
+    collect_events(c);
+    memset(o, 0, sizeof(*o));
+    o->tokens = c->tokens;
+    o->units_with_reps = c->units_done;
+    o->n_mem = c->last_nmem;
+    o->n_selected = c->last_kk;
+    o->window_base = c->last_B;
+    o->active_tokens = c->last_active;
+    o->kernel_launches = c->launches;
+    o->ms_append = c->ms[K_APPEND];
+    o->ms_reps = c->ms[K_REPS];
+    o->ms_prep = c->ms[K_PREP];
+    o->ms_select = c->ms[K_SELECT];
+    o->ms_attend = c->ms[K_ATTEND];
+    o->ms_decode = c->ms[K_DECODE];
+    o->n_append = c->cnt[K_APPEND];
+    o->n_reps = c->cnt[K_REPS];
+    o->n_prep = c->cnt[K_PREP];
+    o->n_select = c->cnt[K_SELECT];
+    o->n_attend = c->cnt[K_ATTEND];
+    o->n_decode = c->cnt[K_DECODE];
+    return INFLLM_OK;
+}
+
+infllm_status infllm_set_profiling(infllm_ctx* c, int32_t enable) {
+    if (!c) return INFLLM_EINVAL;
+    collect_events(c);
+    c->profiling = enable != 0;
+    for (int k = 0; k < K_NKIND; ++k) {
+        c->ms[k] = 0;
+        c->cnt[k] = 0;
+    }
+    c->launches = 0;
+    return INFLLM_OK;
+}
+
+}  // extern "C"

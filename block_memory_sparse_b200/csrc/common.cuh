@@ -1,0 +1,145 @@
+// Shared device-side definitions for the InfLLM layer kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace infllm {
+
+// Everything a kernel needs to know about the layer and the context's device buffers.
+// Passed by value to every kernel.
+struct Dev {
+    // shape
+    int Hq, Hkv, G, d, half;
+    int S, W, U, r, topk;
+    int gblk;             // query-sum block length (gcd(U, W)); blocks start at token S
+    int64_t T_max;        // token capacity
+    int64_t units_max;    // unit capacity
+    float inv_sqrt_d;
+    // stores, [Hkv][T_max][d] in the context dtype
+    void* Kraw;           // keys as given (sinks and memory frame)
+    void* Krot;           // R(n) k_n (window frame, absolute position n)
+    void* V;
+    // query block sums: Y[b][hk][d] = sum_{t in block b} sum_{h in group hk} R(t - s_b) q_{t,h}
+    float* Y;
+    // representatives
+    int32_t* rep_ids;     // [Hkv][units_max][r] unit-local offsets, ascending
+    void* rep_keys;       // [Hkv][units_max][r][d] raw keys (context dtype)
+    float* repsum;        // [Hkv][units_max][d] fp32 sum of the r raw keys
+    // lookup
+    int32_t* sel;         // [Hkv][topk] ascending ids, -1 padded
+    float* uscore;        // [Hkv][units_max] last chunk's unit scores
+    float* qbar_part;     // [Hkv][qtiles_max][d] per-tile raw query sums
+    uint64_t* cand;       // [Hkv][score_splits_max][32] top-k candidate lists
+    unsigned* counters;   // [Hkv] arrival counters (last-block-done)
+    // rotated, packed queries of the current chunk: [Hkv][rows][d] (rows tile-ordered)
+    void* Qm;             // R(W) q  (sink / memory frame)
+    void* Qw;             // R(t) q  (window frame)
+    int64_t qrows_max;    // rows capacity per kv head
+    int qt;               // queries per 128-row tile (128 / G, or 1 when G > 128)
+    // position tables
+    const double* inv_freq;  // [half] theta_i in fp64
+    const float2* cs_rel;    // [P_rel][half] (cos, sin)(p theta_i), p < P_rel
+    int P_rel;
+    const float2* cs_W;      // [half] (cos, sin)(W theta_i)
+    float2* cs_chunk;        // [max_chunk][half] (cos, sin)(t theta_i) for the current chunk
+    // decode partials: [Hkv][dec_splits_max][G][d + 2]
+    float* dec_part;
+    int dec_splits_max;
+    int score_splits_max;
+    int qtiles_max;
+    // error word (host-mapped)
+    int* err;
+};
+
+enum ErrBits : int {
+    ERR_SEL_RANGE = 1,     // a selected unit id outside [0, n_mem)
+    ERR_REP_RANGE = 2,     // a representative id outside [0, U)
+    ERR_SPLIT_RANGE = 4,   // decode split bookkeeping out of range
+    ERR_TILE_SCHED = 8,    // attention tile bookkeeping out of range
+};
+
+__device__ __forceinline__ void set_err(const Dev& D, int bit) { atomicOr(D.err, bit); }
+
+// ---- element conversions --------------------------------------------------------------
+template <typename T> __device__ __forceinline__ float to_f(T x);
+template <> __device__ __forceinline__ float to_f<float>(float x) { return x; }
+template <> __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <typename T> __device__ __forceinline__ T from_f(float x);
+template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
+
+// ---- ordered composite keys for deterministic top-k ------------------------------------
+// Larger key = better.  High word: order-preserving image of the float score (+0 == -0).
+// Low word: ~index, so among equal scores the lower index wins.
+__device__ __forceinline__ uint32_t ordered_bits(float s) {
+    s = s + 0.0f;  // canonicalise -0 to +0
+    uint32_t u = __float_as_uint(s);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ uint64_t make_key(float s, uint32_t idx) {
+    return ((uint64_t)ordered_bits(s) << 32) | (uint64_t)(~idx);
+}
+__device__ __forceinline__ uint32_t key_index(uint64_t key) { return ~(uint32_t)(key & 0xffffffffu); }
+
+__device__ __forceinline__ uint64_t shfl_xor64(uint64_t x, int m) {
+    return __shfl_xor_sync(0xffffffffu, x, m);
+}
+__device__ __forceinline__ uint64_t shfl64(uint64_t x, int src) { return __shfl_sync(0xffffffffu, x, src); }
+
+// Sort one key per lane descending across the warp (bitonic network).
+__device__ __forceinline__ uint64_t warp_sort_desc(uint64_t x) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            uint64_t o = shfl_xor64(x, j);
+            bool desc = (lane & k) == 0;
+            bool lower = (lane & j) == 0;
+            uint64_t mx = x > o ? x : o, mn = x > o ? o : x;
+            x = (lower == desc) ? mx : mn;
+        }
+    }
+    return x;
+}
+
+// Merge two warp-wide descending lists (one element per lane) and keep the top 32, descending.
+__device__ __forceinline__ uint64_t warp_merge_desc(uint64_t a, uint64_t b) {
+    const int lane = threadIdx.x & 31;
+    uint64_t br = shfl64(b, 31 - lane);
+    uint64_t x = a > br ? a : br;  // bitonic sequence holding the top 32 of a U b
+#pragma unroll
+    for (int j = 16; j > 0; j >>= 1) {
+        uint64_t o = shfl_xor64(x, j);
+        bool lower = (lane & j) == 0;
+        x = lower ? (x > o ? x : o) : (x > o ? o : x);
+    }
+    return x;
+}
+
+// Insert one candidate per lane (0 = none) into a running descending top-32 list.
+__device__ __forceinline__ uint64_t warp_topk_insert(uint64_t list, uint64_t cand) {
+    uint64_t thr = shfl64(list, 31);
+    if (__ballot_sync(0xffffffffu, cand > thr) == 0u) return list;
+    return warp_merge_desc(list, warp_sort_desc(cand));
+}
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+    for (int m = 16; m > 0; m >>= 1) x += __shfl_xor_sync(0xffffffffu, x, m);
+    return x;
+}
+__device__ __forceinline__ float warp_max(float x) {
+#pragma unroll
+    for (int m = 16; m > 0; m >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, m));
+    return x;
+}
+
+__host__ __device__ __forceinline__ int64_t n_mem_at(int64_t c0, int S, int W, int U) {
+    int64_t x = c0 - (int64_t)W - (int64_t)S;
+    return x > 0 ? x / U : 0;
+}
+
+}  // namespace infllm

@@ -1,0 +1,44 @@
+// Host-side launchers of the layer kernels (implemented in the .cu files of this directory).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace infllm {
+
+template <typename T>
+cudaError_t launch_append(const Dev& D, const void* k, const void* v, int64_t c0, int n, cudaStream_t st);
+template <typename T>
+cudaError_t launch_ysum(const Dev& D, const void* q, int64_t c0, int n, cudaStream_t st, int* launches);
+template <typename T>
+cudaError_t launch_reps(const Dev& D, int64_t j0, int64_t j1, cudaStream_t st);
+
+// Rotated, packed queries of the chunk + per-tile raw query sums.
+template <typename T>
+cudaError_t launch_prep(const Dev& D, const void* q, int64_t c0, int n, cudaStream_t st);
+
+// Unit scores and top-k selection.  `qraw` != null: single-token query (decode) summed in place
+// of the per-tile partials.  Returns the number of kernels launched in *launches.
+template <typename T>
+cudaError_t launch_select(const Dev& D, int score_mode, int n_mem, int n_qtiles, const void* qraw,
+                          cudaStream_t st, int* launches);
+
+// Exact attention over sinks U selected units U window for a chunk (SIMT fp32-accumulate path).
+template <typename T>
+cudaError_t launch_attend_simt(const Dev& D, int64_t c0, int n, int kk, int64_t B, void* out, cudaStream_t st);
+
+// Exact attention for a chunk on the tcgen05 tensor cores (bf16 in, fp32 accumulate).
+cudaError_t launch_attend_tc(const Dev& D, int64_t c0, int n, int kk, int64_t B, void* out, cudaStream_t st,
+                             const void* tmaps);
+bool attend_tc_supported(const Dev& D);
+
+// Split-KV decode attention for one token with a log-sum-exp merge.
+template <typename T>
+cudaError_t launch_decode(const Dev& D, const void* q, int64_t t, int kk, int64_t B, void* out, cudaStream_t st,
+                          int* n_split_out);
+
+int decode_split_keys(int elt_bytes);
+
+}  // namespace infllm

@@ -1,0 +1,296 @@
+// Unit lookup: score every eligible memory unit against the chunk's queries and keep the
+// top-k per kv head, ties to the lower unit index.
+//
+// Method: "InfLLM Guide: Training-Free Long-Context Memory Units", "Core Innovation 2",
+// item 2 "Query-Aware Top-K Scoring and Loading" (Score(M_j) = q . r_j / sqrt(d), keep the
+// top-k); lookup per chunk during pre-filling: OpenReview rebuttal (paperhub.cn), Q2.
+// A chunk's score of unit j sums the scaled logits of every (query, q head of the group,
+// representative) triple, with the query at relative distance W:
+//   sigma_j = <R(W) sum_t sum_h q_{t,h}, sum_m k_{j,m}> / sqrt(d)
+// which is linear, so the queries are summed first (prep kernel) and each unit costs one
+// read of its representative keys (REPS mode) or of their fp32 sum (REPSUM mode).
+#include "common.cuh"
+#include "kernels.h"
+
+namespace infllm {
+
+// Rotated, packed queries of the chunk.  Grid (tiles, Hkv).  Tile a holds queries
+// [a*qt, a*qt + qt); row r of a tile is (head hg = r / qt, query a*qt + r % qt).
+// Also writes each tile's raw query sum over its rows (fixed-order reduction).
+template <typename T>
+__global__ void k_prep(Dev D, const T* __restrict__ q, int n) {
+    extern __shared__ float red[];
+    const int a = blockIdx.x, hk = blockIdx.y;
+    const int rows = D.qt * D.G;
+    const int i = threadIdx.x % D.half, rg = threadIdx.x / D.half, nrg = blockDim.x / D.half;
+    const float2 cw = D.cs_W[i];
+    T* Qm = (T*)D.Qm + ((int64_t)hk * D.qrows_max + (int64_t)a * rows) * D.d;
+    T* Qw = (T*)D.Qw + ((int64_t)hk * D.qrows_max + (int64_t)a * rows) * D.d;
+    float s1 = 0.f, s2 = 0.f;
+    for (int r = rg; r < rows; r += nrg) {
+        const int hg = r / D.qt, tl = a * D.qt + r % D.qt;
+        float m1 = 0.f, m2 = 0.f, w1 = 0.f, w2 = 0.f;
+        if (tl < n) {
+            const T* src = q + ((int64_t)tl * D.Hq + hk * D.G + hg) * D.d;
+            const float x1 = to_f(src[i]), x2 = to_f(src[i + D.half]);
+            s1 += x1;
+            s2 += x2;
+            m1 = x1 * cw.x - x2 * cw.y;
+            m2 = x2 * cw.x + x1 * cw.y;
+            const float2 ct = D.cs_chunk[(int64_t)tl * D.half + i];
+            w1 = x1 * ct.x - x2 * ct.y;
+            w2 = x2 * ct.x + x1 * ct.y;
+        }
+        Qm[(int64_t)r * D.d + i] = from_f<T>(m1);
+        Qm[(int64_t)r * D.d + i + D.half] = from_f<T>(m2);
+        Qw[(int64_t)r * D.d + i] = from_f<T>(w1);
+        Qw[(int64_t)r * D.d + i + D.half] = from_f<T>(w2);
+    }
+    red[rg * D.d + i] = s1;
+    red[rg * D.d + i + D.half] = s2;
+    __syncthreads();
+    if (rg == 0) {
+        float a1 = 0.f, a2 = 0.f;
+        for (int g = 0; g < nrg; ++g) {
+            a1 += red[g * D.d + i];
+            a2 += red[g * D.d + i + D.half];
+        }
+        float* p = D.qbar_part + ((int64_t)hk * D.qtiles_max + a) * D.d;
+        p[i] = a1;
+        p[i + D.half] = a2;
+    }
+}
+
+// 16-byte vector of the score operand, converted to floats.
+template <typename T> struct Vec16;
+template <> struct Vec16<__nv_bfloat16> {
+    static constexpr int N = 8;
+    __device__ __forceinline__ static void load(const __nv_bfloat16* p, float* f) {
+        uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            float2 x = __bfloat1622float2(h[c]);
+            f[2 * c] = x.x;
+            f[2 * c + 1] = x.y;
+        }
+    }
+};
+template <> struct Vec16<float> {
+    static constexpr int N = 4;
+    __device__ __forceinline__ static void load(const float* p, float* f) {
+        float4 u = __ldg(reinterpret_cast<const float4*>(p));
+        f[0] = u.x; f[1] = u.y; f[2] = u.z; f[3] = u.w;
+    }
+};
+
+// Grid (n_split, Hkv), 256 threads.  Lane-per-unit scoring (each lane streams one unit's
+// operand in 16-byte loads), warp top-32 lists, CTA merge, then the last CTA of each kv head
+// merges every CTA's list (arrival counter, no waiting) and writes the selection.
+template <typename T, int MODE>
+__global__ void __launch_bounds__(256) k_score_topk(Dev D, int n_mem, int n_split, int n_qtiles, const T* qraw,
+                                                    int do_select) {
+    __shared__ float qb[128];
+    __shared__ uint64_t lists[8][32];
+    __shared__ int is_last;
+    const int split = blockIdx.x, hk = blockIdx.y;
+    for (int i = threadIdx.x; i < D.half; i += blockDim.x) {
+        float a = 0.f, b = 0.f;
+        if (qraw) {
+            for (int h = 0; h < D.G; ++h) {
+                a += to_f(qraw[(hk * D.G + h) * D.d + i]);
+                b += to_f(qraw[(hk * D.G + h) * D.d + i + D.half]);
+            }
+        } else {
+            for (int tt = 0; tt < n_qtiles; ++tt) {
+                const float* p = D.qbar_part + ((int64_t)hk * D.qtiles_max + tt) * D.d;
+                a += p[i];
+                b += p[i + D.half];
+            }
+        }
+        const float2 cw = D.cs_W[i];
+        qb[i] = a * cw.x - b * cw.y;
+        qb[i + D.half] = b * cw.x + a * cw.y;
+    }
+    __syncthreads();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int per = (n_mem + n_split - 1) / n_split;
+    const int u0 = split * per;
+    const int u1 = min(n_mem, u0 + per);
+    uint64_t list = 0;
+    for (int jb = u0 + warp * 32; jb < u1; jb += 8 * 32) {
+        const int j = jb + lane;
+        uint64_t cand = 0;
+        if (j < u1) {
+            float acc = 0.f;
+            if (MODE == 0) {  // representative keys [r][d]
+                const T* p = (const T*)D.rep_keys + ((int64_t)hk * D.units_max + j) * D.r * D.d;
+                const int total = D.r * D.d;
+                constexpr int N = Vec16<T>::N;
+#pragma unroll 4
+                for (int e = 0; e < total; e += N) {
+                    float f[N];
+                    Vec16<T>::load(p + e, f);
+                    const int i0 = e % D.d;
+#pragma unroll
+                    for (int c = 0; c < N; ++c) acc += f[c] * qb[i0 + c];
+                }
+            } else {  // fp32 sum of the representative keys [d]
+                const float* p = D.repsum + ((int64_t)hk * D.units_max + j) * D.d;
+#pragma unroll 4
+                for (int e = 0; e < D.d; e += 4) {
+                    float f[4];
+                    Vec16<float>::load(p + e, f);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) acc += f[c] * qb[e + c];
+                }
+            }
+            const float s = acc * D.inv_sqrt_d;
+            D.uscore[(int64_t)hk * D.units_max + j] = s;
+            cand = make_key(s, (uint32_t)j);
+        }
+        if (do_select) list = warp_topk_insert(list, cand);
+    }
+    if (!do_select) return;
+    lists[warp][lane] = list;
+    __syncthreads();
+    if (warp == 0) {
+        uint64_t acc = lists[0][lane];
+        for (int w = 1; w < 8; ++w) acc = warp_merge_desc(acc, lists[w][lane]);
+        D.cand[((int64_t)hk * D.score_splits_max + split) * 32 + lane] = acc;
+    }
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) is_last = (atomicAdd(&D.counters[hk], 1u) == (unsigned)(n_split - 1));
+    __syncthreads();
+    if (!is_last) return;
+    __threadfence();
+    if (warp == 0) {
+        uint64_t acc = 0;
+        for (int s = 0; s < n_split; ++s)
+            acc = warp_merge_desc(acc, __ldcg(&D.cand[((int64_t)hk * D.score_splits_max + s) * 32 + lane]));
+        const int kk = min(D.topk, n_mem);
+        const uint32_t id = key_index(acc);
+        uint64_t sk = (lane < kk) ? (uint64_t)(0xffffffffu - id) : 0ull;
+        sk = warp_sort_desc(sk);
+        if (lane < D.topk) {
+            int o = -1;
+            if (lane < kk) {
+                o = (int)(0xffffffffu - (uint32_t)sk);
+                if (o < 0 || o >= n_mem) {
+                    set_err(D, ERR_SEL_RANGE);
+                    o = 0;
+                }
+            }
+            D.sel[hk * D.topk + lane] = o;
+        }
+        if (lane == 0) D.counters[hk] = 0u;
+    }
+}
+
+// Selection for top_k > 32: one CTA per kv head sorts every unit's composite key in shared
+// memory (bitonic network, descending), keeps the first min(k, n_mem) and sorts their ids.
+__global__ void __launch_bounds__(1024) k_topk_sort(Dev D, int n_mem, int p2) {
+    extern __shared__ uint64_t keys[];
+    const int hk = blockIdx.x;
+    for (int i = threadIdx.x; i < p2; i += blockDim.x)
+        keys[i] = i < n_mem ? make_key(D.uscore[(int64_t)hk * D.units_max + i], (uint32_t)i) : 0ull;
+    __syncthreads();
+    for (int k = 2; k <= p2; k <<= 1) {
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            for (int i = threadIdx.x; i < p2; i += blockDim.x) {
+                const int ixj = i ^ j;
+                if (ixj > i) {
+                    const bool desc = (i & k) == 0;
+                    const uint64_t a = keys[i], b = keys[ixj];
+                    if ((a < b) == desc) {
+                        keys[i] = b;
+                        keys[ixj] = a;
+                    }
+                }
+            }
+            __syncthreads();
+        }
+    }
+    const int kk = min(D.topk, n_mem);
+    // ids of the kept units, re-keyed so that a descending sort gives ascending ids
+    for (int i = threadIdx.x; i < p2; i += blockDim.x)
+        keys[i] = i < kk ? (uint64_t)(0xffffffffu - key_index(keys[i])) : 0ull;
+    __syncthreads();
+    for (int k = 2; k <= p2; k <<= 1) {
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            for (int i = threadIdx.x; i < p2; i += blockDim.x) {
+                const int ixj = i ^ j;
+                if (ixj > i) {
+                    const bool desc = (i & k) == 0;
+                    const uint64_t a = keys[i], b = keys[ixj];
+                    if ((a < b) == desc) {
+                        keys[i] = b;
+                        keys[ixj] = a;
+                    }
+                }
+            }
+            __syncthreads();
+        }
+    }
+    for (int i = threadIdx.x; i < D.topk; i += blockDim.x) {
+        int o = -1;
+        if (i < kk) {
+            o = (int)(0xffffffffu - (uint32_t)keys[i]);
+            if (o < 0 || o >= n_mem) {
+                set_err(D, ERR_SEL_RANGE);
+                o = 0;
+            }
+        }
+        D.sel[hk * D.topk + i] = o;
+    }
+}
+
+// ---- launchers ----------------------------------------------------------------------------
+
+template <typename T>
+cudaError_t launch_prep(const Dev& D, const void* q, int64_t c0, int n, cudaStream_t st) {
+    (void)c0;
+    if (n <= 0) return cudaSuccess;
+    const int tiles = (n + D.qt - 1) / D.qt;
+    const int threads = D.half * (256 / D.half);
+    dim3 grid(tiles, D.Hkv);
+    k_prep<T><<<grid, threads, (threads / D.half) * D.d * sizeof(float), st>>>(D, (const T*)q, n);
+    return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_select(const Dev& D, int score_mode, int n_mem, int n_qtiles, const void* qraw, cudaStream_t st,
+                          int* launches) {
+    *launches = 0;
+    if (n_mem <= 0 || D.topk <= 0) return cudaSuccess;
+    // about 256 units per CTA: one per lane of 8 warps
+    int n_split = (n_mem + 255) / 256;
+    if (n_split > D.score_splits_max) n_split = D.score_splits_max;
+    const int fast = D.topk <= 32;
+    dim3 grid(n_split, D.Hkv);
+    if (score_mode == 0)
+        k_score_topk<T, 0><<<grid, 256, 0, st>>>(D, n_mem, n_split, n_qtiles, (const T*)qraw, fast);
+    else
+        k_score_topk<T, 1><<<grid, 256, 0, st>>>(D, n_mem, n_split, n_qtiles, (const T*)qraw, fast);
+    ++*launches;
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess || fast) return err;
+    int p2 = 1;
+    while (p2 < n_mem) p2 <<= 1;  // n_mem <= 16384 (checked at create when top_k > 32)
+    const size_t smem = (size_t)p2 * sizeof(uint64_t);
+    if (smem > 48 * 1024) {
+        err = cudaFuncSetAttribute(k_topk_sort, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (err != cudaSuccess) return err;
+    }
+    k_topk_sort<<<D.Hkv, 1024, smem, st>>>(D, n_mem, p2);
+    ++*launches;
+    return cudaGetLastError();
+}
+
+template cudaError_t launch_prep<float>(const Dev&, const void*, int64_t, int, cudaStream_t);
+template cudaError_t launch_prep<__nv_bfloat16>(const Dev&, const void*, int64_t, int, cudaStream_t);
+template cudaError_t launch_select<float>(const Dev&, int, int, int, const void*, cudaStream_t, int*);
+template cudaError_t launch_select<__nv_bfloat16>(const Dev&, int, int, int, const void*, cudaStream_t, int*);
+
+}  // namespace infllm

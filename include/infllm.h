@@ -1,0 +1,163 @@
+/*
+ * infllm.h -- C ABI of a single-GPU (sm_100a) InfLLM block-memory sparse attention layer.
+ *
+ * One context holds one attention layer's context memory for one token stream.
+ * Tokens arrive in chunks (prefill) or one at a time (decode).  Distant tokens are
+ * grouped into fixed-size memory units, each represented by its top-n_reps
+ * representative tokens; every chunk (or decode step) scores all units, keeps
+ * the top_k per kv head, and attends with one exact softmax over the sink tokens,
+ * the selected units and the local window.
+ *
+ * Method sources (InfLLM pages):
+ *   - "InfLLM Guide: Training-Free Long-Context Memory Units", sections
+ *     "Core Innovation 1: Structured Context Partitioning" (sinks / memory units /
+ *     local window) and "Core Innovation 2: Semantic Representative Key Vectors &
+ *     Dynamic Top-K Selection", items 2 "Query-Aware Top-K Scoring and Loading"
+ *     (Score(M_j) = q . r_j / sqrt(d), top-k) and 3 "Exact Attention Evaluation"
+ *     (working context = sinks U top-k units U local window).
+ *   - "InfLLM: Training-Free Long-Context Extrapolation for LLMs with an Efficient
+ *     Context Memory" (atlas.scime.ai summary), "Approach": units represented by
+ *     their top-scoring representative tokens chosen by attention scores; lookup
+ *     at every step.  Its ablation rows ("Measured effects") keep lookup during both
+ *     encoding and decoding.
+ *   - OpenReview rebuttal (paperhub.cn), Q2 "Comparison to Well-trained Long LLM":
+ *     lookup during pre-filling is done per block (chunk).
+ *
+ * Conventions for every call:
+ *   - q, k, v and out are CALLER-OWNED DEVICE pointers, contiguous [n][heads][head_dim]
+ *     in the context's dtype (fp32 or bf16), 16-byte aligned.  q has n_q_heads heads,
+ *     k and v have n_kv_heads heads.  k and v are raw (before RoPE): the library applies
+ *     the position scheme.
+ *   - All work is enqueued on the CUDA stream given to infllm_create and runs
+ *     asynchronously; calls return after enqueueing.  Argument and state errors are
+ *     detected on the host and returned before anything is enqueued.
+ *   - The library owns every internal buffer (allocated by create, freed by destroy).
+ *   - A device-side consistency check that fails latches an error word; the next call
+ *     returns INFLLM_EDEVICE.  After any error, infllm_destroy stays valid.
+ *   - Calls on one context are not thread-safe.  Contexts are independent.
+ *
+ * Position scheme (RoPE, rotate-half pairing (i, i + d/2), theta_i = rope_base^(-2i/d)):
+ * a query at token t and a window key at token n interact at their true relative
+ * distance t - n; every sink and memory key sits at one clamped distance equal to
+ * `window` (query rotated by R(window), key unrotated).
+ */
+#ifndef INFLLM_H
+#define INFLLM_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    INFLLM_OK = 0,
+    INFLLM_EINVAL = 1,    /* bad argument or configuration */
+    INFLLM_ECAPACITY = 2, /* max_tokens or max_chunk would be exceeded */
+    INFLLM_ESTATE = 3,    /* call out of order (e.g. attend without a matching append) */
+    INFLLM_ECUDA = 4,     /* a CUDA runtime call failed (message in infllm_last_error) */
+    INFLLM_EDEVICE = 5    /* a device-side check failed in an earlier launch */
+} infllm_status;
+
+typedef enum { INFLLM_F32 = 0, INFLLM_BF16 = 1 } infllm_dtype;
+
+/* How a unit is scored against the chunk's queries.  Both are the same number in exact
+ * arithmetic (the dot product is linear in the key): REPS reads the n_reps representative
+ * keys of every unit; REPSUM reads one fp32 sum of them per unit (half the bytes). */
+typedef enum { INFLLM_SCORE_REPS = 0, INFLLM_SCORE_REPSUM = 1 } infllm_score_mode;
+
+typedef struct {
+    int32_t n_q_heads;   /* Hq; Hq % Hkv == 0; q head h uses kv head h / (Hq/Hkv) */
+    int32_t n_kv_heads;  /* Hkv */
+    int32_t head_dim;    /* d: 64 or 128 */
+    int32_t n_sink;      /* S >= 0: initial tokens always attended */
+    int32_t window;      /* W >= 1: local window length (and the clamped distance) */
+    int32_t unit_size;   /* U in [1, 1024]: tokens per memory unit */
+    int32_t n_reps;      /* r in [1, min(U, 32)]: representative tokens per unit */
+    int32_t top_k;       /* k >= 0: units attended per chunk and kv head */
+    int32_t max_chunk;   /* largest n accepted by append/attend */
+    int64_t max_tokens;  /* capacity of the token stream */
+    double rope_base;    /* RoPE base (> 1) */
+    int32_t dtype;       /* infllm_dtype of q/k/v/out */
+    int32_t score_mode;  /* infllm_score_mode */
+} infllm_config;
+
+typedef struct {
+    int64_t tokens;          /* tokens appended so far */
+    int64_t units_with_reps; /* units whose representatives have been chosen */
+    int32_t n_mem;           /* units eligible for the last attended chunk */
+    int32_t n_selected;      /* min(top_k, n_mem) of the last attended chunk */
+    int64_t window_base;     /* first window token of the last attended chunk */
+    int64_t active_tokens;   /* keys attended by the last query of the last attended chunk */
+    int64_t kernel_launches; /* kernels enqueued since create (or the last stats reset) */
+    /* filled when profiling is on (infllm_set_profiling), device times from CUDA events: */
+    double ms_append, ms_reps, ms_prep, ms_select, ms_attend, ms_decode;
+    int64_t n_append, n_reps, n_prep, n_select, n_attend, n_decode;
+} infllm_stats;
+
+typedef struct infllm_ctx infllm_ctx; /* opaque */
+
+/* Create a context: validates cfg, allocates every pool for max_tokens / max_chunk on
+ * the current CUDA device, and records `cuda_stream` (a cudaStream_t; NULL = legacy
+ * default stream) for all later work.  On failure *out is NULL. */
+infllm_status infllm_create(const infllm_config* cfg, void* cuda_stream, infllm_ctx** out);
+
+/* Free everything.  Waits for the context's pending work.  NULL is accepted. */
+infllm_status infllm_destroy(infllm_ctx* ctx);
+
+/* Start a new token stream in the same context (keeps allocations). */
+infllm_status infllm_reset(infllm_ctx* ctx);
+
+/* Append tokens [t, t+n) where t = tokens so far.  Before storing them, every unit that
+ * becomes eligible at t (its last token at least `window` tokens before t) gets its
+ * representatives, scored against the `window` queries that follow it.  q [n][Hq][d] is
+ * used for those later scores; k, v [n][Hkv][d] are stored.  n == 0 is a no-op.
+ * Errors: EINVAL (null pointer with n > 0, n > max_chunk, n < 0), ECAPACITY (tokens + n >
+ * max_tokens). */
+infllm_status infllm_append_chunk(infllm_ctx* ctx, const void* q, const void* k, const void* v,
+                                  int32_t n);
+
+/* Attention output of the chunk just appended (same n): score every eligible unit, keep
+ * the top min(top_k, n_mem) per kv head (ties to the lower unit index), then
+ * out[n][Hq][d] = softmax over sinks (n < S, causal) U selected units U window [B, t].
+ * Errors: ESTATE (no matching append), EINVAL. */
+infllm_status infllm_attend_chunk(infllm_ctx* ctx, const void* q, int32_t n, void* out);
+
+/* One decode step: append one token (q [1][Hq][d], k, v [1][Hkv][d]) and attend it
+ * (split-KV kernel with a log-sum-exp merge).  out [1][Hq][d]. */
+infllm_status infllm_decode_step(infllm_ctx* ctx, const void* q, const void* k, const void* v,
+                                 void* out);
+
+/* --- introspection (synchronize the context's stream) --------------------------------- */
+
+/* Selected units of the last attended chunk: host_sel [Hkv][top_k] int32, ascending unit
+ * ids, padded with -1. */
+infllm_status infllm_get_selection(infllm_ctx* ctx, int32_t* host_sel);
+
+/* Unit scores of the last attended chunk: host_scores [Hkv][n_mem] float32 (includes the
+ * 1/sqrt(d) factor).  *n_mem_out receives n_mem. */
+infllm_status infllm_get_unit_scores(infllm_ctx* ctx, float* host_scores, int32_t capacity,
+                                     int32_t* n_mem_out);
+
+/* Representatives of units [unit_begin, unit_begin + n_units): host_ids [Hkv][n_units][n_reps]
+ * int32, unit-local token offsets in ascending order.  The units must already have
+ * representatives (ESTATE otherwise). */
+infllm_status infllm_get_reps(infllm_ctx* ctx, int32_t unit_begin, int32_t n_units, int32_t* host_ids);
+
+infllm_status infllm_get_stats(infllm_ctx* ctx, infllm_stats* out);
+
+/* Record CUDA events around every kernel launch (adds host overhead) and accumulate the
+ * device times into infllm_stats.  Toggling clears the accumulated times and counts. */
+infllm_status infllm_set_profiling(infllm_ctx* ctx, int32_t enable);
+
+/* Human-readable description of the last error on this context ("" if none). */
+const char* infllm_last_error(infllm_ctx* ctx);
+
+/* Library version string. */
+const char* infllm_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* INFLLM_H */
