@@ -42,7 +42,7 @@ class Config(ctypes.Structure):
 class Stats(ctypes.Structure):
     _fields_ = [("tokens", ctypes.c_int64), ("units_with_reps", ctypes.c_int64), ("n_mem", ctypes.c_int32),
                 ("n_selected", ctypes.c_int32), ("window_base", ctypes.c_int64), ("active_tokens", ctypes.c_int64),
-                ("kernel_launches", ctypes.c_int64),
+                ("kernel_launches", ctypes.c_int64), ("attend_path", ctypes.c_int32), ("score_mode", ctypes.c_int32),
                 ("ms_append", ctypes.c_double), ("ms_reps", ctypes.c_double), ("ms_prep", ctypes.c_double),
                 ("ms_select", ctypes.c_double), ("ms_attend", ctypes.c_double), ("ms_decode", ctypes.c_double),
                 ("n_append", ctypes.c_int64), ("n_reps", ctypes.c_int64), ("n_prep", ctypes.c_int64),
@@ -66,6 +66,7 @@ SIGNATURES = {
     "infllm_get_reps": (ctypes.c_int, [_P, ctypes.c_int32, ctypes.c_int32, _P]),
     "infllm_get_stats": (ctypes.c_int, [_P, ctypes.POINTER(Stats)]),
     "infllm_set_profiling": (ctypes.c_int, [_P, ctypes.c_int32]),
+    "infllm_set_score_mode": (ctypes.c_int, [_P, ctypes.c_int32]),
     "infllm_last_error": (ctypes.c_char_p, [_P]),
     "infllm_version": (ctypes.c_char_p, []),
 }
@@ -204,6 +205,9 @@ class InfLLMLayer:
 
     def set_profiling(self, on: bool):
         self._check(self.L.infllm_set_profiling(self.h, 1 if on else 0), "infllm_set_profiling")
+
+    def set_score_mode(self, mode: str):
+        self._check(self.L.infllm_set_score_mode(self.h, SCORE_MODES[mode]), "infllm_set_score_mode")
 
     def reset(self):
         self._check(self.L.infllm_reset(self.h), "infllm_reset")

@@ -505,6 +505,8 @@ infllm_status infllm_get_stats(infllm_ctx* c, infllm_stats* o) {
     o->window_base = c->last_B;
     o->active_tokens = c->last_active;
     o->kernel_launches = c->launches;
+    o->attend_path = c->use_tc ? 1 : 0;
+    o->score_mode = c->cfg.score_mode;
     o->ms_append = c->ms[K_APPEND];
     o->ms_reps = c->ms[K_REPS];
     o->ms_prep = c->ms[K_PREP];
@@ -517,6 +519,13 @@ infllm_status infllm_get_stats(infllm_ctx* c, infllm_stats* o) {
     o->n_select = c->cnt[K_SELECT];
     o->n_attend = c->cnt[K_ATTEND];
     o->n_decode = c->cnt[K_DECODE];
+    return INFLLM_OK;
+}
+
+infllm_status infllm_set_score_mode(infllm_ctx* c, int32_t mode) {
+    if (!c) return INFLLM_EINVAL;
+    if (mode != INFLLM_SCORE_REPS && mode != INFLLM_SCORE_REPSUM) return fail(c, INFLLM_EINVAL, "unknown score_mode %d", mode);
+    c->cfg.score_mode = mode;
     return INFLLM_OK;
 }
 

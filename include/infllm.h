@@ -90,6 +90,8 @@ typedef struct {
     int64_t window_base;     /* first window token of the last attended chunk */
     int64_t active_tokens;   /* keys attended by the last query of the last attended chunk */
     int64_t kernel_launches; /* kernels enqueued since create (or the last stats reset) */
+    int32_t attend_path;     /* chunk attention kernel in use: 0 = CUDA-core fp32, 1 = tcgen05 tensor cores */
+    int32_t score_mode;      /* infllm_score_mode in use */
     /* filled when profiling is on (infllm_set_profiling), device times from CUDA events: */
     double ms_append, ms_reps, ms_prep, ms_select, ms_attend, ms_decode;
     int64_t n_append, n_reps, n_prep, n_select, n_attend, n_decode;
@@ -145,6 +147,10 @@ infllm_status infllm_get_unit_scores(infllm_ctx* ctx, float* host_scores, int32_
 infllm_status infllm_get_reps(infllm_ctx* ctx, int32_t unit_begin, int32_t n_units, int32_t* host_ids);
 
 infllm_status infllm_get_stats(infllm_ctx* ctx, infllm_stats* out);
+
+/* Switch the unit-scoring operand (infllm_score_mode) for later calls; both pools are always
+ * maintained, so this is valid at any point of a stream. */
+infllm_status infllm_set_score_mode(infllm_ctx* ctx, int32_t score_mode);
 
 /* Record CUDA events around every kernel launch (adds host overhead) and accumulate the
  * device times into infllm_stats.  Toggling clears the accumulated times and counts. */

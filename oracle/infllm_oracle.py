@@ -154,7 +154,7 @@ def unit_scores(q_chunk: np.ndarray, rep_keys: np.ndarray, window: int, base: fl
     """
     d = q_chunk.shape[-1]
     qr = rope(q_chunk, float(window), base)  # every memory token sits at distance W
-    return np.einsum("thd,jmd->j", qr, rep_keys) / math.sqrt(d)
+    return np.einsum("thd,jmd->j", qr, rep_keys, optimize=True) / math.sqrt(d)
 
 
 # --------------------------------------------------------------------------------------------
@@ -186,8 +186,8 @@ def attend_group(q: np.ndarray, c0: int, sel: Sequence[int], K: Callable, V: Cal
     q_win = rope(q, (t - B)[:, None], base)  # [n, G, d]
     k_win = rope(kk[n_far:], keys[n_far:] - B, base)
     logits = np.empty((n, G, len(keys)), dtype=np.float64)
-    logits[:, :, :n_far] = np.einsum("tgd,kd->tgk", q_far, kk[:n_far])
-    logits[:, :, n_far:] = np.einsum("tgd,kd->tgk", q_win, k_win)
+    logits[:, :, :n_far] = q_far @ kk[:n_far].T
+    logits[:, :, n_far:] = q_win @ k_win.T
     logits /= math.sqrt(d)
 
     valid = np.ones((n, len(keys)), dtype=bool)
@@ -198,7 +198,7 @@ def attend_group(q: np.ndarray, c0: int, sel: Sequence[int], K: Callable, V: Cal
     mx = logits.max(axis=-1, keepdims=True)
     p = np.exp(logits - mx)
     p /= p.sum(axis=-1, keepdims=True)
-    out = np.einsum("tgk,kd->tgd", p, vv)
+    out = p @ vv
     return out, p.sum(axis=-1), keys, valid
 
 
