@@ -67,6 +67,9 @@ SIGNATURES = {
     "infllm_get_stats": (ctypes.c_int, [_P, ctypes.POINTER(Stats)]),
     "infllm_set_profiling": (ctypes.c_int, [_P, ctypes.c_int32]),
     "infllm_set_score_mode": (ctypes.c_int, [_P, ctypes.c_int32]),
+    "infllm_select_units_noalloc": (ctypes.c_int, [_P, _P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                                    ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_double,
+                                                    ctypes.c_int32, ctypes.c_int32, _P, _P, _P]),
     "infllm_last_error": (ctypes.c_char_p, [_P]),
     "infllm_version": (ctypes.c_char_p, []),
 }

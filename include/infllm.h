@@ -159,6 +159,39 @@ infllm_status infllm_set_profiling(infllm_ctx* ctx, int32_t enable);
 /* Human-readable description of the last error on this context ("" if none). */
 const char* infllm_last_error(infllm_ctx* ctx);
 
+/* --- lookup without any device allocation --------------------------------------------- */
+
+/* Unit scores and top-k selection for ONE query token, allocating nothing on the device.
+ *
+ * For callers that cannot call cudaMalloc: code running while a framework captures its stream
+ * into a CUDA graph and forbids allocation there, engines whose memory planner owns every device
+ * byte, and real-time loops where an allocation could synchronise the device.  No context is
+ * needed.  The caller passes every input and output; the only other memory used is a fixed
+ * scratch area inside the library (a static device array of about 1 MiB that every GPU which
+ * loads the library holds until the process exits).  The InfLLM pages have no counterpart to this
+ * call: it computes what the lookup step of infllm_decode_step computes, from caller buffers.
+ *
+ *   rep_keys  device [n_kv_heads][n_units][n_reps][head_dim], `dtype`: raw keys of every unit's
+ *             representative tokens
+ *   q         device [n_q_heads][head_dim], `dtype`: the query token, before RoPE
+ *   sel       device out [n_kv_heads][top_k] int32: ascending ids of the top min(top_k, n_units)
+ *             units of each kv head (ties to the lower id), padded with -1
+ *   scores    device out or NULL, [n_kv_heads][n_units] float32: the unit scores (query at
+ *             relative distance `window`, factor 1/sqrt(head_dim) included)
+ * Limits of the scratch area: n_kv_heads <= 64 and n_units <= 16384; larger sizes return
+ * INFLLM_ECAPACITY before anything is enqueued.  Other bad arguments (top_k outside [1, 32],
+ * head_dim not 64/128, ...) return INFLLM_EINVAL.  Work is enqueued on `cuda_stream`, which must
+ * belong to the current device.
+ * The first call on a device looks up the device address of the scratch array (once per device,
+ * with that device current); make that first call before any stream capture.  Every call shares
+ * the scratch area and keeps the last call's contents (the call clears what must start at zero):
+ * calls whose work overlaps on the GPU -- on different streams or from different host threads --
+ * race and can return wrong results, so serialise them. */
+infllm_status infllm_select_units_noalloc(const void* rep_keys, const void* q, int32_t n_q_heads,
+                                          int32_t n_kv_heads, int32_t head_dim, int32_t n_units,
+                                          int32_t n_reps, int32_t window, double rope_base, int32_t dtype,
+                                          int32_t top_k, int32_t* sel, float* scores, void* cuda_stream);
+
 /* Library version string. */
 const char* infllm_version(void);
 
