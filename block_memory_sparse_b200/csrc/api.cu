@@ -5,6 +5,7 @@
 #include <math.h>
 #include <stdarg.h>
 #include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <algorithm>
@@ -286,6 +287,8 @@ void free_all(infllm_ctx* c) {
     for (void* p : c->allocs) cudaFree(p);
     c->allocs.clear();
     if (c->err_host) cudaFreeHost(c->err_host);
+    free(c->tmaps);
+    c->tmaps = nullptr;
     c->err_host = nullptr;
     for (auto& ev : c->events) {
         cudaEventDestroy(ev.a);
@@ -368,7 +371,11 @@ infllm_status create_impl(infllm_ctx* c) {
     CK(cudaHostAlloc((void**)&c->err_host, sizeof(int), cudaHostAllocMapped));
     *c->err_host = 0;
     CK(cudaHostGetDevicePointer((void**)&D.err, c->err_host, 0));
-    c->use_tc = attend_tc_supported(D) && g.dtype == INFLLM_BF16 && getenv("INFLLM_FORCE_SIMT") == nullptr;
+    c->use_tc = false;
+    if (g.dtype == INFLLM_BF16 && attend_tc_supported(D) && getenv("INFLLM_FORCE_SIMT") == nullptr) {
+        c->tmaps = malloc(tc_maps_size());
+        c->use_tc = c->tmaps && make_tc_maps(D, c->tmaps);
+    }
     infllm_status zs = zero_state(c);
     if (zs != INFLLM_OK) return zs;
     CK(cudaStreamSynchronize(c->stream));

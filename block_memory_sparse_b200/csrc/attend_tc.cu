@@ -1,9 +1,422 @@
-// Placeholder: tensor-core attention path (replaced by the tcgen05 kernel).
+// Exact attention of a prefill chunk over sinks U selected units U local window on the
+// 5th-generation tensor cores (tcgen05, bf16 operands, fp32 accumulators in TMEM).
+//
+// Method: "InfLLM Guide: Training-Free Long-Context Memory Units", "Core Innovation 2",
+// item 3 "Exact Attention Evaluation": one softmax over Sinks U (U_{m in top-k} M_m) U Local
+// Window; for a chunk this is a dense contraction per (query tile, KV tile).
+//
+// One CTA per (128 packed query rows, KV head): the rows are G q heads x 128/G consecutive
+// queries of one KV group, so every K/V tile is read once per group.  Warp roles:
+//   warp 0      TMA producer: the two rotated query tiles once, then K and V tiles (2 stages)
+//   warp 1      MMA issuer:   S_i = Q K_i^T into TMEM (double buffered), O += P_i V_i
+//   warps 2..5  softmax:      one thread per row; masks, online softmax with lazy rescale of
+//                             O (only when the running max grows by > 2^8), P_i to shared
+//                             memory in the swizzled K-major layout, final 1/l and store.
+// Sinks and memory tiles use R(W) q with raw keys; window tiles use R(t) q with R(n) k.
+#include <cuda.h>
+#include <math.h>
+
 #include "common.cuh"
 #include "kernels.h"
+#include "tc_ptx.cuh"
+
 namespace infllm {
-bool attend_tc_supported(const Dev&) { return false; }
-cudaError_t launch_attend_tc(const Dev&, int64_t, int, int, int64_t, void*, cudaStream_t, const void*) {
-    return cudaErrorNotSupported;
+
+struct TcMaps {
+    CUtensorMap kraw, krot, v, qm, qw;
+};
+
+namespace {
+
+constexpr int BM = 128;  // packed query rows per CTA
+constexpr int BN = 128;  // keys per tile
+constexpr int HD = 128;  // head dim handled here
+constexpr int NTHREADS = 192;
+constexpr uint32_t TILE = BN * HD * 2;  // bytes of one bf16 128 x 128 tile
+constexpr uint32_t HALF = TILE / 2;     // one 64-column swizzle block (128 rows x 128 B)
+constexpr int OFF_QM = 0;
+constexpr int OFF_QW = OFF_QM + (int)TILE;
+constexpr int OFF_K = OFF_QW + (int)TILE;      // 2 stages
+constexpr int OFF_V = OFF_K + 2 * (int)TILE;   // 2 stages
+constexpr int OFF_P = OFF_V + 2 * (int)TILE;
+constexpr int OFF_BAR = OFF_P + (int)TILE;
+constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;  // barriers + alignment slack
+constexpr uint32_t TMEM_COLS = 512;              // S0 [0,128) S1 [128,256) O [256,384)
+constexpr uint32_t TM_O = 256;
+constexpr float LOG2E = 1.4426950408889634f;
+constexpr float RESCALE_LOG2 = 8.0f;
+constexpr int ERR_TIMEOUT = 16;
+
+struct Bars {
+    uint64_t q, kfull[2], kempty[2], vfull[2], vempty[2], sfull[2], sfree[2], pfull, pvdone;
+    uint32_t tmem;
+    int abort;
+};
+
+struct TileInfo {
+    int kind;  // 0 sink, 1 memory unit, 2 window
+    int64_t y0;
+    int nv;
+};
+
+struct Plan {
+    int a, hk, kk, nst, tpu, nut, nwt, NT, S_eff;
+    int64_t t_hi, B, win_len;
+
+    __device__ TileInfo tile(const Dev& D, int i) const {
+        if (i < nst) return {0, (int64_t)i * BN, min(BN, S_eff - i * BN)};
+        i -= nst;
+        if (i < nut) {
+            const int u = i / tpu, part = i % tpu;
+            const int j = D.sel[hk * D.topk + u];
+            if (j < 0 || (int64_t)D.S + (int64_t)(j + 1) * D.U > B) {
+                set_err(D, ERR_SEL_RANGE);
+                return {1, 0, 0};
+            }
+            return {1, (int64_t)D.S + (int64_t)j * D.U + (int64_t)part * BN, min(BN, D.U - part * BN)};
+        }
+        i -= nut;
+        const int64_t rem = win_len - (int64_t)i * BN;
+        return {2, B + (int64_t)i * BN, (int)(rem < BN ? rem : BN)};
+    }
+};
+
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Bars* bars, const Dev& D) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!ptx::mbar_try_wait(bar, parity)) {
+        if (*(volatile int*)&bars->abort) return false;
+        if (clock64() - t0 > (1ll << 32)) {  // ~2 s: something is broken; give up cleanly
+            *(volatile int*)&bars->abort = 1;
+            set_err(D, ERR_TIMEOUT);
+            return false;
+        }
+    }
+    return true;
 }
+
+__device__ void producer(const TcMaps& maps, const Plan& P, const Dev& D, uint8_t* sm, Bars* bars) {
+    ptx::prefetch_tmap(&maps.qm);
+    ptx::prefetch_tmap(&maps.qw);
+    ptx::prefetch_tmap(&maps.kraw);
+    ptx::prefetch_tmap(&maps.krot);
+    ptx::prefetch_tmap(&maps.v);
+    const int y = P.a * BM;
+    ptx::mbar_expect_tx(&bars->q, 4 * HALF);
+    ptx::tma_load_3d(sm + OFF_QM, &maps.qm, &bars->q, 0, y, P.hk);
+    ptx::tma_load_3d(sm + OFF_QM + HALF, &maps.qm, &bars->q, 64, y, P.hk);
+    ptx::tma_load_3d(sm + OFF_QW, &maps.qw, &bars->q, 0, y, P.hk);
+    ptx::tma_load_3d(sm + OFF_QW + HALF, &maps.qw, &bars->q, 64, y, P.hk);
+    int issued = 0;
+    for (int i = 0; i < P.NT; ++i) {
+        const int s = i & 1;
+        const uint32_t use = (uint32_t)(i >> 1);
+        if (i >= 2 && !wait_bar(&bars->kempty[s], (use - 1) & 1, bars, D)) break;
+        const TileInfo T = P.tile(D, i);
+        const CUtensorMap* km = T.kind == 2 ? &maps.krot : &maps.kraw;
+        ptx::mbar_expect_tx(&bars->kfull[s], TILE);
+        ptx::tma_load_3d(sm + OFF_K + s * TILE, km, &bars->kfull[s], 0, (int)T.y0, P.hk);
+        ptx::tma_load_3d(sm + OFF_K + s * TILE + HALF, km, &bars->kfull[s], 64, (int)T.y0, P.hk);
+        if (i >= 2 && !wait_bar(&bars->vempty[s], (use - 1) & 1, bars, D)) {
+            issued = i + 1;
+            break;
+        }
+        ptx::mbar_expect_tx(&bars->vfull[s], TILE);
+        ptx::tma_load_3d(sm + OFF_V + s * TILE, &maps.v, &bars->vfull[s], 0, (int)T.y0, P.hk);
+        ptx::tma_load_3d(sm + OFF_V + s * TILE + HALF, &maps.v, &bars->vfull[s], 64, (int)T.y0, P.hk);
+        issued = i + 1;
+    }
+    if (*(volatile int*)&bars->abort) {
+        // let the copies already in flight land before the CTA exits (bounded)
+        for (int i = issued - 2 < 0 ? 0 : issued - 2; i < issued; ++i) {
+            ptx::mbar_wait(&bars->kfull[i & 1], (uint32_t)(i >> 1) & 1, 1ll << 28);
+            ptx::mbar_wait(&bars->vfull[i & 1], (uint32_t)(i >> 1) & 1, 1ll << 28);
+        }
+        ptx::mbar_wait(&bars->q, 0, 1ll << 28);
+    }
+}
+
+__device__ void mma_issuer(const Plan& P, const Dev& D, uint8_t* sm, Bars* bars, uint32_t tmem) {
+    constexpr uint32_t IDESC_QK = ptx::idesc_bf16_f32(BM, BN, false, false);
+    constexpr uint32_t IDESC_PV = ptx::idesc_bf16_f32(BM, HD, false, true);
+    if (!wait_bar(&bars->q, 0, bars, D)) return;
+    ptx::tc_fence_after();
+    const uint32_t qm = ptx::smem_u32(sm + OFF_QM), qw = ptx::smem_u32(sm + OFF_QW);
+    const uint32_t kb = ptx::smem_u32(sm + OFF_K), vb = ptx::smem_u32(sm + OFF_V), pb = ptx::smem_u32(sm + OFF_P);
+    for (int i = 0; i <= P.NT; ++i) {
+        if (i < P.NT) {
+            const int s = i & 1;
+            const uint32_t use = (uint32_t)(i >> 1);
+            if (!wait_bar(&bars->kfull[s], use & 1, bars, D)) return;
+            if (i >= 2 && !wait_bar(&bars->sfree[s], (use - 1) & 1, bars, D)) return;
+            ptx::tc_fence_after();
+            const uint32_t qa = P.tile(D, i).kind == 2 ? qw : qm;
+            const uint32_t ka = kb + s * TILE;
+#pragma unroll
+            for (int ks = 0; ks < HD / 16; ++ks) {
+                const uint32_t off = (uint32_t)(ks >> 2) * HALF + (uint32_t)(ks & 3) * 32;
+                ptx::mma_bf16(tmem + s * BN, ptx::sdesc_sw128(qa + off, 16, 1024), ptx::sdesc_sw128(ka + off, 16, 1024),
+                              IDESC_QK, ks > 0 ? 1u : 0u);
+            }
+            ptx::mma_commit(&bars->sfull[s]);
+            ptx::mma_commit(&bars->kempty[s]);
+        }
+        if (i >= 1) {
+            const int j = i - 1, sj = j & 1;
+            if (!wait_bar(&bars->pfull, (uint32_t)j & 1, bars, D)) return;
+            if (!wait_bar(&bars->vfull[sj], (uint32_t)(j >> 1) & 1, bars, D)) return;
+            ptx::tc_fence_after();
+            const uint32_t va = vb + sj * TILE;
+#pragma unroll
+            for (int ks = 0; ks < BN / 16; ++ks) {
+                const uint32_t aoff = (uint32_t)(ks >> 2) * HALF + (uint32_t)(ks & 3) * 32;
+                ptx::mma_bf16(tmem + TM_O, ptx::sdesc_sw128(pb + aoff, 16, 1024),
+                              ptx::sdesc_sw128(va + (uint32_t)ks * 2048, HALF, 1024), IDESC_PV,
+                              (j > 0 || ks > 0) ? 1u : 0u);
+            }
+            ptx::mma_commit(&bars->pvdone);
+            ptx::mma_commit(&bars->vempty[sj]);
+        }
+    }
+}
+
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Bars* bars, const Dev& D) {
+    const bool ok = wait_bar(bar, parity, bars, D);
+    return __all_sync(0xffffffffu, ok);
+}
+
+__device__ void softmax_role(const Plan& P, const Dev& D, uint8_t* sm, Bars* bars, uint32_t tmem, int64_t c0, int n,
+                             __nv_bfloat16* __restrict__ out, int warp, int lane) {
+    const int quarter = warp & 3;  // TMEM lanes this warp may access
+    const int row = quarter * 32 + lane;
+    const uint32_t tl_addr = tmem + ((uint32_t)(quarter * 32) << 16);
+    const int hg = row / D.qt, tl = P.a * D.qt + row % D.qt;
+    const bool valid = tl < n;
+    const int64_t t = c0 + tl;
+    const float sc = D.inv_sqrt_d * LOG2E;
+    float m_used = -INFINITY, l = 0.f;
+    float s[BN];
+    uint8_t* prow = sm + OFF_P + row * 128;
+    bool ok = true;
+    for (int i = 0; i < P.NT; ++i) {
+        const int b = i & 1;
+        if (!warp_wait(&bars->sfull[b], (uint32_t)(i >> 1) & 1, bars, D)) {
+            ok = false;
+            break;
+        }
+        ptx::tc_fence_after();
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) ptx::tmem_ld32(tl_addr + b * BN + c4 * 32, s + c4 * 32);
+        ptx::tmem_wait_ld();
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(&bars->sfree[b]);
+        const TileInfo T = P.tile(D, i);
+        float mt = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < BN; ++c) {
+            const bool keep = (c < T.nv) && (T.kind == 1 || T.y0 + c <= t);
+            s[c] = keep ? s[c] * sc : -INFINITY;
+            mt = fmaxf(mt, s[c]);
+        }
+        const bool need = mt > m_used + RESCALE_LOG2;
+        const float m_new = need ? mt : m_used;
+        if (i >= 1) {
+            if (!warp_wait(&bars->pvdone, (uint32_t)(i - 1) & 1, bars, D)) {
+                ok = false;
+                break;
+            }
+            ptx::tc_fence_after();
+            if (__any_sync(0xffffffffu, need)) {
+                const float f = need ? exp2f(m_used - m_new) : 1.f;
+                l *= f;
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    float o[32];
+                    ptx::tmem_ld32(tl_addr + TM_O + c4 * 32, o);
+                    ptx::tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) o[e] *= f;
+                    ptx::tmem_st32(tl_addr + TM_O + c4 * 32, o);
+                }
+                ptx::tmem_wait_st();
+            }
+        }
+        m_used = m_new;
+        const float ref = m_used == -INFINITY ? 0.f : m_used;
+        float rs = 0.f;
+#pragma unroll
+        for (int cb = 0; cb < 2; ++cb) {
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) {
+                uint32_t w[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int c = cb * 64 + ch * 8 + 2 * e;
+                    const float p0 = exp2f(s[c] - ref), p1 = exp2f(s[c + 1] - ref);
+                    rs += p0 + p1;
+                    __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
+                    w[e] = *reinterpret_cast<uint32_t*>(&h);
+                }
+                *reinterpret_cast<uint4*>(prow + cb * HALF + ((ch ^ (row & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+        }
+        l += rs;
+        ptx::fence_proxy_async_smem();
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(&bars->pfull);
+    }
+    if (!ok || !warp_wait(&bars->pvdone, (uint32_t)(P.NT - 1) & 1, bars, D)) return;
+    ptx::tc_fence_after();
+    const float inv = 1.f / l;
+    __nv_bfloat16* orow = out + ((int64_t)tl * D.Hq + P.hk * D.G + hg) * HD;
+#pragma unroll
+    for (int c4 = 0; c4 < 4; ++c4) {
+        float o[32];
+        ptx::tmem_ld32(tl_addr + TM_O + c4 * 32, o);
+        ptx::tmem_wait_ld();
+        if (valid) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                uint32_t w[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    __nv_bfloat162 h = __floats2bfloat162_rn(o[e * 8 + 2 * q] * inv, o[e * 8 + 2 * q + 1] * inv);
+                    w[q] = *reinterpret_cast<uint32_t*>(&h);
+                }
+                *reinterpret_cast<uint4*>(orow + c4 * 32 + e * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+        }
+    }
+}
+
+__global__ void __launch_bounds__(NTHREADS, 1)
+    k_attn_tc(const __grid_constant__ TcMaps maps, Dev D, int64_t c0, int n, int kk, int64_t B,
+              __nv_bfloat16* __restrict__ out) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    Bars* bars = reinterpret_cast<Bars*>(sm + OFF_BAR);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    Plan P;
+    P.a = gridDim.x - 1 - blockIdx.x;  // query tiles with more keys start first
+    P.hk = blockIdx.y;
+    P.kk = kk;
+    P.B = B;
+    {
+        const int last = min(n, (P.a + 1) * D.qt);
+        P.t_hi = c0 + last - 1;
+    }
+    P.S_eff = (int)(D.S < P.t_hi + 1 ? D.S : P.t_hi + 1);
+    P.nst = (P.S_eff + BN - 1) / BN;
+    P.tpu = (D.U + BN - 1) / BN;
+    P.nut = kk * P.tpu;
+    P.win_len = P.t_hi + 1 - B;
+    P.nwt = P.win_len > 0 ? (int)((P.win_len + BN - 1) / BN) : 0;
+    P.NT = P.nst + P.nut + P.nwt;
+
+    if (threadIdx.x == 0) {
+        ptx::mbar_init(&bars->q, 1);
+        for (int s = 0; s < 2; ++s) {
+            ptx::mbar_init(&bars->kfull[s], 1);
+            ptx::mbar_init(&bars->kempty[s], 1);
+            ptx::mbar_init(&bars->vfull[s], 1);
+            ptx::mbar_init(&bars->vempty[s], 1);
+            ptx::mbar_init(&bars->sfull[s], 1);
+            ptx::mbar_init(&bars->sfree[s], 128);
+        }
+        ptx::mbar_init(&bars->pfull, 128);
+        ptx::mbar_init(&bars->pvdone, 1);
+        bars->abort = 0;
+        ptx::mbar_fence_init();
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(&bars->tmem, TMEM_COLS);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = bars->tmem;
+
+    if (P.NT > 0) {
+        if (warp == 0) {
+            if (lane == 0) producer(maps, P, D, sm, bars);
+        } else if (warp == 1) {
+            if (lane == 0) mma_issuer(P, D, sm, bars, tmem);
+        } else {
+            softmax_role(P, D, sm, bars, tmem, c0, n, out, warp, lane);
+        }
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    if (warp == 1) ptx::tmem_dealloc(tmem, TMEM_COLS);
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = (EncodeTiledFn)p;
+    }
+    return fn;
+}
+
+// 3-D bf16 map over [dim2][dim1][HD] with box [1][128][64], 128-byte swizzle.
+bool encode_3d(CUtensorMap* m, void* base, uint64_t dim1, uint64_t dim2) {
+    EncodeTiledFn enc = get_encode();
+    if (!enc) return false;
+    cuuint64_t gdim[3] = {(cuuint64_t)HD, (cuuint64_t)dim1, (cuuint64_t)dim2};
+    cuuint64_t gstride[2] = {(cuuint64_t)HD * 2, (cuuint64_t)HD * 2 * dim1};
+    cuuint32_t box[3] = {64, (cuuint32_t)BN, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, gdim, gstride, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool attend_tc_supported(const Dev& D) {
+    if (D.d != HD || D.G > BM || BM % D.G != 0 || D.qt * D.G != BM) return false;
+    int dev = 0, major = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return false;
+    return major == 10 && get_encode() != nullptr;
+}
+
+size_t tc_maps_size() { return sizeof(TcMaps); }
+
+bool make_tc_maps(const Dev& D, void* out) {
+    TcMaps* m = reinterpret_cast<TcMaps*>(out);
+    return encode_3d(&m->kraw, D.Kraw, (uint64_t)D.T_max, (uint64_t)D.Hkv) &&
+           encode_3d(&m->krot, D.Krot, (uint64_t)D.T_max, (uint64_t)D.Hkv) &&
+           encode_3d(&m->v, D.V, (uint64_t)D.T_max, (uint64_t)D.Hkv) &&
+           encode_3d(&m->qm, D.Qm, (uint64_t)D.qrows_max, (uint64_t)D.Hkv) &&
+           encode_3d(&m->qw, D.Qw, (uint64_t)D.qrows_max, (uint64_t)D.Hkv);
+}
+
+cudaError_t launch_attend_tc(const Dev& D, int64_t c0, int n, int kk, int64_t B, void* out, cudaStream_t st,
+                             const void* tmaps) {
+    if (n <= 0) return cudaSuccess;
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(k_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    const int tiles = (n + D.qt - 1) / D.qt;
+    dim3 grid(tiles, D.Hkv);
+    k_attn_tc<<<grid, NTHREADS, SMEM_BYTES, st>>>(*reinterpret_cast<const TcMaps*>(tmaps), D, c0, n, kk, B,
+                                                  (__nv_bfloat16*)out);
+    return cudaGetLastError();
+}
+
 }  // namespace infllm

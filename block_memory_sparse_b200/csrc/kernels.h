@@ -33,6 +33,8 @@ cudaError_t launch_attend_simt(const Dev& D, int64_t c0, int n, int kk, int64_t 
 cudaError_t launch_attend_tc(const Dev& D, int64_t c0, int n, int kk, int64_t B, void* out, cudaStream_t st,
                              const void* tmaps);
 bool attend_tc_supported(const Dev& D);
+size_t tc_maps_size();
+bool make_tc_maps(const Dev& D, void* out);  // TMA descriptors of the stores and packed queries
 
 // Split-KV decode attention for one token with a log-sum-exp merge.
 template <typename T>

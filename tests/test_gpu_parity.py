@@ -45,6 +45,8 @@ def test_prefill_stream_matches_oracle(cuda_ok, name, score_mode):
         g = res[ci]
         nm = O.n_mem(c0, w.n_sink, w.window, w.unit_size)
         assert g["stats"]["n_mem"] == nm
+        # bf16 with d = 128 runs on the tcgen05 kernel; fp32 and d = 64 on the CUDA-core kernel
+        assert g["stats"]["attend_path"] == (1 if (w.dtype == "bf16" and w.head_dim == 128) else 0)
         # unit scores: oracle on the GPU's representatives
         if nm > 0 and w.top_k > 0:
             greps = glayer.reps(0, nm) if nm else None
@@ -167,3 +169,17 @@ def test_state_errors(cuda_ok):
     layer.reset()
     assert layer.stats()["tokens"] == 0
     layer.close()
+
+
+def test_tensor_core_path_matches_cuda_core_path(cuda_ok, monkeypatch):
+    """Same stream through the tcgen05 kernel and the fp32 CUDA-core kernel (forced at create)."""
+    w = synth.SMALL["small_g4"].replace(chunk=512, n_tokens=4096)
+    tc_layer, tc = run_prefill(w)
+    monkeypatch.setenv("INFLLM_FORCE_SIMT", "1")
+    simt_layer, simt = run_prefill(w)
+    assert tc[0]["stats"]["attend_path"] == 1 and simt[0]["stats"]["attend_path"] == 0
+    for ci in tc:
+        assert tc[ci]["sel"].tolist() == simt[ci]["sel"].tolist()
+        assert np.max(np.abs(tc[ci]["out"] - simt[ci]["out"])) <= 2e-2
+    tc_layer.close()
+    simt_layer.close()
