@@ -184,6 +184,8 @@ def run_ours(args, rank, world):
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
     w = synth.WORKLOADS[args.workload]
+    if args.tokens:
+        w = w.replace(n_tokens=min(args.tokens, w.n_tokens))
     P = peaks()
     chunks = synth.chunk_bounds(w)
     q_h, k_h, v_h = gen_full(w, torch, device)
@@ -419,6 +421,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--tokens", type=int, default=0, help="truncate the prefill stream (small profiling cases)")
     args = ap.parse_args()
     assert args.warmup >= 3 or args.impl == "reference", "at least 3 warm-up steps"
     rank, world, _ = dist_env()

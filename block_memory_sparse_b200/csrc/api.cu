@@ -321,7 +321,7 @@ infllm_status create_impl(infllm_ctx* c) {
     const int rpt = D.qt * D.G;
     D.qtiles_max = (g.max_chunk + D.qt - 1) / D.qt;
     D.qrows_max = (int64_t)D.qtiles_max * rpt;
-    D.score_splits_max = (int)std::min<int64_t>(1024, (D.units_max + 255) / 256 + 1);
+    D.score_splits_max = (int)((D.units_max + 3) / 4 + 1);  // up to 32 lanes per unit => 4 units per CTA
     const int SK = decode_split_keys(c->elt);
     D.dec_splits_max = (int)((std::min<int64_t>(g.n_sink, g.max_tokens) + (int64_t)g.top_k * g.unit_size +
                               (int64_t)g.window + g.unit_size + 1 + SK - 1) / SK) + 1;

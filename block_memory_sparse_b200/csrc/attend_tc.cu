@@ -40,7 +40,9 @@ constexpr int OFF_K = OFF_QW + (int)TILE;      // 2 stages
 constexpr int OFF_V = OFF_K + 2 * (int)TILE;   // 2 stages
 constexpr int OFF_P = OFF_V + 2 * (int)TILE;
 constexpr int OFF_BAR = OFF_P + (int)TILE;
-constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;  // barriers + alignment slack
+constexpr int OFF_SEL = OFF_BAR + 256;             // selected unit ids of this KV head
+constexpr int MAX_SEL = 256;
+constexpr int SMEM_BYTES = OFF_SEL + MAX_SEL * 4 + 1024;  // + alignment slack
 constexpr uint32_t TMEM_COLS = 512;              // S0 [0,128) S1 [128,256) O [256,384)
 constexpr uint32_t TM_O = 256;
 constexpr float LOG2E = 1.4426950408889634f;
@@ -62,17 +64,15 @@ struct TileInfo {
 struct Plan {
     int a, hk, kk, nst, tpu, nut, nwt, NT, S_eff;
     int64_t t_hi, B, win_len;
+    const int* sel;  // shared-memory copy; -1 marks an id that failed its range check
 
     __device__ TileInfo tile(const Dev& D, int i) const {
         if (i < nst) return {0, (int64_t)i * BN, min(BN, S_eff - i * BN)};
         i -= nst;
         if (i < nut) {
             const int u = i / tpu, part = i % tpu;
-            const int j = D.sel[hk * D.topk + u];
-            if (j < 0 || (int64_t)D.S + (int64_t)(j + 1) * D.U > B) {
-                set_err(D, ERR_SEL_RANGE);
-                return {1, 0, 0};
-            }
+            const int j = sel[u];
+            if (j < 0) return {1, 0, 0};
             return {1, (int64_t)D.S + (int64_t)j * D.U + (int64_t)part * BN, min(BN, D.U - part * BN)};
         }
         i -= nut;
@@ -185,6 +185,12 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Bars* 
     return __all_sync(0xffffffffu, ok);
 }
 
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 __device__ void softmax_role(const Plan& P, const Dev& D, uint8_t* sm, Bars* bars, uint32_t tmem, int64_t c0, int n,
                              __nv_bfloat16* __restrict__ out, int warp, int lane) {
     const int quarter = warp & 3;  // TMEM lanes this warp may access
@@ -193,8 +199,8 @@ __device__ void softmax_role(const Plan& P, const Dev& D, uint8_t* sm, Bars* bar
     const int hg = row / D.qt, tl = P.a * D.qt + row % D.qt;
     const bool valid = tl < n;
     const int64_t t = c0 + tl;
-    const float sc = D.inv_sqrt_d * LOG2E;
-    float m_used = -INFINITY, l = 0.f;
+    const float sc = D.inv_sqrt_d * LOG2E;  // logits in log2 units: s * sc
+    float m_used = -INFINITY, l = 0.f;      // running max (log2 units) and sum
     float s[BN];
     uint8_t* prow = sm + OFF_P + row * 128;
     bool ok = true;
@@ -210,14 +216,25 @@ __device__ void softmax_role(const Plan& P, const Dev& D, uint8_t* sm, Bars* bar
         ptx::tmem_wait_ld();
         ptx::tc_fence_before();
         ptx::mbar_arrive(&bars->sfree[b]);
+        // columns [0, lim) of this tile are attended by this row (causal limit on sinks and window)
         const TileInfo T = P.tile(D, i);
-        float mt = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < BN; ++c) {
-            const bool keep = (c < T.nv) && (T.kind == 1 || T.y0 + c <= t);
-            s[c] = keep ? s[c] * sc : -INFINITY;
-            mt = fmaxf(mt, s[c]);
+        int lim = T.nv;
+        if (T.kind != 1) {
+            const int64_t c = t - T.y0 + 1;
+            lim = c < (int64_t)lim ? (int)(c < 0 ? 0 : c) : lim;
         }
+        float mx = -INFINITY;
+        if (__all_sync(0xffffffffu, lim >= BN)) {
+#pragma unroll
+            for (int c = 0; c < BN; ++c) mx = fmaxf(mx, s[c]);
+        } else {
+#pragma unroll
+            for (int c = 0; c < BN; ++c) {
+                s[c] = c < lim ? s[c] : -INFINITY;
+                mx = fmaxf(mx, s[c]);
+            }
+        }
+        const float mt = mx * sc;
         const bool need = mt > m_used + RESCALE_LOG2;
         const float m_new = need ? mt : m_used;
         if (i >= 1) {
@@ -227,7 +244,7 @@ __device__ void softmax_role(const Plan& P, const Dev& D, uint8_t* sm, Bars* bar
             }
             ptx::tc_fence_after();
             if (__any_sync(0xffffffffu, need)) {
-                const float f = need ? exp2f(m_used - m_new) : 1.f;
+                const float f = need ? ex2(m_used - m_new) : 1.f;
                 l *= f;
 #pragma unroll
                 for (int c4 = 0; c4 < 4; ++c4) {
@@ -242,8 +259,8 @@ __device__ void softmax_role(const Plan& P, const Dev& D, uint8_t* sm, Bars* bar
             }
         }
         m_used = m_new;
-        const float ref = m_used == -INFINITY ? 0.f : m_used;
-        float rs = 0.f;
+        const float nref = m_used == -INFINITY ? 0.f : -m_used;
+        float rs0 = 0.f, rs1 = 0.f;
 #pragma unroll
         for (int cb = 0; cb < 2; ++cb) {
 #pragma unroll
@@ -252,15 +269,16 @@ __device__ void softmax_role(const Plan& P, const Dev& D, uint8_t* sm, Bars* bar
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int c = cb * 64 + ch * 8 + 2 * e;
-                    const float p0 = exp2f(s[c] - ref), p1 = exp2f(s[c + 1] - ref);
-                    rs += p0 + p1;
+                    const float p0 = ex2(fmaf(s[c], sc, nref)), p1 = ex2(fmaf(s[c + 1], sc, nref));
+                    rs0 += p0;
+                    rs1 += p1;
                     __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
                     w[e] = *reinterpret_cast<uint32_t*>(&h);
                 }
                 *reinterpret_cast<uint4*>(prow + cb * HALF + ((ch ^ (row & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
             }
         }
-        l += rs;
+        l += rs0 + rs1;
         ptx::fence_proxy_async_smem();
         ptx::tc_fence_before();
         ptx::mbar_arrive(&bars->pfull);
@@ -314,6 +332,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     P.nwt = P.win_len > 0 ? (int)((P.win_len + BN - 1) / BN) : 0;
     P.NT = P.nst + P.nut + P.nwt;
 
+    int* sel_s = reinterpret_cast<int*>(sm + OFF_SEL);
+    for (int u = threadIdx.x; u < kk; u += blockDim.x) {
+        int j = D.sel[P.hk * D.topk + u];
+        if (j < 0 || (int64_t)D.S + (int64_t)(j + 1) * D.U > B) {
+            set_err(D, ERR_SEL_RANGE);
+            j = -1;
+        }
+        sel_s[u] = j;
+    }
+    P.sel = sel_s;
     if (threadIdx.x == 0) {
         ptx::mbar_init(&bars->q, 1);
         for (int s = 0; s < 2; ++s) {
@@ -385,7 +413,7 @@ bool encode_3d(CUtensorMap* m, void* base, uint64_t dim1, uint64_t dim2) {
 }  // namespace
 
 bool attend_tc_supported(const Dev& D) {
-    if (D.d != HD || D.G > BM || BM % D.G != 0 || D.qt * D.G != BM) return false;
+    if (D.d != HD || D.G > BM || BM % D.G != 0 || D.qt * D.G != BM || D.topk > MAX_SEL) return false;
     int dev = 0, major = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return false;
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return false;

@@ -137,6 +137,16 @@ __device__ __forceinline__ float warp_max(float x) {
     return x;
 }
 
+// Two consecutive elements as floats (a 4-byte bf16x2 or 8-byte float2 load; 2-element aligned).
+__device__ __forceinline__ float2 ld2f(const __nv_bfloat16* p) {
+    return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
+}
+__device__ __forceinline__ float2 ld2f(const float* p) { return *reinterpret_cast<const float2*>(p); }
+__device__ __forceinline__ void st2f(__nv_bfloat16* p, float a, float b) {
+    *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(a, b);
+}
+__device__ __forceinline__ void st2f(float* p, float a, float b) { *reinterpret_cast<float2*>(p) = make_float2(a, b); }
+
 __host__ __device__ __forceinline__ int64_t n_mem_at(int64_t c0, int S, int W, int U) {
     int64_t x = c0 - (int64_t)W - (int64_t)S;
     return x > 0 ? x / U : 0;

@@ -45,50 +45,55 @@ __global__ void k_append(Dev D, const T* __restrict__ k, const T* __restrict__ v
 }
 
 // Y[b][hk] += sum over the chunk's tokens t in block b of sum_{h in group} R(t - s_b) q_{t,h}.
-// Grid (blocks touched, Hkv); blockDim a multiple of half.  Fixed-order reduction.
+// Grid (blocks touched, Hkv), 512 threads: thread = (pair couple pc: pairs 2pc, 2pc+1; token
+// group tg).  Fixed-order reduction over token groups, so results do not depend on scheduling.
 template <typename T>
-__global__ void k_ysum(Dev D, const T* __restrict__ q, int64_t c0, int n, int64_t b0) {
+__global__ void __launch_bounds__(512) k_ysum(Dev D, const T* __restrict__ q, int64_t c0, int n, int64_t b0) {
     extern __shared__ float red[];
     const int64_t b = b0 + blockIdx.x;
     const int hk = blockIdx.y;
     const int64_t sb = (int64_t)D.S + b * D.gblk;
     const int64_t lo = sb > c0 ? sb : c0;
     const int64_t hi = (sb + D.gblk) < (c0 + n) ? (sb + D.gblk) : (c0 + n);
-    const int i = threadIdx.x % D.half, tg = threadIdx.x / D.half, ntg = blockDim.x / D.half;
-    float a1 = 0.f, a2 = 0.f;
+    const int npc = D.half / 2;
+    const int pc = threadIdx.x % npc, tg = threadIdx.x / npc, ntg = blockDim.x / npc;
+    const int i = 2 * pc;
+    float a1x = 0.f, a1y = 0.f, a2x = 0.f, a2y = 0.f;
+#pragma unroll 2
     for (int64_t t = lo + tg; t < hi; t += ntg) {
-        const float2 cs = D.cs_rel[(t - sb) * D.half + i];
+        const float4 cs = *reinterpret_cast<const float4*>(D.cs_rel + (t - sb) * D.half + i);  // (c_i, s_i, c_i+1, s_i+1)
         const T* qr = q + ((t - c0) * D.Hq + (int64_t)hk * D.G) * D.d;
-        for (int h = 0; h < D.G; ++h) {
-            const float x1 = to_f(qr[h * D.d + i]), x2 = to_f(qr[h * D.d + i + D.half]);
-            a1 += x1 * cs.x - x2 * cs.y;
-            a2 += x2 * cs.x + x1 * cs.y;
+        float2 x1 = make_float2(0.f, 0.f), x2 = make_float2(0.f, 0.f);
+        for (int h = 0; h < D.G; ++h) {  // the rotation is linear: sum the group's heads first
+            const float2 u = ld2f(qr + h * D.d + i), w = ld2f(qr + h * D.d + i + D.half);
+            x1.x += u.x; x1.y += u.y;
+            x2.x += w.x; x2.y += w.y;
         }
+        a1x += x1.x * cs.x - x2.x * cs.y;
+        a2x += x2.x * cs.x + x1.x * cs.y;
+        a1y += x1.y * cs.z - x2.y * cs.w;
+        a2y += x2.y * cs.z + x1.y * cs.w;
     }
-    red[tg * D.d + i] = a1;
-    red[tg * D.d + i + D.half] = a2;
+    float* r = red + tg * D.d;
+    r[i] = a1x; r[i + 1] = a1y; r[i + D.half] = a2x; r[i + D.half + 1] = a2y;
     __syncthreads();
-    if (tg == 0) {
-        float s1 = 0.f, s2 = 0.f;
-        for (int g = 0; g < ntg; ++g) {
-            s1 += red[g * D.d + i];
-            s2 += red[g * D.d + i + D.half];
-        }
-        float* y = D.Y + (b * D.Hkv + hk) * D.d;
-        y[i] += s1;
-        y[i + D.half] += s2;
+    for (int j = threadIdx.x; j < D.d; j += blockDim.x) {
+        float acc = 0.f;
+        for (int g = 0; g < ntg; ++g) acc += red[g * D.d + j];
+        D.Y[(b * D.Hkv + hk) * D.d + j] += acc;
     }
 }
 
-// Representatives of units [j0, j0 + gridDim.x) for kv head blockIdx.y.
+// Representatives of units [j0, j0 + gridDim.x) for kv head blockIdx.y, 256 threads.
 //   Qt = sum_{i=e}^{e+W-1} sum_h R(i - e) q_{i,h}  (from the block sums, e = unit end)
 //   rho_m = <R(e - m) Qt, k_m> / sqrt(d)  ==  sum_i sum_h <R(i) q_{i,h}, R(m) k_m> / sqrt(d)
 // then the top r by (rho desc, m asc), stored ascending, plus the raw rep keys and their sum.
 template <typename T>
-__global__ void k_reps(Dev D, int64_t j0) {
+__global__ void __launch_bounds__(256) k_reps(Dev D, int64_t j0) {
     extern __shared__ float sm[];
-    float* Qt = sm;          // [d]
-    float* rho = sm + D.d;   // [U]
+    float* Qt = sm;                 // [d]
+    float* rho = sm + D.d;          // [U]
+    float* part = rho + D.U;        // [4][d] partial window sums
     __shared__ int ids[32];
     const int64_t j = j0 + blockIdx.x;
     const int hk = blockIdx.y;
@@ -96,32 +101,50 @@ __global__ void k_reps(Dev D, int64_t j0) {
     const int64_t m0 = e - D.U;
     const int64_t be = (e - D.S) / D.gblk;
     const int nb = D.W / D.gblk;
-    for (int i = threadIdx.x; i < D.half; i += blockDim.x) {
+    {
+        const int i = threadIdx.x % D.half, pg = threadIdx.x / D.half, npg = blockDim.x / D.half;
         float a1 = 0.f, a2 = 0.f;
-        for (int p = 0; p < nb; ++p) {
+        for (int p = pg; p < nb; p += npg) {
             const float* y = D.Y + ((be + p) * D.Hkv + hk) * D.d;
             const float2 cs = D.cs_rel[(int64_t)p * D.gblk * D.half + i];
             const float y1 = y[i], y2 = y[i + D.half];
             a1 += y1 * cs.x - y2 * cs.y;
             a2 += y2 * cs.x + y1 * cs.y;
         }
-        Qt[i] = a1;
-        Qt[i + D.half] = a2;
+        part[pg * D.d + i] = a1;
+        part[pg * D.d + i + D.half] = a2;
+        __syncthreads();
+        for (int x = threadIdx.x; x < D.d; x += blockDim.x) {
+            float acc = 0.f;
+            for (int g = 0; g < npg; ++g) acc += part[g * D.d + x];
+            Qt[x] = acc;
+        }
     }
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
     const T* K = (const T*)D.Kraw + ((int64_t)hk * D.T_max + m0) * D.d;
-    for (int m = warp; m < D.U; m += nw) {
-        const int dist = D.U - m;  // e - (m0 + m)
-        float part = 0.f;
+    constexpr int UNR = 4;
+    for (int mb = warp * UNR; mb < D.U; mb += nw * UNR) {
+        float acc[UNR];
+#pragma unroll
+        for (int u = 0; u < UNR; ++u) acc[u] = 0.f;
         for (int i = lane; i < D.half; i += 32) {
-            const float2 cs = D.cs_rel[(int64_t)dist * D.half + i];
             const float q1 = Qt[i], q2 = Qt[i + D.half];
-            const float r1 = q1 * cs.x - q2 * cs.y, r2 = q2 * cs.x + q1 * cs.y;
-            part += r1 * to_f(K[(int64_t)m * D.d + i]) + r2 * to_f(K[(int64_t)m * D.d + i + D.half]);
+#pragma unroll
+            for (int u = 0; u < UNR; ++u) {
+                const int m = mb + u;
+                if (m < D.U) {
+                    const float2 cs = D.cs_rel[(int64_t)(D.U - m) * D.half + i];  // distance e - (m0 + m)
+                    const float r1 = q1 * cs.x - q2 * cs.y, r2 = q2 * cs.x + q1 * cs.y;
+                    acc[u] += r1 * to_f(K[(int64_t)m * D.d + i]) + r2 * to_f(K[(int64_t)m * D.d + i + D.half]);
+                }
+            }
         }
-        part = warp_sum(part);
-        if (lane == 0) rho[m] = part * D.inv_sqrt_d;
+#pragma unroll
+        for (int u = 0; u < UNR; ++u) {
+            const float v = warp_sum(acc[u]);
+            if (lane == 0 && mb + u < D.U) rho[mb + u] = v * D.inv_sqrt_d;
+        }
     }
     __syncthreads();
     if (warp == 0) {
@@ -184,9 +207,9 @@ cudaError_t launch_ysum(const Dev& D, const void* q, int64_t c0, int n, cudaStre
     const int64_t hi = c0 + n;
     if (hi <= lo) return cudaSuccess;
     const int64_t b0 = (lo - D.S) / D.gblk, b1 = (hi - 1 - D.S) / D.gblk;
-    const int threads = D.half * (256 / D.half);
+    const int threads = 512;  // (half / 2) pair couples x token groups
     dim3 grid((unsigned)(b1 - b0 + 1), D.Hkv);
-    k_ysum<T><<<grid, threads, (threads / D.half) * D.d * sizeof(float), st>>>(D, (const T*)q, c0, n, b0);
+    k_ysum<T><<<grid, threads, (threads / (D.half / 2)) * D.d * sizeof(float), st>>>(D, (const T*)q, c0, n, b0);
     ++*launches;
     return cudaGetLastError();
 }
@@ -195,7 +218,7 @@ template <typename T>
 cudaError_t launch_reps(const Dev& D, int64_t j0, int64_t j1, cudaStream_t st) {
     if (j1 <= j0) return cudaSuccess;
     dim3 grid((unsigned)(j1 - j0), D.Hkv);
-    k_reps<T><<<grid, 128, (D.d + D.U) * sizeof(float), st>>>(D, j0);
+    k_reps<T><<<grid, 256, (D.d + D.U + (256 / D.half) * D.d) * sizeof(float), st>>>(D, j0);
     return cudaGetLastError();
 }
 

@@ -14,50 +14,48 @@
 
 namespace infllm {
 
-// Rotated, packed queries of the chunk.  Grid (tiles, Hkv).  Tile a holds queries
-// [a*qt, a*qt + qt); row r of a tile is (head hg = r / qt, query a*qt + r % qt).
-// Also writes each tile's raw query sum over its rows (fixed-order reduction).
+// Rotated, packed queries of the chunk.  Grid (tiles, Hkv), 512 threads.  Tile a holds
+// queries [a*qt, a*qt + qt); row r of a tile is (head hg = r / qt, query a*qt + r % qt).
+// Thread = (pair couple pc: pairs 2pc, 2pc+1; row group).  Also writes each tile's raw query
+// sum over its rows (fixed-order reduction).
 template <typename T>
-__global__ void k_prep(Dev D, const T* __restrict__ q, int n) {
+__global__ void __launch_bounds__(512) k_prep(Dev D, const T* __restrict__ q, int n) {
     extern __shared__ float red[];
     const int a = blockIdx.x, hk = blockIdx.y;
     const int rows = D.qt * D.G;
-    const int i = threadIdx.x % D.half, rg = threadIdx.x / D.half, nrg = blockDim.x / D.half;
-    const float2 cw = D.cs_W[i];
+    const int npc = D.half / 2;
+    const int pc = threadIdx.x % npc, rg = threadIdx.x / npc, nrg = blockDim.x / npc;
+    const int i = 2 * pc;
+    const float4 cw = *reinterpret_cast<const float4*>(D.cs_W + i);
     T* Qm = (T*)D.Qm + ((int64_t)hk * D.qrows_max + (int64_t)a * rows) * D.d;
     T* Qw = (T*)D.Qw + ((int64_t)hk * D.qrows_max + (int64_t)a * rows) * D.d;
-    float s1 = 0.f, s2 = 0.f;
+    float s1x = 0.f, s1y = 0.f, s2x = 0.f, s2y = 0.f;
+#pragma unroll 4
     for (int r = rg; r < rows; r += nrg) {
         const int hg = r / D.qt, tl = a * D.qt + r % D.qt;
-        float m1 = 0.f, m2 = 0.f, w1 = 0.f, w2 = 0.f;
+        float2 x1 = make_float2(0.f, 0.f), x2 = make_float2(0.f, 0.f);
+        float4 ct = make_float4(1.f, 0.f, 1.f, 0.f);
         if (tl < n) {
             const T* src = q + ((int64_t)tl * D.Hq + hk * D.G + hg) * D.d;
-            const float x1 = to_f(src[i]), x2 = to_f(src[i + D.half]);
-            s1 += x1;
-            s2 += x2;
-            m1 = x1 * cw.x - x2 * cw.y;
-            m2 = x2 * cw.x + x1 * cw.y;
-            const float2 ct = D.cs_chunk[(int64_t)tl * D.half + i];
-            w1 = x1 * ct.x - x2 * ct.y;
-            w2 = x2 * ct.x + x1 * ct.y;
+            x1 = ld2f(src + i);
+            x2 = ld2f(src + i + D.half);
+            ct = *reinterpret_cast<const float4*>(D.cs_chunk + (int64_t)tl * D.half + i);
         }
-        Qm[(int64_t)r * D.d + i] = from_f<T>(m1);
-        Qm[(int64_t)r * D.d + i + D.half] = from_f<T>(m2);
-        Qw[(int64_t)r * D.d + i] = from_f<T>(w1);
-        Qw[(int64_t)r * D.d + i + D.half] = from_f<T>(w2);
+        s1x += x1.x; s1y += x1.y; s2x += x2.x; s2y += x2.y;
+        T* dm = Qm + (int64_t)r * D.d;
+        T* dw = Qw + (int64_t)r * D.d;
+        st2f(dm + i, x1.x * cw.x - x2.x * cw.y, x1.y * cw.z - x2.y * cw.w);
+        st2f(dm + i + D.half, x2.x * cw.x + x1.x * cw.y, x2.y * cw.z + x1.y * cw.w);
+        st2f(dw + i, x1.x * ct.x - x2.x * ct.y, x1.y * ct.z - x2.y * ct.w);
+        st2f(dw + i + D.half, x2.x * ct.x + x1.x * ct.y, x2.y * ct.z + x1.y * ct.w);
     }
-    red[rg * D.d + i] = s1;
-    red[rg * D.d + i + D.half] = s2;
+    float* rr = red + rg * D.d;
+    rr[i] = s1x; rr[i + 1] = s1y; rr[i + D.half] = s2x; rr[i + D.half + 1] = s2y;
     __syncthreads();
-    if (rg == 0) {
-        float a1 = 0.f, a2 = 0.f;
-        for (int g = 0; g < nrg; ++g) {
-            a1 += red[g * D.d + i];
-            a2 += red[g * D.d + i + D.half];
-        }
-        float* p = D.qbar_part + ((int64_t)hk * D.qtiles_max + a) * D.d;
-        p[i] = a1;
-        p[i + D.half] = a2;
+    for (int j = threadIdx.x; j < D.d; j += blockDim.x) {
+        float acc = 0.f;
+        for (int g = 0; g < nrg; ++g) acc += red[g * D.d + j];
+        D.qbar_part[((int64_t)hk * D.qtiles_max + a) * D.d + j] = acc;
     }
 }
 
@@ -84,14 +82,15 @@ template <> struct Vec16<float> {
     }
 };
 
-// Grid (n_split, Hkv), 256 threads.  Lane-per-unit scoring (each lane streams one unit's
-// operand in 16-byte loads), warp top-32 lists, CTA merge, then the last CTA of each kv head
-// merges every CTA's list (arrival counter, no waiting) and writes the selection.
-template <typename T, int MODE>
-__global__ void __launch_bounds__(256) k_score_topk(Dev D, int n_mem, int n_split, int n_qtiles, const T* qraw,
+// Grid (n_split, Hkv), 128 threads.  Each unit is scored by a group of LPU lanes that split
+// its operand (16-byte loads, all in flight), reduced inside the group; per = 128 / LPU units
+// per CTA.  Warp top-32 lists, CTA merge, then the last CTA of each kv head (arrival counter,
+// no waiting) merges every CTA's list with all four warps and writes the selection.
+template <typename T, int MODE, int LPU>
+__global__ void __launch_bounds__(128) k_score_topk(Dev D, int n_mem, int n_split, int n_qtiles, const T* qraw,
                                                     int do_select) {
     __shared__ float qb[128];
-    __shared__ uint64_t lists[8][32];
+    __shared__ uint64_t lists[4][32];
     __shared__ int is_last;
     const int split = blockIdx.x, hk = blockIdx.y;
     for (int i = threadIdx.x; i < D.half; i += blockDim.x) {
@@ -114,50 +113,50 @@ __global__ void __launch_bounds__(256) k_score_topk(Dev D, int n_mem, int n_spli
     }
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int per = (n_mem + n_split - 1) / n_split;
-    const int u0 = split * per;
-    const int u1 = min(n_mem, u0 + per);
-    uint64_t list = 0;
-    for (int jb = u0 + warp * 32; jb < u1; jb += 8 * 32) {
-        const int j = jb + lane;
-        uint64_t cand = 0;
-        if (j < u1) {
-            float acc = 0.f;
-            if (MODE == 0) {  // representative keys [r][d]
-                const T* p = (const T*)D.rep_keys + ((int64_t)hk * D.units_max + j) * D.r * D.d;
-                const int total = D.r * D.d;
-                constexpr int N = Vec16<T>::N;
-#pragma unroll 4
-                for (int e = 0; e < total; e += N) {
-                    float f[N];
-                    Vec16<T>::load(p + e, f);
-                    const int i0 = e % D.d;
+    constexpr int PER = 128 / LPU;       // units per CTA
+    constexpr int UPW = 32 / LPU;        // units per warp
+    const int j = split * PER + warp * UPW + lane / LPU;
+    const int sub = lane % LPU;
+    uint64_t cand = 0;
+    float acc = 0.f;
+    if (j < n_mem) {
+        if (MODE == 0) {  // representative keys [r][d]
+            const T* p = (const T*)D.rep_keys + ((int64_t)hk * D.units_max + j) * D.r * D.d;
+            constexpr int N = Vec16<T>::N;
+            const int total = D.r * D.d;
+#pragma unroll 8
+            for (int e = sub * N; e < total; e += LPU * N) {
+                float f[N];
+                Vec16<T>::load(p + e, f);
+                const int i0 = e % D.d;
 #pragma unroll
-                    for (int c = 0; c < N; ++c) acc += f[c] * qb[i0 + c];
-                }
-            } else {  // fp32 sum of the representative keys [d]
-                const float* p = D.repsum + ((int64_t)hk * D.units_max + j) * D.d;
-#pragma unroll 4
-                for (int e = 0; e < D.d; e += 4) {
-                    float f[4];
-                    Vec16<float>::load(p + e, f);
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) acc += f[c] * qb[e + c];
-                }
+                for (int c = 0; c < N; ++c) acc += f[c] * qb[i0 + c];
             }
-            const float s = acc * D.inv_sqrt_d;
-            D.uscore[(int64_t)hk * D.units_max + j] = s;
-            cand = make_key(s, (uint32_t)j);
+        } else {  // fp32 sum of the representative keys [d]
+            const float* p = D.repsum + ((int64_t)hk * D.units_max + j) * D.d;
+#pragma unroll 8
+            for (int e = sub * 4; e < D.d; e += LPU * 4) {
+                float f[4];
+                Vec16<float>::load(p + e, f);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) acc += f[c] * qb[e + c];
+            }
         }
-        if (do_select) list = warp_topk_insert(list, cand);
+    }
+#pragma unroll
+    for (int m = LPU / 2; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
+    if (j < n_mem && sub == 0) {
+        const float s = acc * D.inv_sqrt_d;
+        D.uscore[(int64_t)hk * D.units_max + j] = s;
+        cand = make_key(s, (uint32_t)j);
     }
     if (!do_select) return;
-    lists[warp][lane] = list;
+    lists[warp][lane] = warp_sort_desc(cand);
     __syncthreads();
     if (warp == 0) {
-        uint64_t acc = lists[0][lane];
-        for (int w = 1; w < 8; ++w) acc = warp_merge_desc(acc, lists[w][lane]);
-        D.cand[((int64_t)hk * D.score_splits_max + split) * 32 + lane] = acc;
+        uint64_t m = lists[0][lane];
+        for (int w = 1; w < 4; ++w) m = warp_merge_desc(m, lists[w][lane]);
+        D.cand[((int64_t)hk * D.score_splits_max + split) * 32 + lane] = m;
     }
     __threadfence();
     __syncthreads();
@@ -165,12 +164,18 @@ __global__ void __launch_bounds__(256) k_score_topk(Dev D, int n_mem, int n_spli
     __syncthreads();
     if (!is_last) return;
     __threadfence();
+    {   // each warp merges a strided quarter of the lists, then warp 0 merges the four
+        uint64_t m = 0;
+        for (int s = warp; s < n_split; s += 4)
+            m = warp_merge_desc(m, __ldcg(&D.cand[((int64_t)hk * D.score_splits_max + s) * 32 + lane]));
+        lists[warp][lane] = m;
+    }
+    __syncthreads();
     if (warp == 0) {
-        uint64_t acc = 0;
-        for (int s = 0; s < n_split; ++s)
-            acc = warp_merge_desc(acc, __ldcg(&D.cand[((int64_t)hk * D.score_splits_max + s) * 32 + lane]));
+        uint64_t m = lists[0][lane];
+        for (int w = 1; w < 4; ++w) m = warp_merge_desc(m, lists[w][lane]);
         const int kk = min(D.topk, n_mem);
-        const uint32_t id = key_index(acc);
+        const uint32_t id = key_index(m);
         uint64_t sk = (lane < kk) ? (uint64_t)(0xffffffffu - id) : 0ull;
         sk = warp_sort_desc(sk);
         if (lane < D.topk) {
@@ -253,10 +258,30 @@ cudaError_t launch_prep(const Dev& D, const void* q, int64_t c0, int n, cudaStre
     (void)c0;
     if (n <= 0) return cudaSuccess;
     const int tiles = (n + D.qt - 1) / D.qt;
-    const int threads = D.half * (256 / D.half);
+    const int threads = 512;
     dim3 grid(tiles, D.Hkv);
-    k_prep<T><<<grid, threads, (threads / D.half) * D.d * sizeof(float), st>>>(D, (const T*)q, n);
+    k_prep<T><<<grid, threads, (threads / (D.half / 2)) * D.d * sizeof(float), st>>>(D, (const T*)q, n);
     return cudaGetLastError();
+}
+
+// Lanes per unit: the fewest that still give about two CTAs per SM (296 CTAs).
+int score_lanes_per_unit(int n_mem, int Hkv) {
+    int lpu = 1;
+    while (lpu < 32 && (int64_t)((n_mem + 128 / lpu - 1) / (128 / lpu)) * Hkv < 296) lpu *= 2;
+    return lpu;
+}
+
+template <typename T, int MODE>
+static void launch_score(const Dev& D, int lpu, dim3 grid, int n_mem, int n_split, int n_qtiles, const T* qraw,
+                         int do_select, cudaStream_t st) {
+    switch (lpu) {
+        case 1: k_score_topk<T, MODE, 1><<<grid, 128, 0, st>>>(D, n_mem, n_split, n_qtiles, qraw, do_select); break;
+        case 2: k_score_topk<T, MODE, 2><<<grid, 128, 0, st>>>(D, n_mem, n_split, n_qtiles, qraw, do_select); break;
+        case 4: k_score_topk<T, MODE, 4><<<grid, 128, 0, st>>>(D, n_mem, n_split, n_qtiles, qraw, do_select); break;
+        case 8: k_score_topk<T, MODE, 8><<<grid, 128, 0, st>>>(D, n_mem, n_split, n_qtiles, qraw, do_select); break;
+        case 16: k_score_topk<T, MODE, 16><<<grid, 128, 0, st>>>(D, n_mem, n_split, n_qtiles, qraw, do_select); break;
+        default: k_score_topk<T, MODE, 32><<<grid, 128, 0, st>>>(D, n_mem, n_split, n_qtiles, qraw, do_select); break;
+    }
 }
 
 template <typename T>
@@ -264,15 +289,16 @@ cudaError_t launch_select(const Dev& D, int score_mode, int n_mem, int n_qtiles,
                           int* launches) {
     *launches = 0;
     if (n_mem <= 0 || D.topk <= 0) return cudaSuccess;
-    // about 256 units per CTA: one per lane of 8 warps
-    int n_split = (n_mem + 255) / 256;
-    if (n_split > D.score_splits_max) n_split = D.score_splits_max;
+    const int lpu = score_lanes_per_unit(n_mem, D.Hkv);
+    const int per = 128 / lpu;
+    const int n_split = (n_mem + per - 1) / per;
+    if (n_split > D.score_splits_max) return cudaErrorInvalidValue;
     const int fast = D.topk <= 32;
     dim3 grid(n_split, D.Hkv);
     if (score_mode == 0)
-        k_score_topk<T, 0><<<grid, 256, 0, st>>>(D, n_mem, n_split, n_qtiles, (const T*)qraw, fast);
+        launch_score<T, 0>(D, lpu, grid, n_mem, n_split, n_qtiles, (const T*)qraw, fast, st);
     else
-        k_score_topk<T, 1><<<grid, 256, 0, st>>>(D, n_mem, n_split, n_qtiles, (const T*)qraw, fast);
+        launch_score<T, 1>(D, lpu, grid, n_mem, n_split, n_qtiles, (const T*)qraw, fast, st);
     ++*launches;
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess || fast) return err;
