@@ -11,7 +11,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 OUT = os.path.join(HERE, "libinfllm.so")
 OBJ = os.path.join(HERE, "_build")
-SOURCES = ["api.cu", "memory.cu", "select.cu", "attend_simt.cu", "attend_tc.cu", "decode.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "memory.cu", "select.cu", "attend_simt.cu", "attend_tc.cu", "decode.cu", "decode_tc.cu", "noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
          "-I", os.path.join(ROOT, "include")]

@@ -243,8 +243,30 @@ infllm_status attend_impl(infllm_ctx* c, const void* q, int32_t n, void* out) {
 
 template <typename T>
 infllm_status decode_impl(infllm_ctx* c, const void* q, const void* k, const void* v, void* out) {
-    infllm_status s = append_impl<T>(c, q, k, v, 1);
-    if (s != INFLLM_OK) return s;
+    infllm_status s;
+    if (sizeof(T) == 2 && c->use_tc && decode_tc_supported(c->D) && c->D.G <= 8) {
+        const Dev& D = c->D;
+        const int64_t t = c->tokens;
+        const int64_t target = n_mem_at(t, D.S, D.W, D.U);
+        if (target > c->units_done) {
+            Prof p(c, K_REPS);
+            CK(launch_reps<T>(D, c->units_done, target, c->stream));
+            p.done();
+            c->launches += 1;
+            c->units_done = target;
+        }
+        Prof p(c, K_APPEND);
+        CK(launch_decode_append(D, q, k, v, t, c->stream));
+        p.done();
+        c->launches += 1;
+        c->tokens = t + 1;
+        c->pending = true;
+        c->pending_n = 1;
+        c->pending_c0 = t;
+    } else {
+        s = append_impl<T>(c, q, k, v, 1);
+        if (s != INFLLM_OK) return s;
+    }
     const Dev& D = c->D;
     const int64_t t = c->pending_c0;
     c->pending = false;
@@ -254,6 +276,23 @@ infllm_status decode_impl(infllm_ctx* c, const void* q, const void* k, const voi
     if (D.G > 8) {  // wide groups: the chunk kernels handle a single token as well
         c->pending = true;
         return attend_impl<T>(c, q, 1, out);
+    }
+    if (sizeof(T) == 2 && c->use_tc && decode_tc_supported(D)) {
+        if (kk > 0) {
+            int l = 0;
+            Prof p(c, K_SELECT);
+            CK(launch_select<T>(D, c->cfg.score_mode, nm, 1, q, c->stream, &l, /*pdl=*/true));
+            p.done();
+            c->launches += l;
+        }
+        Prof p(c, K_DECODE);
+        int nt = 0;
+        cudaError_t e = launch_decode_tc(D, q, t, kk, B, out, c->stream, c->tmaps, &nt);
+        if (e != cudaSuccess) return fail(c, INFLLM_ECUDA, "decode launch (%d tiles): %s", nt, cudaGetErrorString(e));
+        p.done();
+        c->launches += 1;
+        record_attend(c, t, 1, nm, kk, B);
+        return INFLLM_OK;
     }
     if (kk > 0) {
         s = select_impl<T>(c, nm, 1, q);
@@ -325,6 +364,11 @@ infllm_status create_impl(infllm_ctx* c) {
     const int SK = decode_split_keys(c->elt);
     D.dec_splits_max = (int)((std::min<int64_t>(g.n_sink, g.max_tokens) + (int64_t)g.top_k * g.unit_size +
                               (int64_t)g.window + g.unit_size + 1 + SK - 1) / SK) + 1;
+    {   // tile-per-CTA decode: sink tiles + top_k * tiles per unit + window tiles
+        const int64_t tiles = (std::min<int64_t>(g.n_sink, g.max_tokens) + 127) / 128 +
+                              (int64_t)g.top_k * ((g.unit_size + 127) / 128) + ((int64_t)g.window + g.unit_size + 1 + 127) / 128 + 2;
+        D.dec_splits_max = std::max<int>(D.dec_splits_max, (int)tiles);
+    }
     D.P_rel = std::max(g.window, g.unit_size) + 1;
 
     CK(cudaGetDevice(&c->device));

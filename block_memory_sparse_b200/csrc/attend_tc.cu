@@ -18,13 +18,10 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "tc_maps.cuh"
 #include "tc_ptx.cuh"
 
 namespace infllm {
-
-struct TcMaps {
-    CUtensorMap kraw, krot, v, qm, qw;
-};
 
 namespace {
 

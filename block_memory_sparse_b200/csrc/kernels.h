@@ -23,7 +23,7 @@ cudaError_t launch_prep(const Dev& D, const void* q, int64_t c0, int n, cudaStre
 // of the per-tile partials.  Returns the number of kernels launched in *launches.
 template <typename T>
 cudaError_t launch_select(const Dev& D, int score_mode, int n_mem, int n_qtiles, const void* qraw,
-                          cudaStream_t st, int* launches);
+                          cudaStream_t st, int* launches, bool pdl = false);
 
 // Exact attention over sinks U selected units U window for a chunk (SIMT fp32-accumulate path).
 template <typename T>
@@ -42,5 +42,12 @@ cudaError_t launch_decode(const Dev& D, const void* q, int64_t t, int kk, int64_
                           int* n_split_out);
 
 int decode_split_keys(int elt_bytes);
+
+// Decode on the TMA path (bf16, head dim 128, G <= 8): store the token, then (after the lookup)
+// split-KV attention over 128-key tiles with a last-CTA log-sum-exp merge.
+bool decode_tc_supported(const Dev& D);
+cudaError_t launch_decode_append(const Dev& D, const void* q, const void* k, const void* v, int64_t t, cudaStream_t st);
+cudaError_t launch_decode_tc(const Dev& D, const void* q, int64_t t, int kk, int64_t B, void* out, cudaStream_t st,
+                             const void* tmaps, int* n_tiles_out);
 
 }  // namespace infllm

@@ -11,6 +11,7 @@
 // read of its representative keys (REPS mode) or of their fp32 sum (REPSUM mode).
 #include "common.cuh"
 #include "kernels.h"
+#include "tc_maps.cuh"
 
 namespace infllm {
 
@@ -92,6 +93,7 @@ __global__ void __launch_bounds__(128) k_score_topk(Dev D, int n_mem, int n_spli
     __shared__ float qb[128];
     __shared__ uint64_t lists[4][32];
     __shared__ int is_last;
+    asm volatile("griddepcontrol.launch_dependents;");  // a dependent attention kernel may start its prologue
     const int split = blockIdx.x, hk = blockIdx.y;
     for (int i = threadIdx.x; i < D.half; i += blockDim.x) {
         float a = 0.f, b = 0.f;
@@ -150,6 +152,10 @@ __global__ void __launch_bounds__(128) k_score_topk(Dev D, int n_mem, int n_spli
         D.uscore[(int64_t)hk * D.units_max + j] = s;
         cand = make_key(s, (uint32_t)j);
     }
+    // Under a programmatic dependent launch this grid may start before the preceding kernel ends;
+    // the scores do not depend on it, but this grid must not complete before it (the kernel after
+    // this one relies on both).
+    pdl_wait();
     if (!do_select) return;
     lists[warp][lane] = warp_sort_desc(cand);
     __syncthreads();
@@ -271,22 +277,38 @@ int score_lanes_per_unit(int n_mem, int Hkv) {
     return lpu;
 }
 
+template <typename T, int MODE, int LPU>
+static cudaError_t launch_score1(const Dev& D, dim3 grid, int n_mem, int n_split, int n_qtiles, const T* qraw,
+                                 int do_select, cudaStream_t st, bool pdl) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, k_score_topk<T, MODE, LPU>, D, n_mem, n_split, n_qtiles, qraw, do_select);
+}
+
 template <typename T, int MODE>
-static void launch_score(const Dev& D, int lpu, dim3 grid, int n_mem, int n_split, int n_qtiles, const T* qraw,
-                         int do_select, cudaStream_t st) {
+static cudaError_t launch_score(const Dev& D, int lpu, dim3 grid, int n_mem, int n_split, int n_qtiles, const T* qraw,
+                                int do_select, cudaStream_t st, bool pdl) {
     switch (lpu) {
-        case 1: k_score_topk<T, MODE, 1><<<grid, 128, 0, st>>>(D, n_mem, n_split, n_qtiles, qraw, do_select); break;
-        case 2: k_score_topk<T, MODE, 2><<<grid, 128, 0, st>>>(D, n_mem, n_split, n_qtiles, qraw, do_select); break;
-        case 4: k_score_topk<T, MODE, 4><<<grid, 128, 0, st>>>(D, n_mem, n_split, n_qtiles, qraw, do_select); break;
-        case 8: k_score_topk<T, MODE, 8><<<grid, 128, 0, st>>>(D, n_mem, n_split, n_qtiles, qraw, do_select); break;
-        case 16: k_score_topk<T, MODE, 16><<<grid, 128, 0, st>>>(D, n_mem, n_split, n_qtiles, qraw, do_select); break;
-        default: k_score_topk<T, MODE, 32><<<grid, 128, 0, st>>>(D, n_mem, n_split, n_qtiles, qraw, do_select); break;
+        case 1: return launch_score1<T, MODE, 1>(D, grid, n_mem, n_split, n_qtiles, qraw, do_select, st, pdl);
+        case 2: return launch_score1<T, MODE, 2>(D, grid, n_mem, n_split, n_qtiles, qraw, do_select, st, pdl);
+        case 4: return launch_score1<T, MODE, 4>(D, grid, n_mem, n_split, n_qtiles, qraw, do_select, st, pdl);
+        case 8: return launch_score1<T, MODE, 8>(D, grid, n_mem, n_split, n_qtiles, qraw, do_select, st, pdl);
+        case 16: return launch_score1<T, MODE, 16>(D, grid, n_mem, n_split, n_qtiles, qraw, do_select, st, pdl);
+        default: return launch_score1<T, MODE, 32>(D, grid, n_mem, n_split, n_qtiles, qraw, do_select, st, pdl);
     }
 }
 
 template <typename T>
 cudaError_t launch_select(const Dev& D, int score_mode, int n_mem, int n_qtiles, const void* qraw, cudaStream_t st,
-                          int* launches) {
+                          int* launches, bool pdl) {
     *launches = 0;
     if (n_mem <= 0 || D.topk <= 0) return cudaSuccess;
     const int lpu = score_lanes_per_unit(n_mem, D.Hkv);
@@ -295,12 +317,12 @@ cudaError_t launch_select(const Dev& D, int score_mode, int n_mem, int n_qtiles,
     if (n_split > D.score_splits_max) return cudaErrorInvalidValue;
     const int fast = D.topk <= 32;
     dim3 grid(n_split, D.Hkv);
-    if (score_mode == 0)
-        launch_score<T, 0>(D, lpu, grid, n_mem, n_split, n_qtiles, (const T*)qraw, fast, st);
-    else
-        launch_score<T, 1>(D, lpu, grid, n_mem, n_split, n_qtiles, (const T*)qraw, fast, st);
+    cudaError_t err = score_mode == 0
+                          ? launch_score<T, 0>(D, lpu, grid, n_mem, n_split, n_qtiles, (const T*)qraw, fast, st, pdl)
+                          : launch_score<T, 1>(D, lpu, grid, n_mem, n_split, n_qtiles, (const T*)qraw, fast, st, pdl);
     ++*launches;
-    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+    err = cudaGetLastError();
     if (err != cudaSuccess || fast) return err;
     int p2 = 1;
     while (p2 < n_mem) p2 <<= 1;  // n_mem <= 16384 (checked at create when top_k > 32)
@@ -316,7 +338,7 @@ cudaError_t launch_select(const Dev& D, int score_mode, int n_mem, int n_qtiles,
 
 template cudaError_t launch_prep<float>(const Dev&, const void*, int64_t, int, cudaStream_t);
 template cudaError_t launch_prep<__nv_bfloat16>(const Dev&, const void*, int64_t, int, cudaStream_t);
-template cudaError_t launch_select<float>(const Dev&, int, int, int, const void*, cudaStream_t, int*);
-template cudaError_t launch_select<__nv_bfloat16>(const Dev&, int, int, int, const void*, cudaStream_t, int*);
+template cudaError_t launch_select<float>(const Dev&, int, int, int, const void*, cudaStream_t, int*, bool);
+template cudaError_t launch_select<__nv_bfloat16>(const Dev&, int, int, int, const void*, cudaStream_t, int*, bool);
 
 }  // namespace infllm
