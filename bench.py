@@ -422,6 +422,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--tokens", type=int, default=0, help="truncate the prefill stream (small profiling cases)")
+    ap.add_argument("--only", choices=["prefill", "decode"], default=None,
+                    help="run only one part (profiling); the JSON line then carries that part alone")
     args = ap.parse_args()
     assert args.warmup >= 3 or args.impl == "reference", "at least 3 warm-up steps"
     rank, world, _ = dist_env()
@@ -431,7 +433,14 @@ def main():
             print(json.dumps(res), flush=True)
         return
     dist_init("nccl")
-    res = run_ours(args, rank, world)
+    if args.only == "decode":
+        import torch
+        _, _, local = dist_env()
+        torch.cuda.set_device(local)
+        res = {"impl": "ours", "decode": run_decode(args, torch, torch.device("cuda", local),
+                                                    torch.cuda.current_stream(), local)}
+    else:
+        res = run_ours(args, rank, world)
     if rank == 0:
         print(json.dumps(res), flush=True)
     import torch.distributed as dist

@@ -290,7 +290,7 @@ infllm_status decode_impl(infllm_ctx* c, const void* q, const void* k, const voi
         cudaError_t e = launch_decode_tc(D, q, t, kk, B, out, c->stream, c->tmaps, &nt);
         if (e != cudaSuccess) return fail(c, INFLLM_ECUDA, "decode launch (%d tiles): %s", nt, cudaGetErrorString(e));
         p.done();
-        c->launches += 1;
+        c->launches += 2;  // tiles + merge
         record_attend(c, t, 1, nm, kk, B);
         return INFLLM_OK;
     }
@@ -395,7 +395,9 @@ infllm_status create_impl(infllm_ctx* c) {
     double* invf = nullptr;
     float2* cs_rel = nullptr;
     float2* cs_w = nullptr;
+    double2* cs3 = nullptr;
     AL(invf, sizeof(double) * D.half);
+    AL(cs3, sizeof(double2) * 3 * 2048 * (size_t)D.half);
     AL(cs_rel, sizeof(float2) * (size_t)D.P_rel * D.half);
     AL(cs_w, sizeof(float2) * D.half);
 #undef AL
@@ -406,6 +408,17 @@ infllm_status create_impl(infllm_ctx* c) {
     for (int p = 0; p < D.P_rel; ++p)
         for (int i = 0; i < D.half; ++i) rel[(size_t)p * D.half + i] = make_float2((float)cos(p * th[i]), (float)sin(p * th[i]));
     for (int i = 0; i < D.half; ++i) w[i] = make_float2((float)cos(g.window * th[i]), (float)sin(g.window * th[i]));
+    {
+        std::vector<double2> t3((size_t)3 * 2048 * D.half);
+        for (int L = 0; L < 3; ++L)
+            for (int x = 0; x < 2048; ++x)
+                for (int i = 0; i < D.half; ++i) {
+                    const double ang = ldexp((double)x, 11 * L) * th[i];
+                    t3[((size_t)L * 2048 + x) * D.half + i] = make_double2(cos(ang), sin(ang));
+                }
+        CK(cudaMemcpy(cs3, t3.data(), sizeof(double2) * t3.size(), cudaMemcpyHostToDevice));
+        D.cs_abs3 = cs3;
+    }
     CK(cudaMemcpy(invf, th.data(), sizeof(double) * D.half, cudaMemcpyHostToDevice));
     CK(cudaMemcpy(cs_rel, rel.data(), sizeof(float2) * rel.size(), cudaMemcpyHostToDevice));
     CK(cudaMemcpy(cs_w, w.data(), sizeof(float2) * w.size(), cudaMemcpyHostToDevice));

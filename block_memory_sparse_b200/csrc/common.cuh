@@ -44,6 +44,9 @@ struct Dev {
     int P_rel;
     const float2* cs_W;      // [half] (cos, sin)(W theta_i)
     float2* cs_chunk;        // [max_chunk][half] (cos, sin)(t theta_i) for the current chunk
+    // (cos, sin)(x 2^(11 L) theta_i) in fp64 for L < 3, x < 2048: exp(i t theta) for any
+    // t < 2^33 is the product of three entries (t's 11-bit digits)
+    const double2* cs_abs3;  // [3][2048][half]
     // decode partials: [Hkv][dec_splits_max][G][d + 2]
     float* dec_part;
     int dec_splits_max;
@@ -146,6 +149,16 @@ __device__ __forceinline__ void st2f(__nv_bfloat16* p, float a, float b) {
     *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(a, b);
 }
 __device__ __forceinline__ void st2f(float* p, float a, float b) { *reinterpret_cast<float2*>(p) = make_float2(a, b); }
+
+// (cos, sin)(t theta_i) in fp64 from the three digit tables, rounded to float.
+__device__ __forceinline__ float2 cs_abs(const double2* tab, int half, int64_t t, int i) {
+    const double2 a = tab[(size_t)(t & 2047) * half + i];
+    const double2 b = tab[((size_t)2048 + ((t >> 11) & 2047)) * half + i];
+    const double2 c = tab[((size_t)4096 + ((t >> 22) & 2047)) * half + i];
+    const double re1 = a.x * b.x - a.y * b.y, im1 = a.x * b.y + a.y * b.x;
+    const double re = re1 * c.x - im1 * c.y, im = re1 * c.y + im1 * c.x;
+    return make_float2((float)re, (float)im);
+}
 
 __host__ __device__ __forceinline__ int64_t n_mem_at(int64_t c0, int S, int W, int U) {
     int64_t x = c0 - (int64_t)W - (int64_t)S;

@@ -46,9 +46,7 @@ __global__ void __launch_bounds__(DTHREADS) k_decode_append(Dev D, const __nv_bf
     asm volatile("griddepcontrol.launch_dependents;");  // the lookup kernel may start now
     const int hk = blockIdx.x;
     for (int i = threadIdx.x; i < D.half; i += blockDim.x) {
-        double s, c;
-        sincos((double)t * D.inv_freq[i], &s, &c);
-        cs[i] = make_float2((float)c, (float)s);
+        cs[i] = cs_abs(D.cs_abs3, D.half, t, i);
         if (hk == 0) D.cs_chunk[i] = cs[i];
     }
     __syncthreads();
@@ -119,10 +117,10 @@ __global__ void __launch_bounds__(DTHREADS) k_decode_attn(const __grid_constant_
     float* ps = reinterpret_cast<float*>(sm + OFF_PS);   // [G][DK]
     float* red = reinterpret_cast<float*>(sm + OFF_RED); // [2][4][G]
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + OFF_MISC);
-    int* is_last = reinterpret_cast<int*>(sm + OFF_MISC + 8);
     const int hk = blockIdx.y, ti = blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int G = D.G, d = DHD;
+    asm volatile("griddepcontrol.launch_dependents;");  // the merge kernel may start its prologue
     if (tid == 0) {
         ptx::mbar_init(bar, 1);
         ptx::mbar_fence_init();
@@ -244,27 +242,56 @@ __global__ void __launch_bounds__(DTHREADS) k_decode_attn(const __grid_constant_
             }
         }
     }
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) *is_last = (atomicAdd(&D.counters[D.Hkv + hk], 1u) == (unsigned)(NT - 1));
-    __syncthreads();
-    if (!*is_last) return;
-    __threadfence();
-    const float* base = D.dec_part + (int64_t)hk * D.dec_splits_max * G * (d + 2);
-    for (int h = 0; h < G; ++h) {
-        float M = -INFINITY;
-        for (int s = 0; s < NT; ++s) M = fmaxf(M, __ldcg(base + ((int64_t)s * G + h) * (d + 2)));
-        float L = 0.f, O = 0.f;
-        for (int s = 0; s < NT; ++s) {
-            const float* pp = base + ((int64_t)s * G + h) * (d + 2);
-            const float m = __ldcg(pp);
-            const float w = m == -INFINITY ? 0.f : expf(m - M);
-            L += w * __ldcg(pp + 1);
-            O += w * __ldcg(pp + 2 + tid);
-        }
-        out[(int64_t)(hk * G + h) * d + tid] = __float2bfloat16_rn(O / L);
+}
+
+// Log-sum-exp merge of the NT tile partials of one (KV head, q head): grid (G, Hkv), 512 threads
+// = 4 slices of tiles x 128 output dims; every load of a slice issued in one batch.
+constexpr int MERGE_SLICES = 4;
+constexpr int MERGE_BATCH = 32;
+
+__global__ void __launch_bounds__(MERGE_SLICES * DHD) k_decode_merge(Dev D, __nv_bfloat16* __restrict__ out, int NT) {
+    __shared__ float ml[2][MERGE_SLICES * MERGE_BATCH];
+    __shared__ float red[2][MERGE_SLICES][DHD];
+    pdl_wait();  // the tile partials are complete past this point
+    const int h = blockIdx.x, hk = blockIdx.y, G = D.G, d = DHD;
+    const int dim = threadIdx.x % DHD, z = threadIdx.x / DHD;
+    const float* base = D.dec_part + (int64_t)hk * D.dec_splits_max * G * (d + 2) + (int64_t)h * (d + 2);
+    const int64_t stride = (int64_t)G * (d + 2);
+    for (int s = threadIdx.x; s < NT && s < MERGE_SLICES * MERGE_BATCH; s += blockDim.x) {
+        ml[0][s] = base[s * stride];
+        ml[1][s] = base[s * stride + 1];
     }
-    if (tid == 0) D.counters[D.Hkv + hk] = 0u;
+    __syncthreads();
+    float M = -INFINITY;
+    for (int s = 0; s < NT; ++s) M = fmaxf(M, ml[0][s]);
+    float L = 0.f, O = 0.f;
+    float acc[MERGE_BATCH];
+#pragma unroll
+    for (int u = 0; u < MERGE_BATCH; ++u) {
+        const int s = z + MERGE_SLICES * u;
+        acc[u] = s < NT ? base[s * stride + 2 + dim] : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < MERGE_BATCH; ++u) {
+        const int s = z + MERGE_SLICES * u;
+        if (s < NT) {
+            const float m = ml[0][s];
+            const float w = m == -INFINITY ? 0.f : expf(m - M);
+            L += w * ml[1][s];
+            O += w * acc[u];
+        }
+    }
+    red[0][z][dim] = L;
+    red[1][z][dim] = O;
+    __syncthreads();
+    if (z == 0) {
+        float Lt = 0.f, Ot = 0.f;
+        for (int q = 0; q < MERGE_SLICES; ++q) {
+            Lt += red[0][q][dim];
+            Ot += red[1][q][dim];
+        }
+        out[(int64_t)(hk * G + h) * d + dim] = __float2bfloat16_rn(Ot / Lt);
+    }
 }
 
 }  // namespace
@@ -284,7 +311,7 @@ cudaError_t launch_decode_tc(const Dev& D, const void* q, int64_t t, int kk, int
     const int64_t win = t - B + 1;
     const int NT = (S_eff + DK - 1) / DK + kk * ((D.U + DK - 1) / DK) + (int)((win + DK - 1) / DK);
     *n_tiles_out = NT;
-    if (NT > D.dec_splits_max) return cudaErrorInvalidValue;
+    if (NT > D.dec_splits_max || NT > MERGE_SLICES * MERGE_BATCH) return cudaErrorInvalidValue;
     static bool attr_set = false;
     if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(k_decode_attn, cudaFuncAttributeMaxDynamicSharedMemorySize, DSMEM);
@@ -301,8 +328,17 @@ cudaError_t launch_decode_tc(const Dev& D, const void* q, int64_t t, int kk, int
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_decode_attn, *reinterpret_cast<const TcMaps*>(tmaps), D,
-                              (const __nv_bfloat16*)q, (__nv_bfloat16*)out, t, kk, B, NT);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, k_decode_attn, *reinterpret_cast<const TcMaps*>(tmaps), D,
+                                       (const __nv_bfloat16*)q, (__nv_bfloat16*)out, t, kk, B, NT);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t mcfg = {};
+    mcfg.gridDim = dim3(D.G, D.Hkv);
+    mcfg.blockDim = dim3(MERGE_SLICES * DHD);
+    mcfg.dynamicSmemBytes = 0;
+    mcfg.stream = st;
+    mcfg.attrs = attr;
+    mcfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&mcfg, k_decode_merge, D, (__nv_bfloat16*)out, NT);
 }
 
 }  // namespace infllm

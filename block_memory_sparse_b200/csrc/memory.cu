@@ -9,17 +9,15 @@
 
 namespace infllm {
 
-// One CTA per appended token: (cos, sin)(t * theta_i) in fp64 once per token (absolute
-// positions reach ~1e6 rad, beyond fp32 angle accuracy), then the three stores.
+// One CTA per appended token: (cos, sin)(t * theta_i) from the fp64 digit tables once per
+// token (absolute positions reach ~1e6 rad, beyond fp32 angle accuracy), then the three stores.
 template <typename T>
 __global__ void k_append(Dev D, const T* __restrict__ k, const T* __restrict__ v, int64_t c0) {
     extern __shared__ float2 cs_sh[];
     const int tl = blockIdx.x;
     const int64_t t = c0 + tl;
     for (int i = threadIdx.x; i < D.half; i += blockDim.x) {
-        double s, c;
-        sincos((double)t * D.inv_freq[i], &s, &c);
-        float2 cs = make_float2((float)c, (float)s);
+        const float2 cs = cs_abs(D.cs_abs3, D.half, t, i);
         cs_sh[i] = cs;
         D.cs_chunk[(int64_t)tl * D.half + i] = cs;
     }
@@ -45,37 +43,76 @@ __global__ void k_append(Dev D, const T* __restrict__ k, const T* __restrict__ v
 }
 
 // Y[b][hk] += sum over the chunk's tokens t in block b of sum_{h in group} R(t - s_b) q_{t,h}.
-// Grid (blocks touched, Hkv), 512 threads: thread = (pair couple pc: pairs 2pc, 2pc+1; token
-// group tg).  Fixed-order reduction over token groups, so results do not depend on scheduling.
+// Grid (blocks touched, Hkv), 256 threads: thread = (octet of pairs, token group), 16-byte
+// loads issued in batches (two tokens x up to four heads) before use.  Fixed-order reduction
+// over token groups, so results do not depend on scheduling.
 template <typename T>
-__global__ void __launch_bounds__(512) k_ysum(Dev D, const T* __restrict__ q, int64_t c0, int n, int64_t b0) {
+__global__ void __launch_bounds__(256) k_ysum(Dev D, const T* __restrict__ q, int64_t c0, int n, int64_t b0) {
     extern __shared__ float red[];
+    constexpr int V = 16 / sizeof(T);
+    constexpr int TB = 2, HB = 4;  // tokens and heads per load batch
     const int64_t b = b0 + blockIdx.x;
     const int hk = blockIdx.y;
     const int64_t sb = (int64_t)D.S + b * D.gblk;
     const int64_t lo = sb > c0 ? sb : c0;
     const int64_t hi = (sb + D.gblk) < (c0 + n) ? (sb + D.gblk) : (c0 + n);
-    const int npc = D.half / 2;
-    const int pc = threadIdx.x % npc, tg = threadIdx.x / npc, ntg = blockDim.x / npc;
-    const int i = 2 * pc;
-    float a1x = 0.f, a1y = 0.f, a2x = 0.f, a2y = 0.f;
-#pragma unroll 2
-    for (int64_t t = lo + tg; t < hi; t += ntg) {
-        const float4 cs = *reinterpret_cast<const float4*>(D.cs_rel + (t - sb) * D.half + i);  // (c_i, s_i, c_i+1, s_i+1)
-        const T* qr = q + ((t - c0) * D.Hq + (int64_t)hk * D.G) * D.d;
-        float2 x1 = make_float2(0.f, 0.f), x2 = make_float2(0.f, 0.f);
-        for (int h = 0; h < D.G; ++h) {  // the rotation is linear: sum the group's heads first
-            const float2 u = ld2f(qr + h * D.d + i), w = ld2f(qr + h * D.d + i + D.half);
-            x1.x += u.x; x1.y += u.y;
-            x2.x += w.x; x2.y += w.y;
+    const int nv = D.half / V;
+    const int o = threadIdx.x % nv, tg = threadIdx.x / nv, ntg = blockDim.x / nv;
+    const int i0 = o * V;
+    float a1[V], a2[V];
+#pragma unroll
+    for (int e = 0; e < V; ++e) a1[e] = a2[e] = 0.f;
+    for (int64_t t0 = lo + tg; t0 < hi; t0 += (int64_t)ntg * TB) {
+        float x1[TB][V], x2[TB][V];
+#pragma unroll
+        for (int u = 0; u < TB; ++u)
+#pragma unroll
+            for (int e = 0; e < V; ++e) x1[u][e] = x2[u][e] = 0.f;
+        for (int h0 = 0; h0 < D.G; h0 += HB) {
+            union { uint4 u; T v[V]; } r1[TB][HB], r2[TB][HB];
+#pragma unroll
+            for (int u = 0; u < TB; ++u) {
+                const int64_t t = t0 + (int64_t)u * ntg;
+#pragma unroll
+                for (int hh = 0; hh < HB; ++hh) {
+                    r1[u][hh].u = r2[u][hh].u = make_uint4(0, 0, 0, 0);
+                    if (t < hi && h0 + hh < D.G) {
+                        const T* qr = q + ((t - c0) * D.Hq + (int64_t)hk * D.G + h0 + hh) * D.d;
+                        r1[u][hh].u = *reinterpret_cast<const uint4*>(qr + i0);
+                        r2[u][hh].u = *reinterpret_cast<const uint4*>(qr + i0 + D.half);
+                    }
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < TB; ++u)
+#pragma unroll
+                for (int hh = 0; hh < HB; ++hh)
+#pragma unroll
+                    for (int e = 0; e < V; ++e) {  // the rotation is linear: sum the group's heads first
+                        x1[u][e] += to_f(r1[u][hh].v[e]);
+                        x2[u][e] += to_f(r2[u][hh].v[e]);
+                    }
         }
-        a1x += x1.x * cs.x - x2.x * cs.y;
-        a2x += x2.x * cs.x + x1.x * cs.y;
-        a1y += x1.y * cs.z - x2.y * cs.w;
-        a2y += x2.y * cs.z + x1.y * cs.w;
+#pragma unroll
+        for (int u = 0; u < TB; ++u) {
+            const int64_t t = t0 + (int64_t)u * ntg;
+            if (t < hi) {
+                const float2* cs = D.cs_rel + (t - sb) * D.half + i0;
+#pragma unroll
+                for (int e = 0; e < V; ++e) {
+                    const float2 c = cs[e];
+                    a1[e] += x1[u][e] * c.x - x2[u][e] * c.y;
+                    a2[e] += x2[u][e] * c.x + x1[u][e] * c.y;
+                }
+            }
+        }
     }
     float* r = red + tg * D.d;
-    r[i] = a1x; r[i + 1] = a1y; r[i + D.half] = a2x; r[i + D.half + 1] = a2y;
+#pragma unroll
+    for (int e = 0; e < V; ++e) {
+        r[i0 + e] = a1[e];
+        r[i0 + e + D.half] = a2[e];
+    }
     __syncthreads();
     for (int j = threadIdx.x; j < D.d; j += blockDim.x) {
         float acc = 0.f;
@@ -104,12 +141,27 @@ __global__ void __launch_bounds__(256) k_reps(Dev D, int64_t j0) {
     {
         const int i = threadIdx.x % D.half, pg = threadIdx.x / D.half, npg = blockDim.x / D.half;
         float a1 = 0.f, a2 = 0.f;
-        for (int p = pg; p < nb; p += npg) {
-            const float* y = D.Y + ((be + p) * D.Hkv + hk) * D.d;
-            const float2 cs = D.cs_rel[(int64_t)p * D.gblk * D.half + i];
-            const float y1 = y[i], y2 = y[i + D.half];
-            a1 += y1 * cs.x - y2 * cs.y;
-            a2 += y2 * cs.x + y1 * cs.y;
+        constexpr int PB = 8;  // window blocks per load batch
+        for (int p0 = pg; p0 < nb; p0 += npg * PB) {
+            float y1[PB], y2[PB];
+            float2 cs[PB];
+#pragma unroll
+            for (int u = 0; u < PB; ++u) {
+                const int p = p0 + u * npg;
+                y1[u] = y2[u] = 0.f;
+                cs[u] = make_float2(0.f, 0.f);
+                if (p < nb) {
+                    const float* y = D.Y + ((be + p) * D.Hkv + hk) * D.d;
+                    y1[u] = y[i];
+                    y2[u] = y[i + D.half];
+                    cs[u] = D.cs_rel[(int64_t)p * D.gblk * D.half + i];
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < PB; ++u) {
+                a1 += y1[u] * cs[u].x - y2[u] * cs[u].y;
+                a2 += y2[u] * cs[u].x + y1[u] * cs[u].y;
+            }
         }
         part[pg * D.d + i] = a1;
         part[pg * D.d + i + D.half] = a2;
@@ -128,15 +180,24 @@ __global__ void __launch_bounds__(256) k_reps(Dev D, int64_t j0) {
         float acc[UNR];
 #pragma unroll
         for (int u = 0; u < UNR; ++u) acc[u] = 0.f;
-        for (int i = lane; i < D.half; i += 32) {
-            const float q1 = Qt[i], q2 = Qt[i + D.half];
 #pragma unroll
-            for (int u = 0; u < UNR; ++u) {
-                const int m = mb + u;
-                if (m < D.U) {
-                    const float2 cs = D.cs_rel[(int64_t)(D.U - m) * D.half + i];  // distance e - (m0 + m)
-                    const float r1 = q1 * cs.x - q2 * cs.y, r2 = q2 * cs.x + q1 * cs.y;
-                    acc[u] += r1 * to_f(K[(int64_t)m * D.d + i]) + r2 * to_f(K[(int64_t)m * D.d + i + D.half]);
+        for (int ii = 0; ii < 2; ++ii) {  // half <= 64: pairs lane and lane + 32
+            const int i = lane + 32 * ii;
+            if (i < D.half) {
+                const float q1 = Qt[i], q2 = Qt[i + D.half];
+                float k1[UNR], k2[UNR];
+                float2 cs[UNR];
+#pragma unroll
+                for (int u = 0; u < UNR; ++u) {
+                    const int m = mb + u < D.U ? mb + u : D.U - 1;
+                    cs[u] = D.cs_rel[(int64_t)(D.U - m) * D.half + i];  // distance e - (m0 + m)
+                    k1[u] = to_f(K[(int64_t)m * D.d + i]);
+                    k2[u] = to_f(K[(int64_t)m * D.d + i + D.half]);
+                }
+#pragma unroll
+                for (int u = 0; u < UNR; ++u) {
+                    const float r1 = q1 * cs[u].x - q2 * cs[u].y, r2 = q2 * cs[u].x + q1 * cs[u].y;
+                    acc[u] += r1 * k1[u] + r2 * k2[u];
                 }
             }
         }
@@ -183,10 +244,17 @@ __global__ void __launch_bounds__(256) k_reps(Dev D, int64_t j0) {
     float* rs = D.repsum + ((int64_t)hk * D.units_max + j) * D.d;
     for (int i = threadIdx.x; i < D.d; i += blockDim.x) {
         float s = 0.f;
-        for (int qq = 0; qq < D.r; ++qq) {
-            const T x = K[(int64_t)ids[qq] * D.d + i];
-            rk[(int64_t)qq * D.d + i] = x;
-            s += to_f(x);
+        for (int q0 = 0; q0 < D.r; q0 += 8) {
+            T x[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (q0 + u < D.r) x[u] = K[(int64_t)ids[q0 + u] * D.d + i];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (q0 + u < D.r) {
+                    rk[(int64_t)(q0 + u) * D.d + i] = x[u];
+                    s += to_f(x[u]);
+                }
         }
         rs[i] = s;
     }

@@ -83,30 +83,66 @@ template <> struct Vec16<float> {
     }
 };
 
-// Grid (n_split, Hkv), 128 threads.  Each unit is scored by a group of LPU lanes that split
-// its operand (16-byte loads, all in flight), reduced inside the group; per = 128 / LPU units
-// per CTA.  Warp top-32 lists, CTA merge, then the last CTA of each kv head (arrival counter,
-// no waiting) merges every CTA's list with all four warps and writes the selection.
+// Grid (n_split, Hkv), 512 threads.  Each unit is scored by a group of LPU lanes that split
+// its operand (16-byte loads issued in batches of 16), reduced inside the group; PER = 512 / LPU
+// units per CTA.  Warp top-32 lists, tree merge inside the CTA, then the last CTA of each kv
+// head (arrival counter, no waiting) merges every CTA's list and writes the selection.
+constexpr int SC_THREADS = 512;
+constexpr int SC_WARPS = SC_THREADS / 32;
+
+__device__ __forceinline__ void tree_merge(uint64_t (*lists)[32], int warp, int lane) {
+#pragma unroll
+    for (int stride = 1; stride < SC_WARPS; stride *= 2) {
+        __syncthreads();
+        if ((warp % (2 * stride)) == 0) lists[warp][lane] = warp_merge_desc(lists[warp][lane], lists[warp + stride][lane]);
+    }
+    __syncthreads();
+}
+
 template <typename T, int MODE, int LPU>
-__global__ void __launch_bounds__(128) k_score_topk(Dev D, int n_mem, int n_split, int n_qtiles, const T* qraw,
-                                                    int do_select) {
+__global__ void __launch_bounds__(SC_THREADS) k_score_topk(Dev D, int n_mem, int n_split, int n_qtiles,
+                                                           const T* qraw, int do_select) {
     __shared__ float qb[128];
-    __shared__ uint64_t lists[4][32];
+    __shared__ uint64_t lists[SC_WARPS][32];
     __shared__ int is_last;
     asm volatile("griddepcontrol.launch_dependents;");  // a dependent attention kernel may start its prologue
     const int split = blockIdx.x, hk = blockIdx.y;
     for (int i = threadIdx.x; i < D.half; i += blockDim.x) {
         float a = 0.f, b = 0.f;
         if (qraw) {
-            for (int h = 0; h < D.G; ++h) {
-                a += to_f(qraw[(hk * D.G + h) * D.d + i]);
-                b += to_f(qraw[(hk * D.G + h) * D.d + i + D.half]);
+            for (int h0 = 0; h0 < D.G; h0 += 8) {
+                float x[8], y[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    x[u] = y[u] = 0.f;
+                    if (h0 + u < D.G) {
+                        x[u] = to_f(qraw[(hk * D.G + h0 + u) * D.d + i]);
+                        y[u] = to_f(qraw[(hk * D.G + h0 + u) * D.d + i + D.half]);
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    a += x[u];
+                    b += y[u];
+                }
             }
         } else {
-            for (int tt = 0; tt < n_qtiles; ++tt) {
-                const float* p = D.qbar_part + ((int64_t)hk * D.qtiles_max + tt) * D.d;
-                a += p[i];
-                b += p[i + D.half];
+            for (int t0 = 0; t0 < n_qtiles; t0 += 8) {
+                float x[8], y[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    x[u] = y[u] = 0.f;
+                    if (t0 + u < n_qtiles) {
+                        const float* p = D.qbar_part + ((int64_t)hk * D.qtiles_max + t0 + u) * D.d;
+                        x[u] = p[i];
+                        y[u] = p[i + D.half];
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    a += x[u];
+                    b += y[u];
+                }
             }
         }
         const float2 cw = D.cs_W[i];
@@ -115,8 +151,8 @@ __global__ void __launch_bounds__(128) k_score_topk(Dev D, int n_mem, int n_spli
     }
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    constexpr int PER = 128 / LPU;       // units per CTA
-    constexpr int UPW = 32 / LPU;        // units per warp
+    constexpr int PER = SC_THREADS / LPU;  // units per CTA
+    constexpr int UPW = 32 / LPU;          // units per warp
     const int j = split * PER + warp * UPW + lane / LPU;
     const int sub = lane % LPU;
     uint64_t cand = 0;
@@ -126,22 +162,40 @@ __global__ void __launch_bounds__(128) k_score_topk(Dev D, int n_mem, int n_spli
             const T* p = (const T*)D.rep_keys + ((int64_t)hk * D.units_max + j) * D.r * D.d;
             constexpr int N = Vec16<T>::N;
             const int total = D.r * D.d;
-#pragma unroll 8
-            for (int e = sub * N; e < total; e += LPU * N) {
-                float f[N];
-                Vec16<T>::load(p + e, f);
-                const int i0 = e % D.d;
+            for (int e0 = sub * N; e0 < total; e0 += 16 * LPU * N) {
+                float f[16][N];
 #pragma unroll
-                for (int c = 0; c < N; ++c) acc += f[c] * qb[i0 + c];
+                for (int u = 0; u < 16; ++u) {
+                    const int e = e0 + u * LPU * N;
+                    if (e < total) Vec16<T>::load(p + e, f[u]);
+                }
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    const int e = e0 + u * LPU * N;
+                    if (e < total) {
+                        const int i0 = e % D.d;
+#pragma unroll
+                        for (int c = 0; c < N; ++c) acc += f[u][c] * qb[i0 + c];
+                    }
+                }
             }
         } else {  // fp32 sum of the representative keys [d]
             const float* p = D.repsum + ((int64_t)hk * D.units_max + j) * D.d;
-#pragma unroll 8
-            for (int e = sub * 4; e < D.d; e += LPU * 4) {
-                float f[4];
-                Vec16<float>::load(p + e, f);
+            for (int e0 = sub * 4; e0 < D.d; e0 += 16 * LPU * 4) {
+                float f[16][4];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) acc += f[c] * qb[e + c];
+                for (int u = 0; u < 16; ++u) {
+                    const int e = e0 + u * LPU * 4;
+                    if (e < D.d) Vec16<float>::load(p + e, f[u]);
+                }
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    const int e = e0 + u * LPU * 4;
+                    if (e < D.d) {
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) acc += f[u][c] * qb[e + c];
+                    }
+                }
             }
         }
     }
@@ -158,28 +212,32 @@ __global__ void __launch_bounds__(128) k_score_topk(Dev D, int n_mem, int n_spli
     pdl_wait();
     if (!do_select) return;
     lists[warp][lane] = warp_sort_desc(cand);
-    __syncthreads();
-    if (warp == 0) {
-        uint64_t m = lists[0][lane];
-        for (int w = 1; w < 4; ++w) m = warp_merge_desc(m, lists[w][lane]);
-        D.cand[((int64_t)hk * D.score_splits_max + split) * 32 + lane] = m;
-    }
+    tree_merge(lists, warp, lane);
+    if (warp == 0) D.cand[((int64_t)hk * D.score_splits_max + split) * 32 + lane] = lists[0][lane];
     __threadfence();
     __syncthreads();
     if (threadIdx.x == 0) is_last = (atomicAdd(&D.counters[hk], 1u) == (unsigned)(n_split - 1));
     __syncthreads();
     if (!is_last) return;
     __threadfence();
-    {   // each warp merges a strided quarter of the lists, then warp 0 merges the four
+    {   // each warp merges a strided share of the lists (loads of a batch issued together)
         uint64_t m = 0;
-        for (int s = warp; s < n_split; s += 4)
-            m = warp_merge_desc(m, __ldcg(&D.cand[((int64_t)hk * D.score_splits_max + s) * 32 + lane]));
+        const uint64_t* cb = D.cand + (int64_t)hk * D.score_splits_max * 32 + lane;
+        for (int s0 = warp; s0 < n_split; s0 += SC_WARPS * 4) {
+            uint64_t b[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int s = s0 + SC_WARPS * u;
+                b[u] = s < n_split ? __ldcg(cb + (int64_t)s * 32) : 0ull;
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) m = warp_merge_desc(m, b[u]);
+        }
         lists[warp][lane] = m;
     }
-    __syncthreads();
+    tree_merge(lists, warp, lane);
     if (warp == 0) {
-        uint64_t m = lists[0][lane];
-        for (int w = 1; w < 4; ++w) m = warp_merge_desc(m, lists[w][lane]);
+        const uint64_t m = lists[0][lane];
         const int kk = min(D.topk, n_mem);
         const uint32_t id = key_index(m);
         uint64_t sk = (lane < kk) ? (uint64_t)(0xffffffffu - id) : 0ull;
@@ -270,10 +328,10 @@ cudaError_t launch_prep(const Dev& D, const void* q, int64_t c0, int n, cudaStre
     return cudaGetLastError();
 }
 
-// Lanes per unit: the fewest that still give about two CTAs per SM (296 CTAs).
+// Lanes per unit: the fewest that still give at least one CTA per SM (148).
 int score_lanes_per_unit(int n_mem, int Hkv) {
     int lpu = 1;
-    while (lpu < 32 && (int64_t)((n_mem + 128 / lpu - 1) / (128 / lpu)) * Hkv < 296) lpu *= 2;
+    while (lpu < 32 && (int64_t)((n_mem + SC_THREADS / lpu - 1) / (SC_THREADS / lpu)) * Hkv < 148) lpu *= 2;
     return lpu;
 }
 
@@ -282,7 +340,7 @@ static cudaError_t launch_score1(const Dev& D, dim3 grid, int n_mem, int n_split
                                  int do_select, cudaStream_t st, bool pdl) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
-    cfg.blockDim = dim3(128);
+    cfg.blockDim = dim3(SC_THREADS);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
@@ -312,7 +370,7 @@ cudaError_t launch_select(const Dev& D, int score_mode, int n_mem, int n_qtiles,
     *launches = 0;
     if (n_mem <= 0 || D.topk <= 0) return cudaSuccess;
     const int lpu = score_lanes_per_unit(n_mem, D.Hkv);
-    const int per = 128 / lpu;
+    const int per = SC_THREADS / lpu;
     const int n_split = (n_mem + per - 1) / per;
     if (n_split > D.score_splits_max) return cudaErrorInvalidValue;
     const int fast = D.topk <= 32;
