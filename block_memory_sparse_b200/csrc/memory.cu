@@ -44,13 +44,13 @@ __global__ void k_append(Dev D, const T* __restrict__ k, const T* __restrict__ v
 
 // Y[b][hk] += sum over the chunk's tokens t in block b of sum_{h in group} R(t - s_b) q_{t,h}.
 // Grid (blocks touched, Hkv), 256 threads: thread = (octet of pairs, token group), 16-byte
-// loads issued in batches (two tokens x up to four heads) before use.  Fixed-order reduction
+// loads issued in batches (up to four heads of a token) before use.  Fixed-order reduction
 // over token groups, so results do not depend on scheduling.
 template <typename T>
-__global__ void __launch_bounds__(256) k_ysum(Dev D, const T* __restrict__ q, int64_t c0, int n, int64_t b0) {
+__global__ void __launch_bounds__(256, 2) k_ysum(Dev D, const T* __restrict__ q, int64_t c0, int n, int64_t b0) {
     extern __shared__ float red[];
     constexpr int V = 16 / sizeof(T);
-    constexpr int TB = 2, HB = 4;  // tokens and heads per load batch
+    constexpr int TB = 1, HB = 4;  // tokens and heads per load batch
     const int64_t b = b0 + blockIdx.x;
     const int hk = blockIdx.y;
     const int64_t sb = (int64_t)D.S + b * D.gblk;
@@ -275,9 +275,10 @@ cudaError_t launch_ysum(const Dev& D, const void* q, int64_t c0, int n, cudaStre
     const int64_t hi = c0 + n;
     if (hi <= lo) return cudaSuccess;
     const int64_t b0 = (lo - D.S) / D.gblk, b1 = (hi - 1 - D.S) / D.gblk;
-    const int threads = 512;  // (half / 2) pair couples x token groups
+    const int threads = 256;  // (half / V) octets x token groups
+    const int nv = D.half / (16 / (int)sizeof(T));
     dim3 grid((unsigned)(b1 - b0 + 1), D.Hkv);
-    k_ysum<T><<<grid, threads, (threads / (D.half / 2)) * D.d * sizeof(float), st>>>(D, (const T*)q, c0, n, b0);
+    k_ysum<T><<<grid, threads, (threads / nv) * D.d * sizeof(float), st>>>(D, (const T*)q, c0, n, b0);
     ++*launches;
     return cudaGetLastError();
 }
