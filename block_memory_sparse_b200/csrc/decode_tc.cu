@@ -26,15 +26,16 @@ constexpr int DHD = 128;                    // head dim
 constexpr uint32_t DTILE = DK * DHD * 2;    // bytes of a bf16 tile
 constexpr uint32_t DHALF = DTILE / 2;       // one 64-column swizzle block
 constexpr int DTHREADS = 128;
-constexpr int MAXG = 8;
+constexpr int MAXG = 8;  // q heads per KV head on this path (rows of the padded MMA tile)
 constexpr int ERR_TIMEOUT = 16;
-// dynamic shared memory: K tile | V tile | q frames [2][G][d] | p [G][DK] | reductions
+// dynamic shared memory: K tile | V tile | this tile's rotated query [16 rows][d] bf16 (rows >= G
+// zero, padded row stride) | reductions.  The P V partials of the four warps reuse the K tile.
+constexpr int QSTRIDE = DHD * 2 + 16;  // bytes per padded query row (conflict-free ldmatrix)
 constexpr int OFF_K = 0;
 constexpr int OFF_V = OFF_K + (int)DTILE;
 constexpr int OFF_Q = OFF_V + (int)DTILE;
-constexpr int OFF_PS = OFF_Q + 2 * MAXG * DHD * 4;
-constexpr int OFF_RED = OFF_PS + MAXG * DK * 4;
-constexpr int OFF_MISC = OFF_RED + 2 * 4 * MAXG * 4;
+constexpr int OFF_RED = OFF_Q + 16 * QSTRIDE;
+constexpr int OFF_MISC = OFF_RED + 2 * 4 * 8 * 4;
 constexpr int DSMEM = OFF_MISC + 64 + 1024;  // + alignment slack
 
 // One CTA per KV head: K, R(t) K and V of token t into the stores, the query block sum of t,
@@ -105,21 +106,48 @@ __device__ __forceinline__ DTile decode_tile(const Dev& D, int hk, int i, int64_
     return {2, B + (int64_t)i * DK, (int)(rem < DK ? rem : DK)};
 }
 
-// Grid (tiles, Hkv), 128 threads.  Thread j owns key j of the tile for the logits and output
-// dimension j for P V.
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+// D (16x8 fp32) += A (16x16 bf16, row) * B (16x8 bf16, col)
+__device__ __forceinline__ void mma16816(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+// Shared address of the 16-byte chunk c (8 elements) of row j in a TMA tile (two 64-column
+// blocks of 128 rows x 128 bytes, 16-byte chunks XOR-swizzled by row % 8).
+__device__ __forceinline__ uint32_t tile_chunk(uint32_t base, int j, int c) {
+    return base + (uint32_t)(c >> 3) * DHALF + (uint32_t)j * 128 + ((uint32_t)((c & 7) ^ (j & 7)) << 4);
+}
+
+// Grid (tiles, Hkv), 128 threads = 4 warps, warp w owns keys [32w, 32w + 32) of the tile.
+// The group's G query heads (rows, padded to 16 with zeros) times the tile on the tensor cores
+// (mma.sync m16n8k16, bf16 in, fp32 accumulate): S = Q K^T, then O = P V with P kept in
+// registers; softmax statistics are combined across the four warps through shared memory.
 __global__ void __launch_bounds__(DTHREADS) k_decode_attn(const __grid_constant__ TcMaps maps, Dev D,
                                                           const __nv_bfloat16* __restrict__ q,
                                                           __nv_bfloat16* __restrict__ out, int64_t t, int kk, int64_t B,
                                                           int NT) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    float* qs = reinterpret_cast<float*>(sm + OFF_Q);    // [2][G][d]: R(W) q, R(t) q
-    float* ps = reinterpret_cast<float*>(sm + OFF_PS);   // [G][DK]
-    float* red = reinterpret_cast<float*>(sm + OFF_RED); // [2][4][G]
+    float* red = reinterpret_cast<float*>(sm + OFF_RED);  // [2][4 warps][8 rows]
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + OFF_MISC);
     const int hk = blockIdx.y, ti = blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int G = D.G, d = DHD;
+    const int g = lane >> 2, tg = lane & 3;
+    const int G = D.G;
     asm volatile("griddepcontrol.launch_dependents;");  // the merge kernel may start its prologue
     if (tid == 0) {
         ptx::mbar_init(bar, 1);
@@ -136,110 +164,123 @@ __global__ void __launch_bounds__(DTHREADS) k_decode_attn(const __grid_constant_
         ptx::tma_load_3d(sm + OFF_V, &maps.v, bar, 0, (int)T.y0, hk);
         ptx::tma_load_3d(sm + OFF_V + DHALF, &maps.v, bar, 64, (int)T.y0, hk);
     }
-    // rotated queries of the group's heads while the tiles land
-    for (int idx = tid; idx < G * D.half; idx += blockDim.x) {
-        const int h = idx / D.half, i = idx % D.half;
-        const float x1 = __bfloat162float(q[(hk * G + h) * d + i]), x2 = __bfloat162float(q[(hk * G + h) * d + i + D.half]);
-        const float2 cw = D.cs_W[i], ct = D.cs_chunk[i];
-        qs[h * d + i] = x1 * cw.x - x2 * cw.y;
-        qs[h * d + i + D.half] = x2 * cw.x + x1 * cw.y;
-        qs[(G + h) * d + i] = x1 * ct.x - x2 * ct.y;
-        qs[(G + h) * d + i + D.half] = x2 * ct.x + x1 * ct.y;
+    // this tile's query frame (R(W) q for sinks and memory, R(t) q for the window) as bf16 rows
+    {
+        const float2* cs = T.kind == 2 ? D.cs_chunk : D.cs_W;
+        for (int idx = tid; idx < 16 * (DHD / 2); idx += DTHREADS) {
+            const int h = idx / (DHD / 2), i = idx % (DHD / 2);
+            float r1 = 0.f, r2 = 0.f;
+            if (h < G) {
+                const float x1 = __bfloat162float(q[(hk * G + h) * DHD + i]);
+                const float x2 = __bfloat162float(q[(hk * G + h) * DHD + i + DHD / 2]);
+                const float2 c = cs[i];
+                r1 = x1 * c.x - x2 * c.y;
+                r2 = x2 * c.x + x1 * c.y;
+            }
+            __nv_bfloat16* row = reinterpret_cast<__nv_bfloat16*>(sm + OFF_Q + h * QSTRIDE);
+            row[i] = __float2bfloat16_rn(r1);
+            row[i + DHD / 2] = __float2bfloat16_rn(r2);
+        }
     }
     __syncthreads();
+    uint32_t qa[DHD / 16][4];
+    {
+        const uint32_t qbase = ptx::smem_u32(sm + OFF_Q) + (uint32_t)(lane & 15) * QSTRIDE + (uint32_t)(lane >> 4) * 16;
+#pragma unroll
+        for (int ks = 0; ks < DHD / 16; ++ks) ldsm_x4(qbase + ks * 32, qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3]);
+    }
     bool ok = ptx::mbar_wait(bar, 0);
     if (!ok) set_err(D, ERR_TIMEOUT);
     ok = __syncthreads_and(ok);
-    float sc[MAXG];
+    // S for the warp's 32 keys: n-tiles nt -> keys 32w + 8nt + (0..7)
+    const uint32_t kbase = ptx::smem_u32(sm + OFF_K), vbase = ptx::smem_u32(sm + OFF_V);
+    float sacc[4][4];
 #pragma unroll
-    for (int h = 0; h < MAXG; ++h) sc[h] = -INFINITY;
-    if (ok && tid < T.nv) {
-        const float* qf = qs + (T.kind == 2 ? G : 0) * d;
-        float acc[MAXG];
+    for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-        for (int h = 0; h < MAXG; ++h) acc[h] = 0.f;
-        const uint8_t* krow = sm + OFF_K + tid * 128;
-#pragma unroll 4
-        for (int c = 0; c < 16; ++c) {  // 16-byte chunk c of the row (swizzled inside its 128-byte line)
-            const uint4 u = *reinterpret_cast<const uint4*>(krow + (c >> 3) * DHALF + (((c & 7) ^ (tid & 7)) << 4));
-            const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
-            float kv[8];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 f = __bfloat1622float2(h2[e]);
-                kv[2 * e] = f.x;
-                kv[2 * e + 1] = f.y;
-            }
-#pragma unroll
-            for (int h = 0; h < MAXG; ++h) {
-                if (h < G) {
-                    const float4 qa = *reinterpret_cast<const float4*>(qf + h * d + c * 8);
-                    const float4 qb = *reinterpret_cast<const float4*>(qf + h * d + c * 8 + 4);
-                    acc[h] += qa.x * kv[0] + qa.y * kv[1] + qa.z * kv[2] + qa.w * kv[3] + qb.x * kv[4] +
-                              qb.y * kv[5] + qb.z * kv[6] + qb.w * kv[7];
-                }
-            }
-        }
-#pragma unroll
-        for (int h = 0; h < MAXG; ++h) sc[h] = acc[h] * D.inv_sqrt_d;
-    }
-    // per-head max and sum over the tile
-    float mh[MAXG], lh[MAXG];
-#pragma unroll
-    for (int h = 0; h < MAXG; ++h) {
-        if (h < G) {
-            const float m = warp_max(sc[h]);
-            if (lane == 0) red[warp * G + h] = m;
-        }
-    }
-    __syncthreads();
-#pragma unroll
-    for (int h = 0; h < MAXG; ++h) {
-        mh[h] = -INFINITY;
-        if (h < G)
-            for (int w = 0; w < 4; ++w) mh[h] = fmaxf(mh[h], red[w * G + h]);
-    }
-#pragma unroll
-    for (int h = 0; h < MAXG; ++h) {
-        if (h < G) {
-            const float p = (tid < T.nv && ok) ? expf(sc[h] - mh[h]) : 0.f;
-            ps[h * DK + tid] = p;
-            const float s = warp_sum(p);
-            if (lane == 0) red[4 * G + warp * G + h] = s;
-        }
-    }
-    __syncthreads();
-#pragma unroll
-    for (int h = 0; h < MAXG; ++h) {
-        lh[h] = 0.f;
-        if (h < G)
-            for (int w = 0; w < 4; ++w) lh[h] += red[4 * G + w * G + h];
-    }
-    // P V: thread owns output dimension tid (d == blockDim)
-    float o[MAXG];
-#pragma unroll
-    for (int h = 0; h < MAXG; ++h) o[h] = 0.f;
+        for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
     {
-        const int dim = tid;
-        const uint8_t* vcol = sm + OFF_V + (dim >> 6) * DHALF + (dim & 7) * 2;
-        const int chunk = (dim & 63) >> 3;
-        for (int j = 0; j < T.nv; ++j) {
-            const float vv = __bfloat162float(
-                *reinterpret_cast<const __nv_bfloat16*>(vcol + j * 128 + ((chunk ^ (j & 7)) << 4)));
+        const int key_a = 32 * warp + (lane & 7);  // lanes 0-15: n-tile 2p, lanes 16-31: n-tile 2p + 1
 #pragma unroll
-            for (int h = 0; h < MAXG; ++h)
-                if (h < G) o[h] += ps[h * DK + j] * vv;
+        for (int ks = 0; ks < DHD / 16; ++ks) {
+#pragma unroll
+            for (int pr = 0; pr < 2; ++pr) {
+                const int key = key_a + 16 * pr + ((lane >> 4) << 3);
+                const int c = 2 * ks + ((lane >> 3) & 1);
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4(tile_chunk(kbase, key, c), b0, b1, b2, b3);
+                mma16816(sacc[2 * pr], qa[ks], b0, b1);
+                mma16816(sacc[2 * pr + 1], qa[ks], b2, b3);
+            }
         }
     }
-    float* part = D.dec_part + ((int64_t)hk * D.dec_splits_max + ti) * G * (d + 2);
+    // softmax over the tile for row g (heads g < G); keys >= nv are masked
+    const float sc = D.inv_sqrt_d * 1.4426950408889634f;
+    float mx = -INFINITY;
 #pragma unroll
-    for (int h = 0; h < MAXG; ++h) {
-        if (h < G) {
-            part[h * (d + 2) + 2 + tid] = o[h];
-            if (tid == 0) {
-                part[h * (d + 2) + 0] = mh[h];
-                part[h * (d + 2) + 1] = lh[h];
-            }
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int key = 32 * warp + 8 * nt + 2 * tg + e;
+            if (!ok || key >= T.nv) sacc[nt][e] = -INFINITY;
+            mx = fmaxf(mx, sacc[nt][e]);
+        }
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    if (tg == 0) red[warp * 8 + g] = mx;
+    __syncthreads();
+    float m = fmaxf(fmaxf(red[g], red[8 + g]), fmaxf(red[16 + g], red[24 + g]));
+    const float mref = m == -INFINITY ? 0.f : m;
+    float rs = 0.f;
+    uint32_t pa[2][4];
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) {
+        float p0, p1;
+        asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(p0) : "f"((sacc[nt][0] - mref) * sc));
+        asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(p1) : "f"((sacc[nt][1] - mref) * sc));
+        rs += p0 + p1;
+        // A fragment of P for k-step nt / 2: n-tile 2s -> a0a1 (rows g), 2s + 1 -> a4a5; rows 8..15 zero
+        pa[nt >> 1][(nt & 1) ? 2 : 0] = pack_bf16(p0, p1);
+        pa[nt >> 1][(nt & 1) ? 3 : 1] = 0u;
+    }
+    rs += __shfl_xor_sync(0xffffffffu, rs, 1);
+    rs += __shfl_xor_sync(0xffffffffu, rs, 2);
+    if (tg == 0) red[32 + warp * 8 + g] = rs;
+    // O partial of this warp's 32 keys: 16 n-tiles of output dims
+    float oacc[16][4];
+#pragma unroll
+    for (int nt = 0; nt < 16; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) oacc[nt][e] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < 2; ++ks) {
+        const int key = 32 * warp + 16 * ks + (lane & 7) + (((lane >> 3) & 1) << 3);
+#pragma unroll
+        for (int np = 0; np < 8; ++np) {
+            const int c = 2 * np + (lane >> 4);
+            uint32_t b0, b1, b2, b3;
+            ldsm_x4_t(tile_chunk(vbase, key, c), b0, b1, b2, b3);
+            mma16816(oacc[2 * np], pa[ks], b0, b1);
+            mma16816(oacc[2 * np + 1], pa[ks], b2, b3);
+        }
+    }
+    __syncthreads();  // every warp is done with the K tile: reuse it for the cross-warp sum of O
+    float* obuf = reinterpret_cast<float*>(sm + OFF_K);  // [4 warps][8 rows][DHD]
+#pragma unroll
+    for (int nt = 0; nt < 16; ++nt) {
+        obuf[(warp * 8 + g) * DHD + 8 * nt + 2 * tg] = oacc[nt][0];
+        obuf[(warp * 8 + g) * DHD + 8 * nt + 2 * tg + 1] = oacc[nt][1];
+    }
+    __syncthreads();
+    float* part = D.dec_part + ((int64_t)hk * D.dec_splits_max + ti) * G * (DHD + 2);
+    for (int h = 0; h < G; ++h) {
+        const float o = obuf[(0 * 8 + h) * DHD + tid] + obuf[(1 * 8 + h) * DHD + tid] + obuf[(2 * 8 + h) * DHD + tid] +
+                        obuf[(3 * 8 + h) * DHD + tid];
+        part[h * (DHD + 2) + 2 + tid] = o;
+        if (tid == 0) {
+            const float mh = fmaxf(fmaxf(red[h], red[8 + h]), fmaxf(red[16 + h], red[24 + h]));
+            part[h * (DHD + 2) + 0] = mh == -INFINITY ? -INFINITY : mh * D.inv_sqrt_d;  // natural-log units
+            part[h * (DHD + 2) + 1] = red[32 + h] + red[40 + h] + red[48 + h] + red[56 + h];
         }
     }
 }

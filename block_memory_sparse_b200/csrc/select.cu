@@ -100,7 +100,7 @@ __device__ __forceinline__ void tree_merge(uint64_t (*lists)[32], int warp, int 
 }
 
 template <typename T, int MODE, int LPU>
-__global__ void __launch_bounds__(SC_THREADS) k_score_topk(Dev D, int n_mem, int n_split, int n_qtiles,
+__global__ void __launch_bounds__(SC_THREADS, 2) k_score_topk(Dev D, int n_mem, int n_split, int n_qtiles,
                                                            const T* qraw, int do_select) {
     __shared__ float qb[128];
     __shared__ uint64_t lists[SC_WARPS][32];
@@ -158,42 +158,37 @@ __global__ void __launch_bounds__(SC_THREADS) k_score_topk(Dev D, int n_mem, int
     uint64_t cand = 0;
     float acc = 0.f;
     if (j < n_mem) {
-        if (MODE == 0) {  // representative keys [r][d]
-            const T* p = (const T*)D.rep_keys + ((int64_t)hk * D.units_max + j) * D.r * D.d;
-            constexpr int N = Vec16<T>::N;
-            const int total = D.r * D.d;
-            for (int e0 = sub * N; e0 < total; e0 += 16 * LPU * N) {
-                float f[16][N];
+        // 16-byte vectors kept raw in registers (8 per batch), converted at use
+        const T* p = MODE == 0 ? (const T*)D.rep_keys + ((int64_t)hk * D.units_max + j) * D.r * D.d
+                               : nullptr;
+        const float* pf = MODE == 0 ? nullptr : D.repsum + ((int64_t)hk * D.units_max + j) * D.d;
+        constexpr int N = MODE == 0 ? Vec16<T>::N : 4;  // elements per vector
+        const int total = MODE == 0 ? D.r * D.d : D.d;
+        for (int e0 = sub * N; e0 < total; e0 += 8 * LPU * N) {
+            uint4 raw[8];
 #pragma unroll
-                for (int u = 0; u < 16; ++u) {
-                    const int e = e0 + u * LPU * N;
-                    if (e < total) Vec16<T>::load(p + e, f[u]);
-                }
-#pragma unroll
-                for (int u = 0; u < 16; ++u) {
-                    const int e = e0 + u * LPU * N;
-                    if (e < total) {
-                        const int i0 = e % D.d;
-#pragma unroll
-                        for (int c = 0; c < N; ++c) acc += f[u][c] * qb[i0 + c];
-                    }
-                }
+            for (int u = 0; u < 8; ++u) {
+                const int e = e0 + u * LPU * N;
+                if (e < total)
+                    raw[u] = MODE == 0 ? __ldg(reinterpret_cast<const uint4*>(p + e))
+                                       : __ldg(reinterpret_cast<const uint4*>(pf + e));
             }
-        } else {  // fp32 sum of the representative keys [d]
-            const float* p = D.repsum + ((int64_t)hk * D.units_max + j) * D.d;
-            for (int e0 = sub * 4; e0 < D.d; e0 += 16 * LPU * 4) {
-                float f[16][4];
 #pragma unroll
-                for (int u = 0; u < 16; ++u) {
-                    const int e = e0 + u * LPU * 4;
-                    if (e < D.d) Vec16<float>::load(p + e, f[u]);
-                }
+            for (int u = 0; u < 8; ++u) {
+                const int e = e0 + u * LPU * N;
+                if (e < total) {
+                    const int i0 = e % D.d;
+                    if (MODE == 0 && sizeof(T) == 2) {
+                        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw[u]);
 #pragma unroll
-                for (int u = 0; u < 16; ++u) {
-                    const int e = e0 + u * LPU * 4;
-                    if (e < D.d) {
+                        for (int c = 0; c < 4; ++c) {
+                            const float2 f = __bfloat1622float2(h2[c]);
+                            acc += f.x * qb[i0 + 2 * c] + f.y * qb[i0 + 2 * c + 1];
+                        }
+                    } else {
+                        const float* f = reinterpret_cast<const float*>(&raw[u]);
 #pragma unroll
-                        for (int c = 0; c < 4; ++c) acc += f[u][c] * qb[e + c];
+                        for (int c = 0; c < 4; ++c) acc += f[c] * qb[i0 + c];
                     }
                 }
             }
