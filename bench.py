@@ -317,7 +317,7 @@ def run_decode(args, torch, device, stream, local):
     P = peaks()
     out = {}
     # memory of 1,052,800 tokens built once (untimed); both scoring pools are kept by the library
-    layer = InfLLMLayer.from_workload(w, max_tokens=w.n_tokens + 2 * steps, max_chunk=w.build_chunk)
+    layer = InfLLMLayer.from_workload(w, max_tokens=w.n_tokens + 2 * steps + 32, max_chunk=w.build_chunk)
     t0 = time.time()
     for c0 in range(0, w.n_tokens, w.build_chunk):
         n = min(w.build_chunk, w.n_tokens - c0)
@@ -326,6 +326,8 @@ def run_decode(args, torch, device, stream, local):
     torch.cuda.synchronize()
     build_s = time.time() - t0
     qkv = [tuple(to_dev(a, torch, device) for a in synth.gen_chunk(w, w.n_tokens + s, 1)) for s in range(2 * steps)]
+    qkv_extra = [tuple(to_dev(a, torch, device) for a in synth.gen_chunk(w, w.n_tokens + 2 * steps + s, 1))
+                 for s in range(32)]
     o = torch.empty((1, w.n_q_heads, w.head_dim), dtype=torch.bfloat16, device=device)
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
     for mi, mode in enumerate(("reps", "repsum")):
@@ -342,6 +344,15 @@ def run_decode(args, torch, device, stream, local):
             torch.cuda.synchronize()
         us = np.array([a.elapsed_time(b) * 1e3 for a, b in evs])
         launches = layer.stats()["kernel_launches"] - n_launch0
+        # per-kernel-class device time (events around each launch; breaks launch overlap, so the
+        # sum exceeds the step time above): where a step's time goes
+        layer.set_profiling(True)
+        for s in range(16):  # extra tokens after both timed passes' tokens
+            flush.fill_(float(s))
+            layer.decode_step(*qkv_extra[16 * mi + s], out=o)
+        torch.cuda.synchronize()
+        st_prof = layer.stats()
+        layer.set_profiling(False)
         byts = np.array([decode_bytes(w, w.n_tokens + mi * steps + s, mode) for s in range(steps)])
         med = float(np.median(us))
         gbs = float(np.median(byts / (us * 1e-6) / 1e9))
@@ -349,6 +360,9 @@ def run_decode(args, torch, device, stream, local):
                      "algorithmic_bytes_per_step": float(np.median(byts)),
                      "hbm_gbs": gbs, "hbm_frac_of_measured": gbs / P["hbm"], "hbm_frac_of_8tbs_nominal": gbs / 8000.0,
                      "launches_per_step": launches / steps, "steps": steps, "clocks": clk.summary()}
+        if st_prof["n_decode"]:
+            out[mode]["profiled_us_per_step"] = {k: 1e3 * st_prof[f"ms_{k}"] / 16 for k in
+                                                 ("append", "reps", "select", "decode")}
     layer.close()
     del qkv, flush
     torch.cuda.empty_cache()

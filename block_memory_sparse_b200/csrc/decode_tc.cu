@@ -66,10 +66,20 @@ __global__ void __launch_bounds__(DTHREADS) k_decode_append(Dev D, const __nv_bf
         V[dst + i + D.half] = v[hk * D.d + i + D.half];
         if (t >= D.S) {  // query block sum (same arithmetic as the chunk kernel for one token)
             const int64_t b = (t - D.S) / D.gblk, p = (t - D.S) % D.gblk;
+            float qx[MAXG], qy[MAXG];
+#pragma unroll
+            for (int h = 0; h < MAXG; ++h) {
+                qx[h] = qy[h] = 0.f;
+                if (h < D.G) {
+                    qx[h] = __bfloat162float(q[(hk * D.G + h) * D.d + i]);
+                    qy[h] = __bfloat162float(q[(hk * D.G + h) * D.d + i + D.half]);
+                }
+            }
             float s1 = 0.f, s2 = 0.f;
-            for (int h = 0; h < D.G; ++h) {
-                s1 += __bfloat162float(q[(hk * D.G + h) * D.d + i]);
-                s2 += __bfloat162float(q[(hk * D.G + h) * D.d + i + D.half]);
+#pragma unroll
+            for (int h = 0; h < MAXG; ++h) {
+                s1 += qx[h];
+                s2 += qy[h];
             }
             const float2 c = D.cs_rel[p * D.half + i];
             float* y = D.Y + (b * D.Hkv + hk) * D.d;

@@ -43,80 +43,80 @@ __global__ void k_append(Dev D, const T* __restrict__ k, const T* __restrict__ v
 }
 
 // Y[b][hk] += sum over the chunk's tokens t in block b of sum_{h in group} R(t - s_b) q_{t,h}.
-// Grid (blocks touched, Hkv), 256 threads: thread = (octet of pairs, token group), 16-byte
-// loads issued in batches (up to four heads of a token) before use.  Fixed-order reduction
-// over token groups, so results do not depend on scheduling.
+// Grid (blocks touched, Hkv), 1024 threads: thread = (octet of pairs, token), so every load of
+// the block is issued at once (heads in batches of four).  Fixed-order reduction (warp shuffles,
+// then warps in order), so results do not depend on scheduling.
 template <typename T>
-__global__ void __launch_bounds__(256, 2) k_ysum(Dev D, const T* __restrict__ q, int64_t c0, int n, int64_t b0) {
-    extern __shared__ float red[];
+__global__ void __launch_bounds__(1024) k_ysum(Dev D, const T* __restrict__ q, int64_t c0, int n, int64_t b0) {
+    extern __shared__ float red[];  // [warps][d]
     constexpr int V = 16 / sizeof(T);
-    constexpr int TB = 1, HB = 4;  // tokens and heads per load batch
+    constexpr int HB = 4;
     const int64_t b = b0 + blockIdx.x;
     const int hk = blockIdx.y;
     const int64_t sb = (int64_t)D.S + b * D.gblk;
     const int64_t lo = sb > c0 ? sb : c0;
     const int64_t hi = (sb + D.gblk) < (c0 + n) ? (sb + D.gblk) : (c0 + n);
-    const int nv = D.half / V;
+    const int nv = D.half / V;  // octets per token (power of two, <= 8)
     const int o = threadIdx.x % nv, tg = threadIdx.x / nv, ntg = blockDim.x / nv;
     const int i0 = o * V;
     float a1[V], a2[V];
 #pragma unroll
     for (int e = 0; e < V; ++e) a1[e] = a2[e] = 0.f;
-    for (int64_t t0 = lo + tg; t0 < hi; t0 += (int64_t)ntg * TB) {
-        float x1[TB][V], x2[TB][V];
+    for (int64_t t = lo + tg; t < hi; t += ntg) {
+        float x1[V], x2[V];
 #pragma unroll
-        for (int u = 0; u < TB; ++u)
-#pragma unroll
-            for (int e = 0; e < V; ++e) x1[u][e] = x2[u][e] = 0.f;
+        for (int e = 0; e < V; ++e) x1[e] = x2[e] = 0.f;
+        const T* qr = q + ((t - c0) * D.Hq + (int64_t)hk * D.G) * D.d;
         for (int h0 = 0; h0 < D.G; h0 += HB) {
-            union { uint4 u; T v[V]; } r1[TB][HB], r2[TB][HB];
+            union { uint4 u; T v[V]; } r1[HB], r2[HB];
 #pragma unroll
-            for (int u = 0; u < TB; ++u) {
-                const int64_t t = t0 + (int64_t)u * ntg;
-#pragma unroll
-                for (int hh = 0; hh < HB; ++hh) {
-                    r1[u][hh].u = r2[u][hh].u = make_uint4(0, 0, 0, 0);
-                    if (t < hi && h0 + hh < D.G) {
-                        const T* qr = q + ((t - c0) * D.Hq + (int64_t)hk * D.G + h0 + hh) * D.d;
-                        r1[u][hh].u = *reinterpret_cast<const uint4*>(qr + i0);
-                        r2[u][hh].u = *reinterpret_cast<const uint4*>(qr + i0 + D.half);
-                    }
+            for (int hh = 0; hh < HB; ++hh) {
+                r1[hh].u = r2[hh].u = make_uint4(0, 0, 0, 0);
+                if (h0 + hh < D.G) {
+                    r1[hh].u = *reinterpret_cast<const uint4*>(qr + (h0 + hh) * D.d + i0);
+                    r2[hh].u = *reinterpret_cast<const uint4*>(qr + (h0 + hh) * D.d + i0 + D.half);
                 }
             }
 #pragma unroll
-            for (int u = 0; u < TB; ++u)
+            for (int hh = 0; hh < HB; ++hh)
 #pragma unroll
-                for (int hh = 0; hh < HB; ++hh)
-#pragma unroll
-                    for (int e = 0; e < V; ++e) {  // the rotation is linear: sum the group's heads first
-                        x1[u][e] += to_f(r1[u][hh].v[e]);
-                        x2[u][e] += to_f(r2[u][hh].v[e]);
-                    }
+                for (int e = 0; e < V; ++e) {  // the rotation is linear: sum the group's heads first
+                    x1[e] += to_f(r1[hh].v[e]);
+                    x2[e] += to_f(r2[hh].v[e]);
+                }
         }
+        const float2* cs = D.cs_rel + (t - sb) * D.half + i0;
 #pragma unroll
-        for (int u = 0; u < TB; ++u) {
-            const int64_t t = t0 + (int64_t)u * ntg;
-            if (t < hi) {
-                const float2* cs = D.cs_rel + (t - sb) * D.half + i0;
-#pragma unroll
-                for (int e = 0; e < V; ++e) {
-                    const float2 c = cs[e];
-                    a1[e] += x1[u][e] * c.x - x2[u][e] * c.y;
-                    a2[e] += x2[u][e] * c.x + x1[u][e] * c.y;
-                }
-            }
+        for (int e = 0; e < V; ++e) {
+            const float2 c = cs[e];
+            a1[e] += x1[e] * c.x - x2[e] * c.y;
+            a2[e] += x2[e] * c.x + x1[e] * c.y;
         }
     }
-    float* r = red + tg * D.d;
+    // lanes holding the same octet of different tokens: xor over the token bits of the lane
 #pragma unroll
-    for (int e = 0; e < V; ++e) {
-        r[i0 + e] = a1[e];
-        r[i0 + e + D.half] = a2[e];
+    for (int m = 16; m >= 1; m >>= 1) {
+        if (m < nv) break;
+#pragma unroll
+        for (int e = 0; e < V; ++e) {
+            a1[e] += __shfl_xor_sync(0xffffffffu, a1[e], m);
+            a2[e] += __shfl_xor_sync(0xffffffffu, a2[e], m);
+        }
+    }
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane < nv) {
+        float* r = red + warp * D.d;
+#pragma unroll
+        for (int e = 0; e < V; ++e) {
+            r[i0 + e] = a1[e];
+            r[i0 + e + D.half] = a2[e];
+        }
     }
     __syncthreads();
+    const int nw = blockDim.x >> 5;
     for (int j = threadIdx.x; j < D.d; j += blockDim.x) {
         float acc = 0.f;
-        for (int g = 0; g < ntg; ++g) acc += red[g * D.d + j];
+        for (int w = 0; w < nw; ++w) acc += red[w * D.d + j];
         D.Y[(b * D.Hkv + hk) * D.d + j] += acc;
     }
 }
@@ -275,10 +275,9 @@ cudaError_t launch_ysum(const Dev& D, const void* q, int64_t c0, int n, cudaStre
     const int64_t hi = c0 + n;
     if (hi <= lo) return cudaSuccess;
     const int64_t b0 = (lo - D.S) / D.gblk, b1 = (hi - 1 - D.S) / D.gblk;
-    const int threads = 256;  // (half / V) octets x token groups
-    const int nv = D.half / (16 / (int)sizeof(T));
+    const int threads = 1024;  // (half / V) octets x tokens
     dim3 grid((unsigned)(b1 - b0 + 1), D.Hkv);
-    k_ysum<T><<<grid, threads, (threads / nv) * D.d * sizeof(float), st>>>(D, (const T*)q, c0, n, b0);
+    k_ysum<T><<<grid, threads, (threads / 32) * D.d * sizeof(float), st>>>(D, (const T*)q, c0, n, b0);
     ++*launches;
     return cudaGetLastError();
 }

@@ -15,43 +15,77 @@
 
 namespace infllm {
 
-// Rotated, packed queries of the chunk.  Grid (tiles, Hkv), 512 threads.  Tile a holds
+// Rotated, packed queries of the chunk.  Grid (tiles, Hkv), 256 threads.  Tile a holds
 // queries [a*qt, a*qt + qt); row r of a tile is (head hg = r / qt, query a*qt + r % qt).
-// Thread = (pair couple pc: pairs 2pc, 2pc+1; row group).  Also writes each tile's raw query
-// sum over its rows (fixed-order reduction).
+// Thread = (vector v: elements [vV, vV+V) of each half, row group): 16-byte loads and stores,
+// four rows per load batch.  Also writes each tile's raw query sum over its rows
+// (fixed-order reduction).
 template <typename T>
-__global__ void __launch_bounds__(512) k_prep(Dev D, const T* __restrict__ q, int n) {
+__global__ void __launch_bounds__(256) k_prep(Dev D, const T* __restrict__ q, int n) {
     extern __shared__ float red[];
+    constexpr int V = 16 / sizeof(T);
+    constexpr int RB = 4;
+    union Vec { uint4 u; T h[V]; };
     const int a = blockIdx.x, hk = blockIdx.y;
     const int rows = D.qt * D.G;
-    const int npc = D.half / 2;
-    const int pc = threadIdx.x % npc, rg = threadIdx.x / npc, nrg = blockDim.x / npc;
-    const int i = 2 * pc;
-    const float4 cw = *reinterpret_cast<const float4*>(D.cs_W + i);
+    const int nv = D.half / V;
+    const int o = threadIdx.x % nv, rg = threadIdx.x / nv, nrg = blockDim.x / nv;
+    const int i0 = o * V;
     T* Qm = (T*)D.Qm + ((int64_t)hk * D.qrows_max + (int64_t)a * rows) * D.d;
     T* Qw = (T*)D.Qw + ((int64_t)hk * D.qrows_max + (int64_t)a * rows) * D.d;
-    float s1x = 0.f, s1y = 0.f, s2x = 0.f, s2y = 0.f;
-#pragma unroll 4
-    for (int r = rg; r < rows; r += nrg) {
-        const int hg = r / D.qt, tl = a * D.qt + r % D.qt;
-        float2 x1 = make_float2(0.f, 0.f), x2 = make_float2(0.f, 0.f);
-        float4 ct = make_float4(1.f, 0.f, 1.f, 0.f);
-        if (tl < n) {
-            const T* src = q + ((int64_t)tl * D.Hq + hk * D.G + hg) * D.d;
-            x1 = ld2f(src + i);
-            x2 = ld2f(src + i + D.half);
-            ct = *reinterpret_cast<const float4*>(D.cs_chunk + (int64_t)tl * D.half + i);
+    float2 cw[V];
+#pragma unroll
+    for (int e = 0; e < V; ++e) cw[e] = D.cs_W[i0 + e];
+    float s1[V], s2[V];
+#pragma unroll
+    for (int e = 0; e < V; ++e) s1[e] = s2[e] = 0.f;
+    for (int r0 = rg; r0 < rows; r0 += nrg * RB) {
+        Vec x1[RB], x2[RB];
+        float2 ct[RB][V];
+#pragma unroll
+        for (int u = 0; u < RB; ++u) {
+            const int r = r0 + u * nrg;
+            const int hg = r / D.qt, tl = a * D.qt + r % D.qt;
+            x1[u].u = x2[u].u = make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int e = 0; e < V; ++e) ct[u][e] = make_float2(1.f, 0.f);
+            if (r < rows && tl < n) {
+                const T* src = q + ((int64_t)tl * D.Hq + hk * D.G + hg) * D.d;
+                x1[u].u = *reinterpret_cast<const uint4*>(src + i0);
+                x2[u].u = *reinterpret_cast<const uint4*>(src + i0 + D.half);
+#pragma unroll
+                for (int e = 0; e < V; ++e) ct[u][e] = D.cs_chunk[(int64_t)tl * D.half + i0 + e];
+            }
         }
-        s1x += x1.x; s1y += x1.y; s2x += x2.x; s2y += x2.y;
-        T* dm = Qm + (int64_t)r * D.d;
-        T* dw = Qw + (int64_t)r * D.d;
-        st2f(dm + i, x1.x * cw.x - x2.x * cw.y, x1.y * cw.z - x2.y * cw.w);
-        st2f(dm + i + D.half, x2.x * cw.x + x1.x * cw.y, x2.y * cw.z + x1.y * cw.w);
-        st2f(dw + i, x1.x * ct.x - x2.x * ct.y, x1.y * ct.z - x2.y * ct.w);
-        st2f(dw + i + D.half, x2.x * ct.x + x1.x * ct.y, x2.y * ct.z + x1.y * ct.w);
+#pragma unroll
+        for (int u = 0; u < RB; ++u) {
+            const int r = r0 + u * nrg;
+            if (r >= rows) continue;
+            Vec m1, m2, w1, w2;
+#pragma unroll
+            for (int e = 0; e < V; ++e) {
+                const float a1 = to_f(x1[u].h[e]), a2 = to_f(x2[u].h[e]);
+                s1[e] += a1;
+                s2[e] += a2;
+                m1.h[e] = from_f<T>(a1 * cw[e].x - a2 * cw[e].y);
+                m2.h[e] = from_f<T>(a2 * cw[e].x + a1 * cw[e].y);
+                w1.h[e] = from_f<T>(a1 * ct[u][e].x - a2 * ct[u][e].y);
+                w2.h[e] = from_f<T>(a2 * ct[u][e].x + a1 * ct[u][e].y);
+            }
+            T* dm = Qm + (int64_t)r * D.d;
+            T* dw = Qw + (int64_t)r * D.d;
+            *reinterpret_cast<uint4*>(dm + i0) = m1.u;
+            *reinterpret_cast<uint4*>(dm + i0 + D.half) = m2.u;
+            *reinterpret_cast<uint4*>(dw + i0) = w1.u;
+            *reinterpret_cast<uint4*>(dw + i0 + D.half) = w2.u;
+        }
     }
     float* rr = red + rg * D.d;
-    rr[i] = s1x; rr[i + 1] = s1y; rr[i + D.half] = s2x; rr[i + D.half + 1] = s2y;
+#pragma unroll
+    for (int e = 0; e < V; ++e) {
+        rr[i0 + e] = s1[e];
+        rr[i0 + e + D.half] = s2[e];
+    }
     __syncthreads();
     for (int j = threadIdx.x; j < D.d; j += blockDim.x) {
         float acc = 0.f;
@@ -84,28 +118,16 @@ template <> struct Vec16<float> {
 };
 
 // Grid (n_split, Hkv), 512 threads.  Each unit is scored by a group of LPU lanes that split
-// its operand (16-byte loads issued in batches of 16), reduced inside the group; PER = 512 / LPU
-// units per CTA.  Warp top-32 lists, tree merge inside the CTA, then the last CTA of each kv
-// head (arrival counter, no waiting) merges every CTA's list and writes the selection.
+// its operand (16-byte loads issued in batches of 8), reduced inside the group; PER = 512 / LPU
+// units per CTA.  Writes the unit scores; the selection kernel picks the top-k.
 constexpr int SC_THREADS = 512;
 constexpr int SC_WARPS = SC_THREADS / 32;
-
-__device__ __forceinline__ void tree_merge(uint64_t (*lists)[32], int warp, int lane) {
-#pragma unroll
-    for (int stride = 1; stride < SC_WARPS; stride *= 2) {
-        __syncthreads();
-        if ((warp % (2 * stride)) == 0) lists[warp][lane] = warp_merge_desc(lists[warp][lane], lists[warp + stride][lane]);
-    }
-    __syncthreads();
-}
 
 template <typename T, int MODE, int LPU>
 __global__ void __launch_bounds__(SC_THREADS, 2) k_score_topk(Dev D, int n_mem, int n_split, int n_qtiles,
                                                            const T* qraw, int do_select) {
     __shared__ float qb[128];
-    __shared__ uint64_t lists[SC_WARPS][32];
-    __shared__ int is_last;
-    asm volatile("griddepcontrol.launch_dependents;");  // a dependent attention kernel may start its prologue
+    asm volatile("griddepcontrol.launch_dependents;");  // the selection kernel may start its prologue
     const int split = blockIdx.x, hk = blockIdx.y;
     for (int i = threadIdx.x; i < D.half; i += blockDim.x) {
         float a = 0.f, b = 0.f;
@@ -155,7 +177,6 @@ __global__ void __launch_bounds__(SC_THREADS, 2) k_score_topk(Dev D, int n_mem, 
     constexpr int UPW = 32 / LPU;          // units per warp
     const int j = split * PER + warp * UPW + lane / LPU;
     const int sub = lane % LPU;
-    uint64_t cand = 0;
     float acc = 0.f;
     if (j < n_mem) {
         // 16-byte vectors kept raw in registers (8 per batch), converted at use
@@ -196,47 +217,54 @@ __global__ void __launch_bounds__(SC_THREADS, 2) k_score_topk(Dev D, int n_mem, 
     }
 #pragma unroll
     for (int m = LPU / 2; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
-    if (j < n_mem && sub == 0) {
-        const float s = acc * D.inv_sqrt_d;
-        D.uscore[(int64_t)hk * D.units_max + j] = s;
-        cand = make_key(s, (uint32_t)j);
-    }
+    if (j < n_mem && sub == 0) D.uscore[(int64_t)hk * D.units_max + j] = acc * D.inv_sqrt_d;
+    (void)do_select;
     // Under a programmatic dependent launch this grid may start before the preceding kernel ends;
-    // the scores do not depend on it, but this grid must not complete before it (the kernel after
-    // this one relies on both).
+    // the scores do not depend on it, but this grid must not complete before it (the kernels after
+    // this one rely on both).
     pdl_wait();
-    if (!do_select) return;
-    lists[warp][lane] = warp_sort_desc(cand);
-    tree_merge(lists, warp, lane);
-    if (warp == 0) D.cand[((int64_t)hk * D.score_splits_max + split) * 32 + lane] = lists[0][lane];
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) is_last = (atomicAdd(&D.counters[hk], 1u) == (unsigned)(n_split - 1));
-    __syncthreads();
-    if (!is_last) return;
-    __threadfence();
-    {   // each warp merges a strided share of the lists (loads of a batch issued together)
-        uint64_t m = 0;
-        const uint64_t* cb = D.cand + (int64_t)hk * D.score_splits_max * 32 + lane;
-        for (int s0 = warp; s0 < n_split; s0 += SC_WARPS * 4) {
-            uint64_t b[4];
+}
+
+// Top-k of one KV head's unit scores: one CTA of 1024 threads per KV head.  Every warp keeps a
+// running descending top-32 list of the composite keys (score, ~unit) over a strided share of
+// the units (a batch is sorted and merged only when one of its keys beats the list's last entry),
+// then the 32 lists are merged pairwise in shared memory.  Ties go to the lower unit index.
+constexpr int SEL_THREADS = 1024;
+constexpr int SEL_WARPS = SEL_THREADS / 32;
+
+__global__ void __launch_bounds__(SEL_THREADS) k_select_topk(Dev D, int n_mem) {
+    __shared__ uint64_t lists[SEL_WARPS][32];
+    asm volatile("griddepcontrol.launch_dependents;");
+    pdl_wait();  // the unit scores are complete past this point
+    const int hk = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const float* sc = D.uscore + (int64_t)hk * D.units_max;
+    uint64_t list = 0;
+    constexpr int B = 4;  // batches of 32 candidates per warp, loads issued together
+    for (int j0 = warp * 32 * B; j0 < n_mem; j0 += SEL_WARPS * 32 * B) {
+        float v[B];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int s = s0 + SC_WARPS * u;
-                b[u] = s < n_split ? __ldcg(cb + (int64_t)s * 32) : 0ull;
-            }
-#pragma unroll
-            for (int u = 0; u < 4; ++u) m = warp_merge_desc(m, b[u]);
+        for (int u = 0; u < B; ++u) {
+            const int j = j0 + u * 32 + lane;
+            v[u] = j < n_mem ? __ldcg(sc + j) : 0.f;
         }
-        lists[warp][lane] = m;
+#pragma unroll
+        for (int u = 0; u < B; ++u) {
+            const int j = j0 + u * 32 + lane;
+            list = warp_topk_insert(list, j < n_mem ? make_key(v[u], (uint32_t)j) : 0ull);
+        }
     }
-    tree_merge(lists, warp, lane);
+    lists[warp][lane] = list;
+#pragma unroll
+    for (int stride = 1; stride < SEL_WARPS; stride *= 2) {
+        __syncthreads();
+        if ((warp % (2 * stride)) == 0) lists[warp][lane] = warp_merge_desc(lists[warp][lane], lists[warp + stride][lane]);
+    }
+    __syncthreads();
     if (warp == 0) {
         const uint64_t m = lists[0][lane];
         const int kk = min(D.topk, n_mem);
-        const uint32_t id = key_index(m);
-        uint64_t sk = (lane < kk) ? (uint64_t)(0xffffffffu - id) : 0ull;
-        sk = warp_sort_desc(sk);
+        uint64_t sk = (lane < kk) ? (uint64_t)(0xffffffffu - key_index(m)) : 0ull;
+        sk = warp_sort_desc(sk);  // ascending ids
         if (lane < D.topk) {
             int o = -1;
             if (lane < kk) {
@@ -248,7 +276,6 @@ __global__ void __launch_bounds__(SC_THREADS, 2) k_score_topk(Dev D, int n_mem, 
             }
             D.sel[hk * D.topk + lane] = o;
         }
-        if (lane == 0) D.counters[hk] = 0u;
     }
 }
 
@@ -317,9 +344,10 @@ cudaError_t launch_prep(const Dev& D, const void* q, int64_t c0, int n, cudaStre
     (void)c0;
     if (n <= 0) return cudaSuccess;
     const int tiles = (n + D.qt - 1) / D.qt;
-    const int threads = 512;
+    const int threads = 256;
+    const int nv = D.half / (16 / (int)sizeof(T));
     dim3 grid(tiles, D.Hkv);
-    k_prep<T><<<grid, threads, (threads / (D.half / 2)) * D.d * sizeof(float), st>>>(D, (const T*)q, n);
+    k_prep<T><<<grid, threads, (threads / nv) * D.d * sizeof(float), st>>>(D, (const T*)q, n);
     return cudaGetLastError();
 }
 
@@ -376,7 +404,21 @@ cudaError_t launch_select(const Dev& D, int score_mode, int n_mem, int n_qtiles,
     ++*launches;
     if (err != cudaSuccess) return err;
     err = cudaGetLastError();
-    if (err != cudaSuccess || fast) return err;
+    if (err != cudaSuccess) return err;
+    if (fast) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(D.Hkv);
+        cfg.blockDim = dim3(SEL_THREADS);
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        err = cudaLaunchKernelEx(&cfg, k_select_topk, D, n_mem);
+        ++*launches;
+        return err;
+    }
     int p2 = 1;
     while (p2 < n_mem) p2 <<= 1;  // n_mem <= 16384 (checked at create when top_k > 32)
     const size_t smem = (size_t)p2 * sizeof(uint64_t);
