@@ -159,7 +159,7 @@ infllm_status validate(const infllm_config* g, char* msg, size_t n) {
     if (g->dtype != INFLLM_F32 && g->dtype != INFLLM_BF16) return bad("dtype must be INFLLM_F32 or INFLLM_BF16");
     if (g->score_mode != INFLLM_SCORE_REPS && g->score_mode != INFLLM_SCORE_REPSUM) return bad("unknown score_mode");
     const int64_t units = g->max_tokens / g->unit_size + 1;
-    if (g->top_k > 32 && units > 16384) return bad("top_k > 32 supports at most 16384 memory units");
+    if (units > 16384) return bad("at most 16384 memory units (max_tokens / unit_size)");
     return INFLLM_OK;
 }
 

@@ -225,45 +225,40 @@ __global__ void __launch_bounds__(SC_THREADS, 2) k_score_topk(Dev D, int n_mem, 
     pdl_wait();
 }
 
-// Top-k of one KV head's unit scores: one CTA of 1024 threads per KV head.  Every warp keeps a
-// running descending top-32 list of the composite keys (score, ~unit) over a strided share of
-// the units (a batch is sorted and merged only when one of its keys beats the list's last entry),
-// then the 32 lists are merged pairwise in shared memory.  Ties go to the lower unit index.
+// Top-k of one KV head's unit scores: one CTA of 1024 threads per KV head sorts the composite
+// keys (score, ~unit) of every eligible unit in shared memory (bitonic network, descending; all
+// threads work on every stage), keeps the first min(k, n_mem) and sorts their ids ascending in
+// one warp.  Ties go to the lower unit index.  Valid for k <= 32.
 constexpr int SEL_THREADS = 1024;
-constexpr int SEL_WARPS = SEL_THREADS / 32;
 
-__global__ void __launch_bounds__(SEL_THREADS) k_select_topk(Dev D, int n_mem) {
-    __shared__ uint64_t lists[SEL_WARPS][32];
+__global__ void __launch_bounds__(SEL_THREADS) k_select_topk(Dev D, int n_mem, int p2) {
+    extern __shared__ uint64_t keys[];
     asm volatile("griddepcontrol.launch_dependents;");
     pdl_wait();  // the unit scores are complete past this point
-    const int hk = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int hk = blockIdx.x;
     const float* sc = D.uscore + (int64_t)hk * D.units_max;
-    uint64_t list = 0;
-    constexpr int B = 4;  // batches of 32 candidates per warp, loads issued together
-    for (int j0 = warp * 32 * B; j0 < n_mem; j0 += SEL_WARPS * 32 * B) {
-        float v[B];
-#pragma unroll
-        for (int u = 0; u < B; ++u) {
-            const int j = j0 + u * 32 + lane;
-            v[u] = j < n_mem ? __ldcg(sc + j) : 0.f;
-        }
-#pragma unroll
-        for (int u = 0; u < B; ++u) {
-            const int j = j0 + u * 32 + lane;
-            list = warp_topk_insert(list, j < n_mem ? make_key(v[u], (uint32_t)j) : 0ull);
-        }
-    }
-    lists[warp][lane] = list;
-#pragma unroll
-    for (int stride = 1; stride < SEL_WARPS; stride *= 2) {
-        __syncthreads();
-        if ((warp % (2 * stride)) == 0) lists[warp][lane] = warp_merge_desc(lists[warp][lane], lists[warp + stride][lane]);
-    }
+    for (int i = threadIdx.x; i < p2; i += blockDim.x) keys[i] = i < n_mem ? make_key(__ldcg(sc + i), (uint32_t)i) : 0ull;
     __syncthreads();
-    if (warp == 0) {
-        const uint64_t m = lists[0][lane];
+    for (int k = 2; k <= p2; k <<= 1) {
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            for (int i = threadIdx.x; i < p2; i += blockDim.x) {
+                const int ixj = i ^ j;
+                if (ixj > i) {
+                    const bool desc = (i & k) == 0;
+                    const uint64_t a = keys[i], b = keys[ixj];
+                    if ((a < b) == desc) {
+                        keys[i] = b;
+                        keys[ixj] = a;
+                    }
+                }
+            }
+            __syncthreads();
+        }
+    }
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
         const int kk = min(D.topk, n_mem);
-        uint64_t sk = (lane < kk) ? (uint64_t)(0xffffffffu - key_index(m)) : 0ull;
+        uint64_t sk = (lane < kk) ? (uint64_t)(0xffffffffu - key_index(keys[lane])) : 0ull;
         sk = warp_sort_desc(sk);  // ascending ids
         if (lane < D.topk) {
             int o = -1;
@@ -406,16 +401,26 @@ cudaError_t launch_select(const Dev& D, int score_mode, int n_mem, int n_qtiles,
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
     if (fast) {
+        int p2 = 1;
+        while (p2 < n_mem) p2 <<= 1;  // n_mem <= units_max <= 16384 (checked at create when top_k > 32)
+        const size_t smem = (size_t)p2 * sizeof(uint64_t);
+        static size_t smem_set = 48 * 1024;
+        if (smem > smem_set) {
+            err = cudaFuncSetAttribute(k_select_topk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (err != cudaSuccess) return err;
+            smem_set = smem;
+        }
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(D.Hkv);
         cfg.blockDim = dim3(SEL_THREADS);
+        cfg.dynamicSmemBytes = smem;
         cfg.stream = st;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
         attr[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        err = cudaLaunchKernelEx(&cfg, k_select_topk, D, n_mem);
+        err = cudaLaunchKernelEx(&cfg, k_select_topk, D, n_mem, p2);
         ++*launches;
         return err;
     }

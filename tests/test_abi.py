@@ -75,7 +75,7 @@ def _cfg(**kw):
     dict(n_q_heads=0), dict(n_q_heads=30), dict(head_dim=96), dict(n_sink=-1), dict(window=0),
     dict(unit_size=0), dict(unit_size=2048), dict(n_reps=0), dict(n_reps=33), dict(n_reps=200, unit_size=128),
     dict(top_k=-1), dict(max_chunk=0), dict(max_tokens=0), dict(rope_base=1.0), dict(dtype=7), dict(score_mode=3),
-    dict(top_k=64, max_tokens=1 << 22),
+    dict(top_k=64, max_tokens=1 << 22), dict(max_tokens=(1 << 21) + 128 * 16384),
 ])
 def test_invalid_configs_are_rejected_before_any_device_work(lib, bad):
     h = ctypes.c_void_p(123)
