@@ -217,48 +217,65 @@ __global__ void __launch_bounds__(SC_THREADS, 2) k_score_topk(Dev D, int n_mem, 
     }
 #pragma unroll
     for (int m = LPU / 2; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
-    if (j < n_mem && sub == 0) D.uscore[(int64_t)hk * D.units_max + j] = acc * D.inv_sqrt_d;
-    (void)do_select;
+    uint64_t cand = 0;
+    if (j < n_mem && sub == 0) {
+        const float sc = acc * D.inv_sqrt_d;
+        D.uscore[(int64_t)hk * D.units_max + j] = sc;
+        cand = make_key(sc, (uint32_t)j);
+    }
+    if (do_select) {  // this CTA's top-32 (composite keys, descending) for the selection kernel
+        __shared__ uint64_t lists[SC_WARPS][32];
+        lists[warp][lane] = warp_sort_desc(cand);
+#pragma unroll
+        for (int stride = 1; stride < SC_WARPS; stride *= 2) {
+            __syncthreads();
+            if ((warp % (2 * stride)) == 0)
+                lists[warp][lane] = warp_merge_desc(lists[warp][lane], lists[warp + stride][lane]);
+        }
+        __syncthreads();
+        if (warp == 0) D.cand[((int64_t)hk * D.score_splits_max + split) * 32 + lane] = lists[0][lane];
+    }
     // Under a programmatic dependent launch this grid may start before the preceding kernel ends;
     // the scores do not depend on it, but this grid must not complete before it (the kernels after
     // this one rely on both).
     pdl_wait();
 }
 
-// Top-k of one KV head's unit scores: one CTA of 1024 threads per KV head sorts the composite
-// keys (score, ~unit) of every eligible unit in shared memory (bitonic network, descending; all
-// threads work on every stage), keeps the first min(k, n_mem) and sorts their ids ascending in
-// one warp.  Ties go to the lower unit index.  Valid for k <= 32.
+// Top-k of one KV head from the scoring CTAs' top-32 lists: one CTA of 1024 threads per KV
+// head; warp w merges lists w, w + 32, ... (loads of a batch issued together), then the 32
+// warp lists are merged pairwise in shared memory.  Ties go to the lower unit index (composite
+// keys).  Valid for k <= 32.
 constexpr int SEL_THREADS = 1024;
+constexpr int SEL_WARPS = SEL_THREADS / 32;
 
-__global__ void __launch_bounds__(SEL_THREADS) k_select_topk(Dev D, int n_mem, int p2) {
-    extern __shared__ uint64_t keys[];
+__global__ void __launch_bounds__(SEL_THREADS) k_select_topk(Dev D, int n_mem, int n_split) {
+    __shared__ uint64_t lists[SEL_WARPS][32];
     asm volatile("griddepcontrol.launch_dependents;");
-    pdl_wait();  // the unit scores are complete past this point
-    const int hk = blockIdx.x;
-    const float* sc = D.uscore + (int64_t)hk * D.units_max;
-    for (int i = threadIdx.x; i < p2; i += blockDim.x) keys[i] = i < n_mem ? make_key(__ldcg(sc + i), (uint32_t)i) : 0ull;
-    __syncthreads();
-    for (int k = 2; k <= p2; k <<= 1) {
-        for (int j = k >> 1; j > 0; j >>= 1) {
-            for (int i = threadIdx.x; i < p2; i += blockDim.x) {
-                const int ixj = i ^ j;
-                if (ixj > i) {
-                    const bool desc = (i & k) == 0;
-                    const uint64_t a = keys[i], b = keys[ixj];
-                    if ((a < b) == desc) {
-                        keys[i] = b;
-                        keys[ixj] = a;
-                    }
-                }
-            }
-            __syncthreads();
+    pdl_wait();  // the candidate lists are complete past this point
+    const int hk = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint64_t* cb = D.cand + (int64_t)hk * D.score_splits_max * 32 + lane;
+    uint64_t m = 0;
+    for (int s0 = warp; s0 < n_split; s0 += SEL_WARPS * 4) {
+        uint64_t b[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int s = s0 + SEL_WARPS * u;
+            b[u] = s < n_split ? __ldcg(cb + (int64_t)s * 32) : 0ull;
         }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (s0 + SEL_WARPS * u < n_split) m = warp_merge_desc(m, b[u]);
     }
-    if (threadIdx.x < 32) {
-        const int lane = threadIdx.x;
+    lists[warp][lane] = m;
+#pragma unroll
+    for (int stride = 1; stride < SEL_WARPS; stride *= 2) {
+        __syncthreads();
+        if ((warp % (2 * stride)) == 0) lists[warp][lane] = warp_merge_desc(lists[warp][lane], lists[warp + stride][lane]);
+    }
+    __syncthreads();
+    if (warp == 0) {
         const int kk = min(D.topk, n_mem);
-        uint64_t sk = (lane < kk) ? (uint64_t)(0xffffffffu - key_index(keys[lane])) : 0ull;
+        uint64_t sk = (lane < kk) ? (uint64_t)(0xffffffffu - key_index(lists[0][lane])) : 0ull;
         sk = warp_sort_desc(sk);  // ascending ids
         if (lane < D.topk) {
             int o = -1;
@@ -401,26 +418,17 @@ cudaError_t launch_select(const Dev& D, int score_mode, int n_mem, int n_qtiles,
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
     if (fast) {
-        int p2 = 1;
-        while (p2 < n_mem) p2 <<= 1;  // n_mem <= units_max <= 16384 (checked at create when top_k > 32)
-        const size_t smem = (size_t)p2 * sizeof(uint64_t);
-        static size_t smem_set = 48 * 1024;
-        if (smem > smem_set) {
-            err = cudaFuncSetAttribute(k_select_topk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-            if (err != cudaSuccess) return err;
-            smem_set = smem;
-        }
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(D.Hkv);
         cfg.blockDim = dim3(SEL_THREADS);
-        cfg.dynamicSmemBytes = smem;
+        cfg.dynamicSmemBytes = 0;
         cfg.stream = st;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
         attr[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        err = cudaLaunchKernelEx(&cfg, k_select_topk, D, n_mem, p2);
+        err = cudaLaunchKernelEx(&cfg, k_select_topk, D, n_mem, n_split);
         ++*launches;
         return err;
     }
