@@ -315,7 +315,8 @@ def query_prefix_sums(qsrc: Callable, c0: int, positions: Sequence[int], cfg: di
     while t0 < stop:
         n = min(block, stop - t0)
         q = qsrc(t0, n).reshape(n, Hkv, G, d)
-        qr = rope(q, (t0 + np.arange(n))[:, None, None], base).sum(axis=2)  # [n, Hkv, d]
+        # sum_h R(i) q_{i,h} = R(i) sum_h q_{i,h}: every head of token i has the same angle
+        qr = rope(q.sum(axis=2), (t0 + np.arange(n))[:, None], base)  # [n, Hkv, d]
         cs = np.cumsum(qr, axis=0) + acc[None]
         while wi < len(want) and want[wi] <= t0 + n:
             out[want[wi]] = cs[want[wi] - t0 - 1].copy()
@@ -336,8 +337,12 @@ def all_reps_linear(qsrc: Callable, ksrc: Callable, c0: int, cfg: dict):
     ends = [S + (j + 1) * U for j in range(nm)]
     P = query_prefix_sums(qsrc, c0, ends + [e + W for e in ends], cfg)
     reps, rhos = [], []
+    kbatch, kb0 = None, 0
     for j, e in enumerate(ends):
-        ku = ksrc(S + j * U, U)  # [U, Hkv, d]
+        if kbatch is None or j >= kb0 + kbatch.shape[0] // U:  # fetch keys 256 units at a time
+            kb0 = j
+            kbatch = ksrc(S + j * U, min(256, nm - j) * U)
+        ku = kbatch[(j - kb0) * U:(j - kb0 + 1) * U]  # [U, Hkv, d]
         per, rr = [], []
         for hk in range(cfg["n_kv_heads"]):
             rho = rep_scores_linear(P[e + W][hk] - P[e][hk], ku[:, hk], S + j * U, base)
@@ -348,8 +353,22 @@ def all_reps_linear(qsrc: Callable, ksrc: Callable, c0: int, cfg: dict):
     return reps, (np.stack(rhos) if rhos else np.zeros((0, cfg["n_kv_heads"], U)))
 
 
+def rep_key_table(ksrc: Callable, reps, n_units: int, cfg: dict) -> np.ndarray:
+    """Raw keys of every unit's representatives: [Hkv, n_units, n_reps, d] (keys fetched 256 units at a time)."""
+    S, U, Hkv, d = cfg["n_sink"], cfg["unit_size"], cfg["n_kv_heads"], cfg["head_dim"]
+    out = np.zeros((Hkv, n_units, cfg["n_reps"], d))
+    for j0 in range(0, n_units, 256):
+        nb = min(256, n_units - j0)
+        kb = ksrc(S + j0 * U, nb * U)
+        for j in range(j0, j0 + nb):
+            ku = kb[(j - j0) * U:(j - j0 + 1) * U]
+            for hk in range(Hkv):
+                out[hk, j] = ku[reps[j][hk], hk]
+    return out
+
+
 def chunk_stateless(qsrc: Callable, ksrc: Callable, vsrc: Callable, c0: int, n: int, cfg: dict,
-                    reps=None, sel_override=None):
+                    reps=None, sel_override=None, rep_keys=None):
     """Recompute chunk [c0, c0+n) from scratch: reps of all eligible units, lookup, attention.
 
     `reps` may be passed in (e.g. the GPU's own representatives, to check the later steps on
@@ -382,12 +401,10 @@ def chunk_stateless(qsrc: Callable, ksrc: Callable, vsrc: Callable, c0: int, n: 
                 res[seg] = cache[key][:, hk]
         return res
 
-    rep_keys = np.zeros((Hkv, nm, cfg["n_reps"], d))  # raw keys of every unit's representatives
-    if k > 0:
-        for j in range(nm):
-            ku = ksrc(S + j * U, U)
-            for hk in range(Hkv):
-                rep_keys[hk, j] = ku[reps[j][hk], hk]
+    if k > 0 and rep_keys is None:
+        rep_keys = rep_key_table(ksrc, reps, nm, cfg)  # raw keys of every unit's representatives
+    elif rep_keys is not None:
+        rep_keys = rep_keys[:, :nm]
     for hk in range(Hkv):
         qg = q[:, hk * G:(hk + 1) * G]
         if nm > 0 and k > 0:
