@@ -206,8 +206,17 @@ class InfLLMLayer:
         self._check(self.L.infllm_get_stats(self.h, ctypes.byref(s)), "infllm_get_stats")
         return s.as_dict()
 
-    def set_profiling(self, on: bool):
-        self._check(self.L.infllm_set_profiling(self.h, 1 if on else 0), "infllm_set_profiling")
+    PROFILE = {"all": 1, "append": 2, "reps": 4, "prep": 8, "select": 16, "attend": 32, "decode": 64}
+
+    def set_profiling(self, on):
+        """on: bool (all kernel classes / off) or an iterable of class names (see PROFILE)."""
+        if isinstance(on, bool) or on is None:
+            mask = 1 if on else 0
+        else:
+            mask = 0
+            for name in on:
+                mask |= self.PROFILE[name]
+        self._check(self.L.infllm_set_profiling(self.h, mask), "infllm_set_profiling")
 
     def set_score_mode(self, mode: str):
         self._check(self.L.infllm_set_score_mode(self.h, SCORE_MODES[mode]), "infllm_set_score_mode")

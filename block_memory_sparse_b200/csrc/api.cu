@@ -50,7 +50,7 @@ struct infllm_ctx {
     bool attended = false;
     int64_t launches = 0;
     // profiling
-    bool profiling = false;
+    int profiling = 0;  // bit mask of kernel classes (1 << Kind) bracketed with events
     std::vector<EventPair> events;
     std::vector<cudaEvent_t> pool;
     double ms[K_NKIND] = {0};
@@ -93,13 +93,13 @@ struct Prof {
     int kind;
     cudaEvent_t a = nullptr;
     Prof(infllm_ctx* c_, int k) : c(c_), kind(k) {
-        if (c->profiling) {
+        if (c->profiling & (1 << kind)) {
             a = get_event(c);
             cudaEventRecord(a, c->stream);
         }
     }
     void done() {
-        if (c->profiling && a) {
+        if (a) {
             cudaEvent_t b = get_event(c);
             cudaEventRecord(b, c->stream);
             c->events.push_back({a, b, kind});
@@ -596,7 +596,8 @@ infllm_status infllm_set_score_mode(infllm_ctx* c, int32_t mode) {
 infllm_status infllm_set_profiling(infllm_ctx* c, int32_t enable) {
     if (!c) return INFLLM_EINVAL;
     collect_events(c);
-    c->profiling = enable != 0;
+    // 1 = every kernel class; otherwise bit (k + 1) selects class k (INFLLM_PROFILE_* in the header)
+    c->profiling = enable == 1 ? ((1 << K_NKIND) - 1) : ((enable >> 1) & ((1 << K_NKIND) - 1));
     for (int k = 0; k < K_NKIND; ++k) {
         c->ms[k] = 0;
         c->cnt[k] = 0;

@@ -152,8 +152,19 @@ infllm_status infllm_get_stats(infllm_ctx* ctx, infllm_stats* out);
  * maintained, so this is valid at any point of a stream. */
 infllm_status infllm_set_score_mode(infllm_ctx* ctx, int32_t score_mode);
 
-/* Record CUDA events around every kernel launch (adds host overhead) and accumulate the
- * device times into infllm_stats.  Toggling clears the accumulated times and counts. */
+/* Record CUDA events around kernel launches and accumulate their device times into
+ * infllm_stats.  enable: 0 = off, INFLLM_PROFILE_ALL = every kernel class, or an OR of the
+ * INFLLM_PROFILE_* class bits below (events break the overlap between consecutive launches, so
+ * profile only the classes being measured).  Any call clears the accumulated times and counts. */
+enum {
+    INFLLM_PROFILE_ALL = 1,
+    INFLLM_PROFILE_APPEND = 2,  /* token store and query block sums */
+    INFLLM_PROFILE_REPS = 4,    /* representative scoring of newly evicted units */
+    INFLLM_PROFILE_PREP = 8,    /* rotated, packed queries of a chunk */
+    INFLLM_PROFILE_SELECT = 16, /* unit scores and top-k */
+    INFLLM_PROFILE_ATTEND = 32, /* chunk attention */
+    INFLLM_PROFILE_DECODE = 64  /* decode attention (tiles and merge) */
+};
 infllm_status infllm_set_profiling(infllm_ctx* ctx, int32_t enable);
 
 /* Human-readable description of the last error on this context ("" if none). */
