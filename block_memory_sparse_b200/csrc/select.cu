@@ -241,6 +241,133 @@ __global__ void __launch_bounds__(SC_THREADS, 2) k_score_topk(Dev D, int n_mem, 
     pdl_wait();
 }
 
+// Rotated sum of the chunk's (or the decode token's) queries of KV head hk into qb[d]:
+// R(W) sum_t sum_h q_{t,h}, from the per-tile partial sums (or the single token's q heads).
+template <typename T>
+__device__ __forceinline__ void rotated_query_sum(const Dev& D, int hk, int n_qtiles, const T* qraw, float* qb) {
+    for (int i = threadIdx.x; i < D.half; i += blockDim.x) {
+        float a = 0.f, b = 0.f;
+        const int n = qraw ? D.G : n_qtiles;
+        for (int t0 = 0; t0 < n; t0 += 8) {
+            float x[8], y[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                x[u] = y[u] = 0.f;
+                if (t0 + u < n) {
+                    if (qraw) {
+                        x[u] = to_f(qraw[(hk * D.G + t0 + u) * D.d + i]);
+                        y[u] = to_f(qraw[(hk * D.G + t0 + u) * D.d + i + D.half]);
+                    } else {
+                        const float* p = D.qbar_part + ((int64_t)hk * D.qtiles_max + t0 + u) * D.d;
+                        x[u] = p[i];
+                        y[u] = p[i + D.half];
+                    }
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                a += x[u];
+                b += y[u];
+            }
+        }
+        const float2 cw = D.cs_W[i];
+        qb[i] = a * cw.x - b * cw.y;
+        qb[i + D.half] = b * cw.x + a * cw.y;
+    }
+}
+
+// Warp-per-32-units scoring.  Grid (n_split, Hkv), 32 * WPC threads; warp w of CTA s scores units
+// [(s * WPC + w) * 32, +32).  Lane l loads 16-byte chunks l, l + 32, ... (C per unit) of every
+// unit's operand -- consecutive lanes read consecutive 16 bytes, so each load instruction reads
+// 512 contiguous bytes -- and multiplies them with the matching slice of the rotated query sum,
+// held in registers.  The 32 partial sums of the warp's 32 units are then transposed across the
+// warp (recursive halving, 31 shuffles) so that lane u ends with unit u's score.  Writes the scores
+// and this CTA's top-32 list for the selection kernel.
+template <typename T, int MODE, int C>
+__global__ void __launch_bounds__(256, 2) k_score_wpu(Dev D, int n_mem, int n_split, int n_qtiles, const T* qraw,
+                                                      int do_select) {
+    __shared__ float qb[128];
+    __shared__ uint64_t lists[8][32];
+    asm volatile("griddepcontrol.launch_dependents;");  // the selection kernel may start its prologue
+    const int split = blockIdx.x, hk = blockIdx.y;
+    rotated_query_sum<T>(D, hk, n_qtiles, qraw, qb);
+    __syncthreads();
+    constexpr int V = MODE == 0 ? (int)(16 / sizeof(T)) : 4;  // elements per 16-byte chunk
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    float qr[C][V];
+#pragma unroll
+    for (int k = 0; k < C; ++k) {
+        const int i0 = ((k * 32 + lane) * V) % D.d;
+#pragma unroll
+        for (int v = 0; v < V; ++v) qr[k][v] = qb[i0 + v];
+    }
+    const int u0 = (split * nw + warp) * 32;
+    const uint4* base = MODE == 0
+        ? reinterpret_cast<const uint4*>((const T*)D.rep_keys + ((int64_t)hk * D.units_max + u0) * D.r * D.d)
+        : reinterpret_cast<const uint4*>(D.repsum + ((int64_t)hk * D.units_max + u0) * D.d);
+    float acc[32];
+    constexpr int UB = C >= 4 ? 4 : 8;  // units per load batch
+#pragma unroll
+    for (int ub = 0; ub < 32; ub += UB) {
+        uint4 raw[UB][C];
+#pragma unroll
+        for (int u = 0; u < UB; ++u)
+#pragma unroll
+            for (int k = 0; k < C; ++k)
+                raw[u][k] = (u0 + ub + u < n_mem) ? __ldg(base + (int64_t)(ub + u) * 32 * C + k * 32 + lane)
+                                                  : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int u = 0; u < UB; ++u) {
+            float a = 0.f;
+#pragma unroll
+            for (int k = 0; k < C; ++k) {
+                if (MODE == 0 && sizeof(T) == 2) {
+                    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw[u][k]);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const float2 f = __bfloat1622float2(h2[c]);
+                        a += f.x * qr[k][2 * c] + f.y * qr[k][2 * c + 1];
+                    }
+                } else {
+                    const float* f = reinterpret_cast<const float*>(&raw[u][k]);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) a += f[c] * qr[k][c];
+                }
+            }
+            acc[ub + u] = a;
+        }
+    }
+    // transpose-reduce: afterwards acc[0] of lane l is the full dot product of unit u0 + l
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) {
+        const bool upper = (lane & m) != 0;
+#pragma unroll
+        for (int i = 0; i < m; ++i) {
+            const float send = upper ? acc[i] : acc[i + m];
+            const float keep = upper ? acc[i + m] : acc[i];
+            acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+        }
+    }
+    const int j = u0 + lane;
+    uint64_t cand = 0;
+    if (j < n_mem) {
+        const float sc = acc[0] * D.inv_sqrt_d;
+        D.uscore[(int64_t)hk * D.units_max + j] = sc;
+        cand = make_key(sc, (uint32_t)j);
+    }
+    if (do_select) {
+        lists[warp][lane] = warp_sort_desc(cand);
+        for (int stride = 1; stride < nw; stride *= 2) {
+            __syncthreads();
+            if ((warp % (2 * stride)) == 0)
+                lists[warp][lane] = warp_merge_desc(lists[warp][lane], lists[warp + stride][lane]);
+        }
+        __syncthreads();
+        if (warp == 0) D.cand[((int64_t)hk * D.score_splits_max + split) * 32 + lane] = lists[0][lane];
+    }
+    pdl_wait();  // this grid must not complete before the preceding kernel (see k_score_topk)
+}
+
 // Top-k of one KV head from the scoring CTAs' top-32 lists: one CTA of 1024 threads per KV
 // head; warp w merges lists w, w + 32, ... (loads of a batch issued together), then the 32
 // warp lists are merged pairwise in shared memory.  Ties go to the lower unit index (composite
@@ -399,20 +526,62 @@ static cudaError_t launch_score(const Dev& D, int lpu, dim3 grid, int n_mem, int
     }
 }
 
+template <typename T, int MODE, int C>
+static cudaError_t launch_wpu1(const Dev& D, dim3 grid, int threads, int n_mem, int n_split, int n_qtiles,
+                               const T* qraw, int do_select, cudaStream_t st, bool pdl) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, k_score_wpu<T, MODE, C>, D, n_mem, n_split, n_qtiles, qraw, do_select);
+}
+
+template <typename T>
+static cudaError_t launch_wpu(const Dev& D, int mode, int C, dim3 grid, int threads, int n_mem, int n_split,
+                              int n_qtiles, const T* qraw, int do_select, cudaStream_t st, bool pdl) {
+    if (mode == 0) {
+        if (C == 1) return launch_wpu1<T, 0, 1>(D, grid, threads, n_mem, n_split, n_qtiles, qraw, do_select, st, pdl);
+        if (C == 2) return launch_wpu1<T, 0, 2>(D, grid, threads, n_mem, n_split, n_qtiles, qraw, do_select, st, pdl);
+        return launch_wpu1<T, 0, 4>(D, grid, threads, n_mem, n_split, n_qtiles, qraw, do_select, st, pdl);
+    }
+    if (C == 1) return launch_wpu1<T, 1, 1>(D, grid, threads, n_mem, n_split, n_qtiles, qraw, do_select, st, pdl);
+    if (C == 2) return launch_wpu1<T, 1, 2>(D, grid, threads, n_mem, n_split, n_qtiles, qraw, do_select, st, pdl);
+    return launch_wpu1<T, 1, 4>(D, grid, threads, n_mem, n_split, n_qtiles, qraw, do_select, st, pdl);
+}
+
 template <typename T>
 cudaError_t launch_select(const Dev& D, int score_mode, int n_mem, int n_qtiles, const void* qraw, cudaStream_t st,
                           int* launches, bool pdl) {
     *launches = 0;
     if (n_mem <= 0 || D.topk <= 0) return cudaSuccess;
-    const int lpu = score_lanes_per_unit(n_mem, D.Hkv);
-    const int per = SC_THREADS / lpu;
-    const int n_split = (n_mem + per - 1) / per;
-    if (n_split > D.score_splits_max) return cudaErrorInvalidValue;
     const int fast = D.topk <= 32;
-    dim3 grid(n_split, D.Hkv);
-    cudaError_t err = score_mode == 0
-                          ? launch_score<T, 0>(D, lpu, grid, n_mem, n_split, n_qtiles, (const T*)qraw, fast, st, pdl)
-                          : launch_score<T, 1>(D, lpu, grid, n_mem, n_split, n_qtiles, (const T*)qraw, fast, st, pdl);
+    // warp-per-32-units scoring when a unit's operand is a whole number of 512-byte rows
+    const int unit_bytes = score_mode == 0 ? D.r * D.d * (int)sizeof(T) : D.d * 4;
+    const int C = unit_bytes % 512 == 0 ? unit_bytes / 512 : 0;
+    int n_split;
+    cudaError_t err;
+    if (C == 1 || C == 2 || C == 4) {
+        int wpc = 8;  // warps per CTA: fewer when that still gives at least one CTA per SM
+        while (wpc > 1 && (int64_t)((n_mem + 32 * wpc - 1) / (32 * wpc)) * D.Hkv < 148) wpc /= 2;
+        n_split = (n_mem + 32 * wpc - 1) / (32 * wpc);
+        if (n_split > D.score_splits_max) return cudaErrorInvalidValue;
+        err = launch_wpu<T>(D, score_mode, C, dim3(n_split, D.Hkv), 32 * wpc, n_mem, n_split, n_qtiles,
+                            (const T*)qraw, fast, st, pdl);
+    } else {
+        const int lpu = score_lanes_per_unit(n_mem, D.Hkv);
+        const int per = SC_THREADS / lpu;
+        n_split = (n_mem + per - 1) / per;
+        if (n_split > D.score_splits_max) return cudaErrorInvalidValue;
+        dim3 grid(n_split, D.Hkv);
+        err = score_mode == 0 ? launch_score<T, 0>(D, lpu, grid, n_mem, n_split, n_qtiles, (const T*)qraw, fast, st, pdl)
+                              : launch_score<T, 1>(D, lpu, grid, n_mem, n_split, n_qtiles, (const T*)qraw, fast, st, pdl);
+    }
     ++*launches;
     if (err != cudaSuccess) return err;
     err = cudaGetLastError();
