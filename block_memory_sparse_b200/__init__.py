@@ -61,6 +61,8 @@ SIGNATURES = {
     "infllm_append_chunk": (ctypes.c_int, [_P, _P, _P, _P, ctypes.c_int32]),
     "infllm_attend_chunk": (ctypes.c_int, [_P, _P, ctypes.c_int32, _P]),
     "infllm_decode_step": (ctypes.c_int, [_P, _P, _P, _P, _P]),
+    "infllm_prefill": (ctypes.c_int, [_P, _P, _P, _P, ctypes.c_int64, ctypes.c_int32, _P]),
+    "infllm_set_launch_chaining": (ctypes.c_int, [_P, ctypes.c_int32]),
     "infllm_get_selection": (ctypes.c_int, [_P, _P]),
     "infllm_get_unit_scores": (ctypes.c_int, [_P, _P, ctypes.c_int32, ctypes.POINTER(ctypes.c_int32)]),
     "infllm_get_reps": (ctypes.c_int, [_P, ctypes.c_int32, ctypes.c_int32, _P]),
@@ -168,6 +170,22 @@ class InfLLMLayer:
         op = _dev_ptr(out, self.dtype, (n, self.Hq, self.d), "out")
         self._check(self.L.infllm_attend_chunk(self.h, qp, n, op), "infllm_attend_chunk")
         return out
+
+    def prefill(self, q, k, v, chunk, out=None):
+        """Whole prompt in chunks of `chunk` tokens (append + attend per chunk, one C call)."""
+        torch = _torch()
+        n = q.shape[0]
+        qp = _dev_ptr(q, self.dtype, (n, self.Hq, self.d), "q")
+        kp = _dev_ptr(k, self.dtype, (n, self.Hkv, self.d), "k")
+        vp = _dev_ptr(v, self.dtype, (n, self.Hkv, self.d), "v")
+        if out is None:
+            out = torch.empty((n, self.Hq, self.d), dtype=self.dtype, device=q.device)
+        op = _dev_ptr(out, self.dtype, (n, self.Hq, self.d), "out")
+        self._check(self.L.infllm_prefill(self.h, qp, kp, vp, n, int(chunk), op), "infllm_prefill")
+        return out
+
+    def set_launch_chaining(self, on: bool):
+        self._check(self.L.infllm_set_launch_chaining(self.h, 1 if on else 0), "infllm_set_launch_chaining")
 
     def decode_step(self, q, k, v, out=None):
         torch = _torch()

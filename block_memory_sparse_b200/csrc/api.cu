@@ -49,6 +49,11 @@ struct infllm_ctx {
     int64_t last_B = 0, last_active = 0;
     bool attended = false;
     int64_t launches = 0;
+    // launch chaining: within one API call every launch after the first may start early
+    // (programmatic dependent launch); the first waits for whatever precedes it on the stream
+    int chaining = 1;   // infllm_set_launch_chaining
+    bool chain = false; // a kernel of the current call has been launched
+    int qpar = 0;       // query buffer the next chunk's packed queries go to
     // profiling
     int profiling = 0;  // bit mask of kernel classes (1 << Kind) bracketed with events
     std::vector<EventPair> events;
@@ -107,6 +112,9 @@ struct Prof {
         }
     }
 };
+
+// Whether the next launch may be chained to the previous one (same API call).
+bool pdl_ok(const infllm_ctx* c) { return c->chaining && c->chain; }
 
 void collect_events(infllm_ctx* c) {
     if (c->events.empty()) return;
@@ -171,15 +179,17 @@ infllm_status append_impl(infllm_ctx* c, const void* q, const void* k, const voi
     const int64_t target = n_mem_at(c0, D.S, D.W, D.U);
     if (target > c->units_done) {
         Prof p(c, K_REPS);
-        CK(launch_reps<T>(D, c->units_done, target, c->stream));
+        CK(launch_reps<T>(D, c->units_done, target, c->stream, pdl_ok(c)));
+        c->chain = true;
         p.done();
         c->launches += 1;
         c->units_done = target;
     }
     Prof p(c, K_APPEND);
-    CK(launch_append<T>(D, k, v, c0, n, c->stream));
+    CK(launch_append<T>(D, k, v, c0, n, c->stream, pdl_ok(c)));
+    c->chain = true;
     int l = 0;
-    CK(launch_ysum<T>(D, q, c0, n, c->stream, &l));
+    CK(launch_ysum<T>(D, q, c0, n, c->stream, &l, pdl_ok(c)));
     p.done();
     c->launches += 1 + l;
     c->tokens = c0 + n;
@@ -193,7 +203,9 @@ template <typename T>
 infllm_status select_impl(infllm_ctx* c, int nm, int n_qtiles, const void* qraw) {
     int l = 0;
     Prof p(c, K_SELECT);
-    CK(launch_select<T>(c->D, c->cfg.score_mode, nm, n_qtiles, qraw, c->stream, &l));
+    const bool pdl = pdl_ok(c);
+    CK(launch_select<T>(c->D, c->cfg.score_mode, nm, n_qtiles, qraw, c->stream, &l, pdl, /*wait_first=*/true));
+    if (l > 0) c->chain = true;
     p.done();
     c->launches += l;
     return INFLLM_OK;
@@ -218,9 +230,12 @@ infllm_status attend_impl(infllm_ctx* c, const void* q, int32_t n, void* out) {
     const int nm = (int)n_mem_at(c0, D.S, D.W, D.U);
     const int kk = std::min(D.topk, nm);
     const int64_t B = (int64_t)D.S + (int64_t)D.U * nm;
+    const int par = c->qpar;
+    c->qpar ^= 1;
     {
         Prof p(c, K_PREP);
-        CK(launch_prep<T>(D, q, c0, n, c->stream));
+        CK(launch_prep<T>(D, q, c0, n, par, c->stream, pdl_ok(c)));
+        c->chain = true;
         p.done();
         c->launches += 1;
     }
@@ -231,10 +246,11 @@ infllm_status attend_impl(infllm_ctx* c, const void* q, int32_t n, void* out) {
     }
     Prof p(c, K_ATTEND);
     if (c->use_tc && sizeof(T) == 2) {
-        CK(launch_attend_tc(D, c0, n, kk, B, out, c->stream, c->tmaps));
+        CK(launch_attend_tc(D, c0, n, kk, B, par, out, c->stream, c->tmaps, pdl_ok(c)));
     } else {
-        CK(launch_attend_simt<T>(D, c0, n, kk, B, out, c->stream));
+        CK(launch_attend_simt<T>(D, c0, n, kk, B, par, out, c->stream, pdl_ok(c)));
     }
+    c->chain = true;
     p.done();
     c->launches += 1;
     record_attend(c, c0, n, nm, kk, B);
@@ -244,19 +260,23 @@ infllm_status attend_impl(infllm_ctx* c, const void* q, int32_t n, void* out) {
 template <typename T>
 infllm_status decode_impl(infllm_ctx* c, const void* q, const void* k, const void* v, void* out) {
     infllm_status s;
+    bool new_reps = false;  // the lookup then needs the representatives just computed
     if (sizeof(T) == 2 && c->use_tc && decode_tc_supported(c->D) && c->D.G <= 8) {
         const Dev& D = c->D;
         const int64_t t = c->tokens;
         const int64_t target = n_mem_at(t, D.S, D.W, D.U);
         if (target > c->units_done) {
             Prof p(c, K_REPS);
-            CK(launch_reps<T>(D, c->units_done, target, c->stream));
+            CK(launch_reps<T>(D, c->units_done, target, c->stream, pdl_ok(c)));
+            c->chain = true;
             p.done();
             c->launches += 1;
             c->units_done = target;
+            new_reps = true;
         }
         Prof p(c, K_APPEND);
-        CK(launch_decode_append(D, q, k, v, t, c->stream));
+        CK(launch_decode_append(D, q, k, v, t, c->stream, pdl_ok(c)));
+        c->chain = true;
         p.done();
         c->launches += 1;
         c->tokens = t + 1;
@@ -281,13 +301,14 @@ infllm_status decode_impl(infllm_ctx* c, const void* q, const void* k, const voi
         if (kk > 0) {
             int l = 0;
             Prof p(c, K_SELECT);
-            CK(launch_select<T>(D, c->cfg.score_mode, nm, 1, q, c->stream, &l, /*pdl=*/true));
+            CK(launch_select<T>(D, c->cfg.score_mode, nm, 1, q, c->stream, &l, pdl_ok(c), new_reps));
+            if (l > 0) c->chain = true;
             p.done();
             c->launches += l;
         }
         Prof p(c, K_DECODE);
         int nt = 0;
-        cudaError_t e = launch_decode_tc(D, q, t, kk, B, out, c->stream, c->tmaps, &nt);
+        cudaError_t e = launch_decode_tc(D, q, t, kk, B, out, c->stream, c->tmaps, &nt, pdl_ok(c));
         if (e != cudaSuccess) return fail(c, INFLLM_ECUDA, "decode launch (%d tiles): %s", nt, cudaGetErrorString(e));
         p.done();
         c->launches += 2;  // tiles + merge
@@ -319,6 +340,7 @@ infllm_status zero_state(infllm_ctx* c) {
     c->attended = false;
     c->last_nmem = c->last_kk = 0;
     c->last_B = c->last_active = 0;
+    c->qpar = 0;
     return INFLLM_OK;
 }
 
@@ -388,8 +410,8 @@ infllm_status create_impl(infllm_ctx* c) {
     AL(D.qbar_part, sizeof(float) * (size_t)D.Hkv * D.qtiles_max * D.d);
     AL(D.cand, sizeof(uint64_t) * (size_t)D.Hkv * D.score_splits_max * 32);
     AL(D.counters, sizeof(unsigned) * 2 * D.Hkv);
-    AL(D.Qm, (size_t)D.Hkv * D.qrows_max * D.d * c->elt);
-    AL(D.Qw, (size_t)D.Hkv * D.qrows_max * D.d * c->elt);
+    AL(D.Qm, (size_t)D.Hkv * 2 * D.qrows_max * D.d * c->elt);  // two buffers, by chunk parity
+    AL(D.Qw, (size_t)D.Hkv * 2 * D.qrows_max * D.d * c->elt);
     AL(D.cs_chunk, sizeof(float2) * (size_t)g.max_chunk * D.half);
     AL(D.dec_part, sizeof(float) * (size_t)D.Hkv * D.dec_splits_max * D.G * (D.d + 2));
     double* invf = nullptr;
@@ -483,6 +505,7 @@ infllm_status infllm_reset(infllm_ctx* c) {
 
 infllm_status infllm_append_chunk(infllm_ctx* c, const void* q, const void* k, const void* v, int32_t n) {
     if (!c) return INFLLM_EINVAL;
+    c->chain = false;
     infllm_status s = check_device_error(c);
     if (s != INFLLM_OK) return s;
     if (n < 0) return fail(c, INFLLM_EINVAL, "append: n = %d < 0", n);
@@ -502,6 +525,7 @@ infllm_status infllm_append_chunk(infllm_ctx* c, const void* q, const void* k, c
 
 infllm_status infllm_attend_chunk(infllm_ctx* c, const void* q, int32_t n, void* out) {
     if (!c) return INFLLM_EINVAL;
+    c->chain = false;
     infllm_status s = check_device_error(c);
     if (s != INFLLM_OK) return s;
     if (!c->pending) return fail(c, INFLLM_ESTATE, "attend: no appended chunk is waiting");
@@ -513,6 +537,7 @@ infllm_status infllm_attend_chunk(infllm_ctx* c, const void* q, int32_t n, void*
 
 infllm_status infllm_decode_step(infllm_ctx* c, const void* q, const void* k, const void* v, void* out) {
     if (!c) return INFLLM_EINVAL;
+    c->chain = false;
     infllm_status s = check_device_error(c);
     if (s != INFLLM_OK) return s;
     if (!q || !k || !v || !out) return fail(c, INFLLM_EINVAL, "decode: null pointer");
@@ -520,6 +545,37 @@ infllm_status infllm_decode_step(infllm_ctx* c, const void* q, const void* k, co
     if (c->tokens + 1 > c->cfg.max_tokens)
         return fail(c, INFLLM_ECAPACITY, "decode: max_tokens = %lld reached", (long long)c->cfg.max_tokens);
     return c->cfg.dtype == INFLLM_BF16 ? decode_impl<__nv_bfloat16>(c, q, k, v, out) : decode_impl<float>(c, q, k, v, out);
+}
+
+infllm_status infllm_prefill(infllm_ctx* c, const void* q, const void* k, const void* v, int64_t n, int32_t chunk,
+                             void* out) {
+    if (!c) return INFLLM_EINVAL;
+    c->chain = false;
+    infllm_status s = check_device_error(c);
+    if (s != INFLLM_OK) return s;
+    if (c->pending && c->pending_n > 0) return fail(c, INFLLM_ESTATE, "prefill: an appended chunk waits for attend");
+    if (n < 0) return fail(c, INFLLM_EINVAL, "prefill: n = %lld < 0", (long long)n);
+    if (chunk < 1 || chunk > c->cfg.max_chunk)
+        return fail(c, INFLLM_EINVAL, "prefill: chunk = %d not in [1, max_chunk = %d]", chunk, c->cfg.max_chunk);
+    if (c->tokens + n > c->cfg.max_tokens)
+        return fail(c, INFLLM_ECAPACITY, "prefill: %lld + %lld tokens exceed max_tokens = %lld", (long long)c->tokens,
+                    (long long)n, (long long)c->cfg.max_tokens);
+    if (n == 0) return INFLLM_OK;
+    if (!q || !k || !v || !out) return fail(c, INFLLM_EINVAL, "prefill: null pointer");
+    const size_t qrow = (size_t)c->D.Hq * c->D.d * c->elt, krow = (size_t)c->D.Hkv * c->D.d * c->elt;
+    for (int64_t t0 = 0; t0 < n; t0 += chunk) {
+        const int m = (int)std::min<int64_t>(chunk, n - t0);
+        const char* qc = (const char*)q + t0 * qrow;
+        if (c->cfg.dtype == INFLLM_BF16) {
+            s = append_impl<__nv_bfloat16>(c, qc, (const char*)k + t0 * krow, (const char*)v + t0 * krow, m);
+            if (s == INFLLM_OK) s = attend_impl<__nv_bfloat16>(c, qc, m, (char*)out + t0 * qrow);
+        } else {
+            s = append_impl<float>(c, qc, (const char*)k + t0 * krow, (const char*)v + t0 * krow, m);
+            if (s == INFLLM_OK) s = attend_impl<float>(c, qc, m, (char*)out + t0 * qrow);
+        }
+        if (s != INFLLM_OK) return s;
+    }
+    return INFLLM_OK;
 }
 
 infllm_status infllm_get_selection(infllm_ctx* c, int32_t* host_sel) {
@@ -590,6 +646,12 @@ infllm_status infllm_set_score_mode(infllm_ctx* c, int32_t mode) {
     if (!c) return INFLLM_EINVAL;
     if (mode != INFLLM_SCORE_REPS && mode != INFLLM_SCORE_REPSUM) return fail(c, INFLLM_EINVAL, "unknown score_mode %d", mode);
     c->cfg.score_mode = mode;
+    return INFLLM_OK;
+}
+
+infllm_status infllm_set_launch_chaining(infllm_ctx* c, int32_t enable) {
+    if (!c) return INFLLM_EINVAL;
+    c->chaining = enable ? 1 : 0;
     return INFLLM_OK;
 }
 

@@ -19,8 +19,11 @@ constexpr int SIMT_ROWS = 8;   // packed query rows per CTA (one per warp)
 constexpr int SIMT_KT = 32;    // keys per smem tile (one per lane)
 
 template <typename T>
-__global__ void __launch_bounds__(256) k_attn_simt(Dev D, int64_t c0, int n, int kk, int64_t B, T* __restrict__ out) {
+__global__ void __launch_bounds__(256) k_attn_simt(Dev D, int64_t c0, int n, int kk, int64_t B, int par,
+                                                   T* __restrict__ out) {
     extern __shared__ float sm[];
+    pdl_wait();  // late kernel: selection, packed queries and keys are complete past this point
+    pdl_trigger();
     const int d = D.d;
     float* qm_s = sm;                                  // [ROWS][d]
     float* qw_s = qm_s + SIMT_ROWS * d;                // [ROWS][d]
@@ -42,8 +45,8 @@ __global__ void __launch_bounds__(256) k_attn_simt(Dev D, int64_t c0, int n, int
     const bool valid = tl < n;
     const int64_t t = c0 + tl;
     if (valid) {  // rows past the packed tiles (rows % 8 != 0) are never read
-        const T* Qm = (const T*)D.Qm + ((int64_t)hk * D.qrows_max + R) * d;
-        const T* Qw = (const T*)D.Qw + ((int64_t)hk * D.qrows_max + R) * d;
+        const T* Qm = (const T*)D.Qm + (((int64_t)hk * 2 + par) * D.qrows_max + R) * d;
+        const T* Qw = (const T*)D.Qw + (((int64_t)hk * 2 + par) * D.qrows_max + R) * d;
         for (int i = lane; i < d; i += 32) {
             qm_s[warp * d + i] = to_f(Qm[i]);
             qw_s[warp * d + i] = to_f(Qw[i]);
@@ -119,7 +122,8 @@ __global__ void __launch_bounds__(256) k_attn_simt(Dev D, int64_t c0, int n, int
 }
 
 template <typename T>
-cudaError_t launch_attend_simt(const Dev& D, int64_t c0, int n, int kk, int64_t B, void* out, cudaStream_t st) {
+cudaError_t launch_attend_simt(const Dev& D, int64_t c0, int n, int kk, int64_t B, int par, void* out, cudaStream_t st,
+                               bool pdl) {
     if (n <= 0) return cudaSuccess;
     const int tiles = (n + D.qt - 1) / D.qt;
     const int rows = tiles * D.qt * D.G;
@@ -129,11 +133,11 @@ cudaError_t launch_attend_simt(const Dev& D, int64_t c0, int n, int kk, int64_t 
         cudaError_t e = cudaFuncSetAttribute(k_attn_simt<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
-    k_attn_simt<T><<<grid, 256, smem, st>>>(D, c0, n, kk, B, (T*)out);
-    return cudaGetLastError();
+    return launch_k(k_attn_simt<T>, grid, dim3(256), smem, st, pdl, D, c0, n, kk, B, par, (T*)out);
 }
 
-template cudaError_t launch_attend_simt<float>(const Dev&, int64_t, int, int, int64_t, void*, cudaStream_t);
-template cudaError_t launch_attend_simt<__nv_bfloat16>(const Dev&, int64_t, int, int, int64_t, void*, cudaStream_t);
+template cudaError_t launch_attend_simt<float>(const Dev&, int64_t, int, int, int64_t, int, void*, cudaStream_t, bool);
+template cudaError_t launch_attend_simt<__nv_bfloat16>(const Dev&, int64_t, int, int, int64_t, int, void*, cudaStream_t,
+                                                       bool);
 
 }  // namespace infllm

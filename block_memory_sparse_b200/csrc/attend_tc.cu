@@ -59,7 +59,7 @@ struct TileInfo {
 };
 
 struct Plan {
-    int a, hk, kk, nst, tpu, nut, nwt, NT, S_eff;
+    int a, hk, kk, nst, tpu, nut, nwt, NT, S_eff, par;
     int64_t t_hi, B, win_len;
     const int* sel;  // shared-memory copy; -1 marks an id that failed its range check
 
@@ -98,7 +98,7 @@ __device__ void producer(const TcMaps& maps, const Plan& P, const Dev& D, uint8_
     ptx::prefetch_tmap(&maps.kraw);
     ptx::prefetch_tmap(&maps.krot);
     ptx::prefetch_tmap(&maps.v);
-    const int y = P.a * BM;
+    const int y = P.par * (int)D.qrows_max + P.a * BM;
     ptx::mbar_expect_tx(&bars->q, 4 * HALF);
     ptx::tma_load_3d(sm + OFF_QM, &maps.qm, &bars->q, 0, y, P.hk);
     ptx::tma_load_3d(sm + OFF_QM + HALF, &maps.qm, &bars->q, 64, y, P.hk);
@@ -305,7 +305,7 @@ __device__ void softmax_role(const Plan& P, const Dev& D, uint8_t* sm, Bars* bar
 }
 
 __global__ void __launch_bounds__(NTHREADS, 1)
-    k_attn_tc(const __grid_constant__ TcMaps maps, Dev D, int64_t c0, int n, int kk, int64_t B,
+    k_attn_tc(const __grid_constant__ TcMaps maps, Dev D, int64_t c0, int n, int kk, int64_t B, int par,
               __nv_bfloat16* __restrict__ out) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -315,6 +315,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     Plan P;
     P.a = gridDim.x - 1 - blockIdx.x;  // query tiles with more keys start first
     P.hk = blockIdx.y;
+    P.par = par;
     P.kk = kk;
     P.B = B;
     {
@@ -330,14 +331,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     P.NT = P.nst + P.nut + P.nwt;
 
     int* sel_s = reinterpret_cast<int*>(sm + OFF_SEL);
-    for (int u = threadIdx.x; u < kk; u += blockDim.x) {
-        int j = D.sel[P.hk * D.topk + u];
-        if (j < 0 || (int64_t)D.S + (int64_t)(j + 1) * D.U > B) {
-            set_err(D, ERR_SEL_RANGE);
-            j = -1;
-        }
-        sel_s[u] = j;
-    }
     P.sel = sel_s;
     if (threadIdx.x == 0) {
         ptx::mbar_init(&bars->q, 1);
@@ -357,6 +350,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (warp == 1) {
         ptx::tmem_alloc(&bars->tmem, TMEM_COLS);
         ptx::tmem_relinquish();
+    }
+    // Late kernel: the selection, the packed queries and this chunk's keys are complete past the
+    // wait; the next chunk's store-side kernels may start once every CTA is here.
+    pdl_wait();
+    pdl_trigger();
+    for (int u = threadIdx.x; u < kk; u += blockDim.x) {
+        int j = D.sel[P.hk * D.topk + u];
+        if (j < 0 || (int64_t)D.S + (int64_t)(j + 1) * D.U > B) {
+            set_err(D, ERR_SEL_RANGE);
+            j = -1;
+        }
+        sel_s[u] = j;
     }
     ptx::tc_fence_before();
     __syncthreads();
@@ -424,12 +429,12 @@ bool make_tc_maps(const Dev& D, void* out) {
     return encode_3d(&m->kraw, D.Kraw, (uint64_t)D.T_max, (uint64_t)D.Hkv) &&
            encode_3d(&m->krot, D.Krot, (uint64_t)D.T_max, (uint64_t)D.Hkv) &&
            encode_3d(&m->v, D.V, (uint64_t)D.T_max, (uint64_t)D.Hkv) &&
-           encode_3d(&m->qm, D.Qm, (uint64_t)D.qrows_max, (uint64_t)D.Hkv) &&
-           encode_3d(&m->qw, D.Qw, (uint64_t)D.qrows_max, (uint64_t)D.Hkv);
+           encode_3d(&m->qm, D.Qm, 2 * (uint64_t)D.qrows_max, (uint64_t)D.Hkv) &&
+           encode_3d(&m->qw, D.Qw, 2 * (uint64_t)D.qrows_max, (uint64_t)D.Hkv);
 }
 
-cudaError_t launch_attend_tc(const Dev& D, int64_t c0, int n, int kk, int64_t B, void* out, cudaStream_t st,
-                             const void* tmaps) {
+cudaError_t launch_attend_tc(const Dev& D, int64_t c0, int n, int kk, int64_t B, int par, void* out, cudaStream_t st,
+                             const void* tmaps, bool pdl) {
     if (n <= 0) return cudaSuccess;
     static bool attr_set = false;
     if (!attr_set) {
@@ -438,10 +443,8 @@ cudaError_t launch_attend_tc(const Dev& D, int64_t c0, int n, int kk, int64_t B,
         attr_set = true;
     }
     const int tiles = (n + D.qt - 1) / D.qt;
-    dim3 grid(tiles, D.Hkv);
-    k_attn_tc<<<grid, NTHREADS, SMEM_BYTES, st>>>(*reinterpret_cast<const TcMaps*>(tmaps), D, c0, n, kk, B,
-                                                  (__nv_bfloat16*)out);
-    return cudaGetLastError();
+    return launch_k(k_attn_tc, dim3(tiles, D.Hkv), dim3(NTHREADS), SMEM_BYTES, st, pdl,
+                    *reinterpret_cast<const TcMaps*>(tmaps), D, c0, n, kk, B, par, (__nv_bfloat16*)out);
 }
 
 }  // namespace infllm

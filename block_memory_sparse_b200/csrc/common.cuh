@@ -33,10 +33,11 @@ struct Dev {
     float* qbar_part;     // [Hkv][qtiles_max][d] per-tile raw query sums
     uint64_t* cand;       // [Hkv][score_splits_max][32] top-k candidate lists
     unsigned* counters;   // [Hkv] arrival counters (last-block-done)
-    // rotated, packed queries of the current chunk: [Hkv][rows][d] (rows tile-ordered)
+    // rotated, packed queries of a chunk: [Hkv][2][qrows_max][d] (two buffers alternating by chunk
+    // parity, so the next chunk's queries can be prepared while this chunk's attention runs)
     void* Qm;             // R(W) q  (sink / memory frame)
     void* Qw;             // R(t) q  (window frame)
-    int64_t qrows_max;    // rows capacity per kv head
+    int64_t qrows_max;    // rows per buffer and kv head
     int qt;               // queries per 128-row tile (128 / G, or 1 when G > 128)
     // position tables
     const double* inv_freq;  // [half] theta_i in fp64
@@ -55,6 +56,21 @@ struct Dev {
     // error word (host-mapped)
     int* err;
 };
+
+// ---- programmatic dependent launch -------------------------------------------------------
+// Kernels of one stream are chained with programmatic dependent launch.  Two kinds:
+//   early: pdl_trigger() at entry, pdl_hold() at exit.  The body runs while the preceding
+//          kernel may still run; it may read only data of kernels before the last "late" kernel.
+//   late:  pdl_wait() at entry (after a prologue that reads no predecessor data), then
+//          pdl_trigger().  Past the wait every earlier kernel of the stream is complete.
+// A kernel launched without the attribute treats both instructions as no-ops.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+// End of an early kernel: one thread of the first CTA waits, so the grid completes only after
+// its predecessor has (completion stays transitive along the chain); the other CTAs leave freely.
+__device__ __forceinline__ void pdl_hold() {
+    if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && threadIdx.x == 0) pdl_wait();
+}
 
 enum ErrBits : int {
     ERR_SEL_RANGE = 1,     // a selected unit id outside [0, n_mem)
@@ -163,6 +179,23 @@ __device__ __forceinline__ float2 cs_abs(const double2* tab, int half, int64_t t
 __host__ __device__ __forceinline__ int64_t n_mem_at(int64_t c0, int S, int W, int U) {
     int64_t x = c0 - (int64_t)W - (int64_t)S;
     return x > 0 ? x / U : 0;
+}
+
+// Launch `kernel` on `st`, with programmatic dependent launch when `pdl` is set.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl,
+                            Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
 }
 
 }  // namespace infllm

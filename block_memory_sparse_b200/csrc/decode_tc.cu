@@ -44,7 +44,7 @@ __global__ void __launch_bounds__(DTHREADS) k_decode_append(Dev D, const __nv_bf
                                                             const __nv_bfloat16* __restrict__ k,
                                                             const __nv_bfloat16* __restrict__ v, int64_t t) {
     __shared__ float2 cs[DHD / 2];
-    asm volatile("griddepcontrol.launch_dependents;");  // the lookup kernel may start now
+    pdl_trigger();  // early kernel: the lookup may start now (it reads none of these stores)
     const int hk = blockIdx.x;
     for (int i = threadIdx.x; i < D.half; i += blockDim.x) {
         cs[i] = cs_abs(D.cs_abs3, D.half, t, i);
@@ -87,6 +87,7 @@ __global__ void __launch_bounds__(DTHREADS) k_decode_append(Dev D, const __nv_bf
             y[i + D.half] += s2 * c.x + s1 * c.y;
         }
     }
+    pdl_hold();
 }
 
 struct DTile {
@@ -158,7 +159,7 @@ __global__ void __launch_bounds__(DTHREADS) k_decode_attn(const __grid_constant_
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, tg = lane & 3;
     const int G = D.G;
-    asm volatile("griddepcontrol.launch_dependents;");  // the merge kernel may start its prologue
+    pdl_trigger();  // the merge kernel may start its prologue
     if (tid == 0) {
         ptx::mbar_init(bar, 1);
         ptx::mbar_fence_init();
@@ -303,7 +304,8 @@ constexpr int MERGE_BATCH = 32;
 __global__ void __launch_bounds__(MERGE_SLICES * DHD) k_decode_merge(Dev D, __nv_bfloat16* __restrict__ out, int NT) {
     __shared__ float ml[2][MERGE_SLICES * MERGE_BATCH];
     __shared__ float red[2][MERGE_SLICES][DHD];
-    pdl_wait();  // the tile partials are complete past this point
+    pdl_wait();     // the tile partials are complete past this point
+    pdl_trigger();  // every earlier kernel is complete: the next step's store kernels may start
     const int h = blockIdx.x, hk = blockIdx.y, G = D.G, d = DHD;
     const int dim = threadIdx.x % DHD, z = threadIdx.x / DHD;
     const float* base = D.dec_part + (int64_t)hk * D.dec_splits_max * G * (d + 2) + (int64_t)h * (d + 2);
@@ -350,14 +352,13 @@ __global__ void __launch_bounds__(MERGE_SLICES * DHD) k_decode_merge(Dev D, __nv
 bool decode_tc_supported(const Dev& D) { return D.d == DHD && D.G <= MAXG && D.topk <= 32; }
 
 cudaError_t launch_decode_append(const Dev& D, const void* q, const void* k, const void* v, int64_t t,
-                                 cudaStream_t st) {
-    k_decode_append<<<D.Hkv, DTHREADS, 0, st>>>(D, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
-                                               (const __nv_bfloat16*)v, t);
-    return cudaGetLastError();
+                                 cudaStream_t st, bool pdl) {
+    return launch_k(k_decode_append, dim3(D.Hkv), dim3(DTHREADS), 0, st, pdl, D, (const __nv_bfloat16*)q,
+                    (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, t);
 }
 
 cudaError_t launch_decode_tc(const Dev& D, const void* q, int64_t t, int kk, int64_t B, void* out, cudaStream_t st,
-                             const void* tmaps, int* n_tiles_out) {
+                             const void* tmaps, int* n_tiles_out, bool pdl) {
     const int S_eff = (int)(D.S < t + 1 ? D.S : t + 1);
     const int64_t win = t - B + 1;
     const int NT = (S_eff + DK - 1) / DK + kk * ((D.U + DK - 1) / DK) + (int)((win + DK - 1) / DK);
@@ -369,27 +370,11 @@ cudaError_t launch_decode_tc(const Dev& D, const void* q, int64_t t, int kk, int
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(NT, D.Hkv);
-    cfg.blockDim = dim3(DTHREADS);
-    cfg.dynamicSmemBytes = DSMEM;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, k_decode_attn, *reinterpret_cast<const TcMaps*>(tmaps), D,
-                                       (const __nv_bfloat16*)q, (__nv_bfloat16*)out, t, kk, B, NT);
+    cudaError_t e = launch_k(k_decode_attn, dim3(NT, D.Hkv), dim3(DTHREADS), DSMEM, st, pdl,
+                             *reinterpret_cast<const TcMaps*>(tmaps), D, (const __nv_bfloat16*)q, (__nv_bfloat16*)out,
+                             t, kk, B, NT);
     if (e != cudaSuccess) return e;
-    cudaLaunchConfig_t mcfg = {};
-    mcfg.gridDim = dim3(D.G, D.Hkv);
-    mcfg.blockDim = dim3(MERGE_SLICES * DHD);
-    mcfg.dynamicSmemBytes = 0;
-    mcfg.stream = st;
-    mcfg.attrs = attr;
-    mcfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&mcfg, k_decode_merge, D, (__nv_bfloat16*)out, NT);
+    return launch_k(k_decode_merge, dim3(D.G, D.Hkv), dim3(MERGE_SLICES * DHD), 0, st, pdl, D, (__nv_bfloat16*)out, NT);
 }
 
 }  // namespace infllm

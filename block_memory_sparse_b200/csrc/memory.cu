@@ -14,6 +14,7 @@ namespace infllm {
 template <typename T>
 __global__ void k_append(Dev D, const T* __restrict__ k, const T* __restrict__ v, int64_t c0) {
     extern __shared__ float2 cs_sh[];
+    pdl_trigger();  // early kernel: reads only the inputs and constant tables
     const int tl = blockIdx.x;
     const int64_t t = c0 + tl;
     for (int i = threadIdx.x; i < D.half; i += blockDim.x) {
@@ -40,6 +41,7 @@ __global__ void k_append(Dev D, const T* __restrict__ k, const T* __restrict__ v
         V[dst + i] = vs[i];
         V[dst + i + D.half] = vs[i + D.half];
     }
+    pdl_hold();
 }
 
 // Y[b][hk] += sum over the chunk's tokens t in block b of sum_{h in group} R(t - s_b) q_{t,h}.
@@ -49,6 +51,7 @@ __global__ void k_append(Dev D, const T* __restrict__ k, const T* __restrict__ v
 template <typename T>
 __global__ void __launch_bounds__(1024) k_ysum(Dev D, const T* __restrict__ q, int64_t c0, int n, int64_t b0) {
     extern __shared__ float red[];  // [warps][d]
+    pdl_trigger();  // early kernel: the blocks it updates hold no position a running kernel reads
     constexpr int V = 16 / sizeof(T);
     constexpr int HB = 4;
     const int64_t b = b0 + blockIdx.x;
@@ -119,6 +122,7 @@ __global__ void __launch_bounds__(1024) k_ysum(Dev D, const T* __restrict__ q, i
         for (int w = 0; w < nw; ++w) acc += red[w * D.d + j];
         D.Y[(b * D.Hkv + hk) * D.d + j] += acc;
     }
+    pdl_hold();
 }
 
 // Representatives of units [j0, j0 + gridDim.x) for kv head blockIdx.y, 256 threads.
@@ -132,6 +136,7 @@ __global__ void __launch_bounds__(256) k_reps(Dev D, int64_t j0) {
     float* rho = sm + D.d;          // [U]
     float* part = rho + D.U;        // [4][d] partial window sums
     __shared__ int ids[32];
+    pdl_trigger();  // early kernel: reads block sums and keys of positions before the chunk
     const int64_t j = j0 + blockIdx.x;
     const int hk = blockIdx.y;
     const int64_t e = (int64_t)D.S + (j + 1) * D.U;
@@ -258,43 +263,43 @@ __global__ void __launch_bounds__(256) k_reps(Dev D, int64_t j0) {
         }
         rs[i] = s;
     }
+    pdl_hold();
 }
 
 // ---- launchers ----------------------------------------------------------------------------
 
 template <typename T>
-cudaError_t launch_append(const Dev& D, const void* k, const void* v, int64_t c0, int n, cudaStream_t st) {
+cudaError_t launch_append(const Dev& D, const void* k, const void* v, int64_t c0, int n, cudaStream_t st, bool pdl) {
     if (n <= 0) return cudaSuccess;
-    k_append<T><<<n, 256, D.half * sizeof(float2), st>>>(D, (const T*)k, (const T*)v, c0);
-    return cudaGetLastError();
+    return launch_k(k_append<T>, dim3(n), dim3(256), D.half * sizeof(float2), st, pdl, D, (const T*)k, (const T*)v, c0);
 }
 
 template <typename T>
-cudaError_t launch_ysum(const Dev& D, const void* q, int64_t c0, int n, cudaStream_t st, int* launches) {
+cudaError_t launch_ysum(const Dev& D, const void* q, int64_t c0, int n, cudaStream_t st, int* launches, bool pdl) {
     const int64_t lo = c0 > D.S ? c0 : (int64_t)D.S;
     const int64_t hi = c0 + n;
     if (hi <= lo) return cudaSuccess;
     const int64_t b0 = (lo - D.S) / D.gblk, b1 = (hi - 1 - D.S) / D.gblk;
     const int threads = 1024;  // (half / V) octets x tokens
     dim3 grid((unsigned)(b1 - b0 + 1), D.Hkv);
-    k_ysum<T><<<grid, threads, (threads / 32) * D.d * sizeof(float), st>>>(D, (const T*)q, c0, n, b0);
     ++*launches;
-    return cudaGetLastError();
+    return launch_k(k_ysum<T>, grid, dim3(threads), (threads / 32) * D.d * sizeof(float), st, pdl, D, (const T*)q, c0,
+                    n, b0);
 }
 
 template <typename T>
-cudaError_t launch_reps(const Dev& D, int64_t j0, int64_t j1, cudaStream_t st) {
+cudaError_t launch_reps(const Dev& D, int64_t j0, int64_t j1, cudaStream_t st, bool pdl) {
     if (j1 <= j0) return cudaSuccess;
     dim3 grid((unsigned)(j1 - j0), D.Hkv);
-    k_reps<T><<<grid, 256, (D.d + D.U + (256 / D.half) * D.d) * sizeof(float), st>>>(D, j0);
-    return cudaGetLastError();
+    return launch_k(k_reps<T>, grid, dim3(256), (D.d + D.U + (256 / D.half) * D.d) * sizeof(float), st, pdl, D, j0);
 }
 
-template cudaError_t launch_append<float>(const Dev&, const void*, const void*, int64_t, int, cudaStream_t);
-template cudaError_t launch_append<__nv_bfloat16>(const Dev&, const void*, const void*, int64_t, int, cudaStream_t);
-template cudaError_t launch_ysum<float>(const Dev&, const void*, int64_t, int, cudaStream_t, int*);
-template cudaError_t launch_ysum<__nv_bfloat16>(const Dev&, const void*, int64_t, int, cudaStream_t, int*);
-template cudaError_t launch_reps<float>(const Dev&, int64_t, int64_t, cudaStream_t);
-template cudaError_t launch_reps<__nv_bfloat16>(const Dev&, int64_t, int64_t, cudaStream_t);
+template cudaError_t launch_append<float>(const Dev&, const void*, const void*, int64_t, int, cudaStream_t, bool);
+template cudaError_t launch_append<__nv_bfloat16>(const Dev&, const void*, const void*, int64_t, int, cudaStream_t,
+                                                  bool);
+template cudaError_t launch_ysum<float>(const Dev&, const void*, int64_t, int, cudaStream_t, int*, bool);
+template cudaError_t launch_ysum<__nv_bfloat16>(const Dev&, const void*, int64_t, int, cudaStream_t, int*, bool);
+template cudaError_t launch_reps<float>(const Dev&, int64_t, int64_t, cudaStream_t, bool);
+template cudaError_t launch_reps<__nv_bfloat16>(const Dev&, int64_t, int64_t, cudaStream_t, bool);
 
 }  // namespace infllm

@@ -19,10 +19,13 @@ namespace infllm {
 // queries [a*qt, a*qt + qt); row r of a tile is (head hg = r / qt, query a*qt + r % qt).
 // Thread = (vector v: elements [vV, vV+V) of each half, row group): 16-byte loads and stores,
 // four rows per load batch.  Also writes each tile's raw query sum over its rows
-// (fixed-order reduction).
+// (fixed-order reduction).  An early kernel: it may run while the previous chunk's attention
+// reads the other query buffer, and while this chunk's keys are stored, so it takes the
+// (cos, sin)(t theta_i) of its queries from the fp64 digit tables itself.
 template <typename T>
-__global__ void __launch_bounds__(256) k_prep(Dev D, const T* __restrict__ q, int n) {
-    extern __shared__ float red[];
+__global__ void __launch_bounds__(256) k_prep(Dev D, const T* __restrict__ q, int64_t c0, int n, int par) {
+    extern __shared__ float red[];  // [row groups][d], then (cos, sin) [qt][half]
+    pdl_trigger();
     constexpr int V = 16 / sizeof(T);
     constexpr int RB = 4;
     union Vec { uint4 u; T h[V]; };
@@ -31,8 +34,15 @@ __global__ void __launch_bounds__(256) k_prep(Dev D, const T* __restrict__ q, in
     const int nv = D.half / V;
     const int o = threadIdx.x % nv, rg = threadIdx.x / nv, nrg = blockDim.x / nv;
     const int i0 = o * V;
-    T* Qm = (T*)D.Qm + ((int64_t)hk * D.qrows_max + (int64_t)a * rows) * D.d;
-    T* Qw = (T*)D.Qw + ((int64_t)hk * D.qrows_max + (int64_t)a * rows) * D.d;
+    float2* cs_sh = reinterpret_cast<float2*>(red + nrg * D.d);
+    for (int x = threadIdx.x; x < D.qt * D.half; x += blockDim.x) {
+        const int tl = a * D.qt + x / D.half;
+        cs_sh[x] = tl < n ? cs_abs(D.cs_abs3, D.half, c0 + tl, x % D.half) : make_float2(1.f, 0.f);
+    }
+    __syncthreads();
+    const int64_t qbase = ((int64_t)hk * 2 + par) * D.qrows_max + (int64_t)a * rows;
+    T* Qm = (T*)D.Qm + qbase * D.d;
+    T* Qw = (T*)D.Qw + qbase * D.d;
     float2 cw[V];
 #pragma unroll
     for (int e = 0; e < V; ++e) cw[e] = D.cs_W[i0 + e];
@@ -54,7 +64,7 @@ __global__ void __launch_bounds__(256) k_prep(Dev D, const T* __restrict__ q, in
                 x1[u].u = *reinterpret_cast<const uint4*>(src + i0);
                 x2[u].u = *reinterpret_cast<const uint4*>(src + i0 + D.half);
 #pragma unroll
-                for (int e = 0; e < V; ++e) ct[u][e] = D.cs_chunk[(int64_t)tl * D.half + i0 + e];
+                for (int e = 0; e < V; ++e) ct[u][e] = cs_sh[(tl - a * D.qt) * D.half + i0 + e];
             }
         }
 #pragma unroll
@@ -92,6 +102,7 @@ __global__ void __launch_bounds__(256) k_prep(Dev D, const T* __restrict__ q, in
         for (int g = 0; g < nrg; ++g) acc += red[g * D.d + j];
         D.qbar_part[((int64_t)hk * D.qtiles_max + a) * D.d + j] = acc;
     }
+    pdl_hold();
 }
 
 // 16-byte vector of the score operand, converted to floats.
@@ -125,9 +136,10 @@ constexpr int SC_WARPS = SC_THREADS / 32;
 
 template <typename T, int MODE, int LPU>
 __global__ void __launch_bounds__(SC_THREADS, 2) k_score_topk(Dev D, int n_mem, int n_split, int n_qtiles,
-                                                           const T* qraw, int do_select) {
+                                                           const T* qraw, int do_select, int wait_first) {
     __shared__ float qb[128];
-    asm volatile("griddepcontrol.launch_dependents;");  // the selection kernel may start its prologue
+    if (wait_first) pdl_wait();  // the query sums (and the representatives) come from the kernels before
+    pdl_trigger();               // the selection kernel may start its prologue
     const int split = blockIdx.x, hk = blockIdx.y;
     for (int i = threadIdx.x; i < D.half; i += blockDim.x) {
         float a = 0.f, b = 0.f;
@@ -235,10 +247,9 @@ __global__ void __launch_bounds__(SC_THREADS, 2) k_score_topk(Dev D, int n_mem, 
         __syncthreads();
         if (warp == 0) D.cand[((int64_t)hk * D.score_splits_max + split) * 32 + lane] = lists[0][lane];
     }
-    // Under a programmatic dependent launch this grid may start before the preceding kernel ends;
-    // the scores do not depend on it, but this grid must not complete before it (the kernels after
-    // this one rely on both).
-    pdl_wait();
+    // Without wait_first this grid may run while the preceding kernel runs (the scores do not
+    // depend on it), but it must not complete before it: the kernels after rely on both.
+    if (!wait_first) pdl_hold();
 }
 
 // Rotated sum of the chunk's (or the decode token's) queries of KV head hk into qb[d]:
@@ -285,10 +296,11 @@ __device__ __forceinline__ void rotated_query_sum(const Dev& D, int hk, int n_qt
 // and this CTA's top-32 list for the selection kernel.
 template <typename T, int MODE, int C>
 __global__ void __launch_bounds__(256, 2) k_score_wpu(Dev D, int n_mem, int n_split, int n_qtiles, const T* qraw,
-                                                      int do_select) {
+                                                      int do_select, int wait_first) {
     __shared__ float qb[128];
     __shared__ uint64_t lists[8][32];
-    asm volatile("griddepcontrol.launch_dependents;");  // the selection kernel may start its prologue
+    if (wait_first) pdl_wait();  // as in k_score_topk
+    pdl_trigger();
     const int split = blockIdx.x, hk = blockIdx.y;
     rotated_query_sum<T>(D, hk, n_qtiles, qraw, qb);
     __syncthreads();
@@ -365,7 +377,7 @@ __global__ void __launch_bounds__(256, 2) k_score_wpu(Dev D, int n_mem, int n_sp
         __syncthreads();
         if (warp == 0) D.cand[((int64_t)hk * D.score_splits_max + split) * 32 + lane] = lists[0][lane];
     }
-    pdl_wait();  // this grid must not complete before the preceding kernel (see k_score_topk)
+    if (!wait_first) pdl_hold();  // this grid must not complete before its predecessor (see k_score_topk)
 }
 
 // Top-k of one KV head from the scoring CTAs' top-32 lists: one CTA of 1024 threads per KV
@@ -377,8 +389,8 @@ constexpr int SEL_WARPS = SEL_THREADS / 32;
 
 __global__ void __launch_bounds__(SEL_THREADS) k_select_topk(Dev D, int n_mem, int n_split) {
     __shared__ uint64_t lists[SEL_WARPS][32];
-    asm volatile("griddepcontrol.launch_dependents;");
-    pdl_wait();  // the candidate lists are complete past this point
+    pdl_trigger();  // the attention kernel after this one is a late kernel as well
+    pdl_wait();     // the candidate lists are complete past this point
     const int hk = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint64_t* cb = D.cand + (int64_t)hk * D.score_splits_max * 32 + lane;
     uint64_t m = 0;
@@ -479,15 +491,19 @@ __global__ void __launch_bounds__(1024) k_topk_sort(Dev D, int n_mem, int p2) {
 // ---- launchers ----------------------------------------------------------------------------
 
 template <typename T>
-cudaError_t launch_prep(const Dev& D, const void* q, int64_t c0, int n, cudaStream_t st) {
-    (void)c0;
+cudaError_t launch_prep(const Dev& D, const void* q, int64_t c0, int n, int par, cudaStream_t st, bool pdl) {
     if (n <= 0) return cudaSuccess;
     const int tiles = (n + D.qt - 1) / D.qt;
     const int threads = 256;
     const int nv = D.half / (16 / (int)sizeof(T));
-    dim3 grid(tiles, D.Hkv);
-    k_prep<T><<<grid, threads, (threads / nv) * D.d * sizeof(float), st>>>(D, (const T*)q, n);
-    return cudaGetLastError();
+    const size_t smem = (threads / nv) * D.d * sizeof(float) + (size_t)D.qt * D.half * sizeof(float2);
+    static bool attr_set = false;  // up to 80 KB (one KV head per q head: 128 queries a tile)
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(k_prep<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    return launch_k(k_prep<T>, dim3(tiles, D.Hkv), dim3(threads), smem, st, pdl, D, (const T*)q, c0, n, par);
 }
 
 // Lanes per unit: the fewest that still give at least one CTA per SM (148).
@@ -499,66 +515,50 @@ int score_lanes_per_unit(int n_mem, int Hkv) {
 
 template <typename T, int MODE, int LPU>
 static cudaError_t launch_score1(const Dev& D, dim3 grid, int n_mem, int n_split, int n_qtiles, const T* qraw,
-                                 int do_select, cudaStream_t st, bool pdl) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
-    cfg.blockDim = dim3(SC_THREADS);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, k_score_topk<T, MODE, LPU>, D, n_mem, n_split, n_qtiles, qraw, do_select);
+                                 int do_select, cudaStream_t st, bool pdl, int wait_first) {
+    return launch_k(k_score_topk<T, MODE, LPU>, grid, dim3(SC_THREADS), 0, st, pdl, D, n_mem, n_split, n_qtiles, qraw,
+                    do_select, wait_first);
 }
 
 template <typename T, int MODE>
 static cudaError_t launch_score(const Dev& D, int lpu, dim3 grid, int n_mem, int n_split, int n_qtiles, const T* qraw,
-                                int do_select, cudaStream_t st, bool pdl) {
+                                int do_select, cudaStream_t st, bool pdl, int wf) {
     switch (lpu) {
-        case 1: return launch_score1<T, MODE, 1>(D, grid, n_mem, n_split, n_qtiles, qraw, do_select, st, pdl);
-        case 2: return launch_score1<T, MODE, 2>(D, grid, n_mem, n_split, n_qtiles, qraw, do_select, st, pdl);
-        case 4: return launch_score1<T, MODE, 4>(D, grid, n_mem, n_split, n_qtiles, qraw, do_select, st, pdl);
-        case 8: return launch_score1<T, MODE, 8>(D, grid, n_mem, n_split, n_qtiles, qraw, do_select, st, pdl);
-        case 16: return launch_score1<T, MODE, 16>(D, grid, n_mem, n_split, n_qtiles, qraw, do_select, st, pdl);
-        default: return launch_score1<T, MODE, 32>(D, grid, n_mem, n_split, n_qtiles, qraw, do_select, st, pdl);
+        case 1: return launch_score1<T, MODE, 1>(D, grid, n_mem, n_split, n_qtiles, qraw, do_select, st, pdl, wf);
+        case 2: return launch_score1<T, MODE, 2>(D, grid, n_mem, n_split, n_qtiles, qraw, do_select, st, pdl, wf);
+        case 4: return launch_score1<T, MODE, 4>(D, grid, n_mem, n_split, n_qtiles, qraw, do_select, st, pdl, wf);
+        case 8: return launch_score1<T, MODE, 8>(D, grid, n_mem, n_split, n_qtiles, qraw, do_select, st, pdl, wf);
+        case 16: return launch_score1<T, MODE, 16>(D, grid, n_mem, n_split, n_qtiles, qraw, do_select, st, pdl, wf);
+        default: return launch_score1<T, MODE, 32>(D, grid, n_mem, n_split, n_qtiles, qraw, do_select, st, pdl, wf);
     }
 }
 
 template <typename T, int MODE, int C>
 static cudaError_t launch_wpu1(const Dev& D, dim3 grid, int threads, int n_mem, int n_split, int n_qtiles,
-                               const T* qraw, int do_select, cudaStream_t st, bool pdl) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
-    cfg.blockDim = dim3(threads);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, k_score_wpu<T, MODE, C>, D, n_mem, n_split, n_qtiles, qraw, do_select);
+                               const T* qraw, int do_select, cudaStream_t st, bool pdl, int wait_first) {
+    return launch_k(k_score_wpu<T, MODE, C>, grid, dim3(threads), 0, st, pdl, D, n_mem, n_split, n_qtiles, qraw,
+                    do_select, wait_first);
 }
 
 template <typename T>
 static cudaError_t launch_wpu(const Dev& D, int mode, int C, dim3 grid, int threads, int n_mem, int n_split,
-                              int n_qtiles, const T* qraw, int do_select, cudaStream_t st, bool pdl) {
+                              int n_qtiles, const T* qraw, int do_select, cudaStream_t st, bool pdl,
+                              int wf) {
     if (mode == 0) {
-        if (C == 1) return launch_wpu1<T, 0, 1>(D, grid, threads, n_mem, n_split, n_qtiles, qraw, do_select, st, pdl);
-        if (C == 2) return launch_wpu1<T, 0, 2>(D, grid, threads, n_mem, n_split, n_qtiles, qraw, do_select, st, pdl);
-        return launch_wpu1<T, 0, 4>(D, grid, threads, n_mem, n_split, n_qtiles, qraw, do_select, st, pdl);
+        if (C == 1) return launch_wpu1<T, 0, 1>(D, grid, threads, n_mem, n_split, n_qtiles, qraw, do_select, st, pdl, wf);
+        if (C == 2) return launch_wpu1<T, 0, 2>(D, grid, threads, n_mem, n_split, n_qtiles, qraw, do_select, st, pdl, wf);
+        return launch_wpu1<T, 0, 4>(D, grid, threads, n_mem, n_split, n_qtiles, qraw, do_select, st, pdl, wf);
     }
-    if (C == 1) return launch_wpu1<T, 1, 1>(D, grid, threads, n_mem, n_split, n_qtiles, qraw, do_select, st, pdl);
-    if (C == 2) return launch_wpu1<T, 1, 2>(D, grid, threads, n_mem, n_split, n_qtiles, qraw, do_select, st, pdl);
-    return launch_wpu1<T, 1, 4>(D, grid, threads, n_mem, n_split, n_qtiles, qraw, do_select, st, pdl);
+    if (C == 1) return launch_wpu1<T, 1, 1>(D, grid, threads, n_mem, n_split, n_qtiles, qraw, do_select, st, pdl, wf);
+    if (C == 2) return launch_wpu1<T, 1, 2>(D, grid, threads, n_mem, n_split, n_qtiles, qraw, do_select, st, pdl, wf);
+    return launch_wpu1<T, 1, 4>(D, grid, threads, n_mem, n_split, n_qtiles, qraw, do_select, st, pdl, wf);
 }
 
 template <typename T>
 cudaError_t launch_select(const Dev& D, int score_mode, int n_mem, int n_qtiles, const void* qraw, cudaStream_t st,
-                          int* launches, bool pdl) {
+                          int* launches, bool pdl, bool wait_first) {
     *launches = 0;
+    const int wf = wait_first ? 1 : 0;
     if (n_mem <= 0 || D.topk <= 0) return cudaSuccess;
     const int fast = D.topk <= 32;
     // warp-per-32-units scoring when a unit's operand is a whole number of 512-byte rows
@@ -572,32 +572,23 @@ cudaError_t launch_select(const Dev& D, int score_mode, int n_mem, int n_qtiles,
         n_split = (n_mem + 32 * wpc - 1) / (32 * wpc);
         if (n_split > D.score_splits_max) return cudaErrorInvalidValue;
         err = launch_wpu<T>(D, score_mode, C, dim3(n_split, D.Hkv), 32 * wpc, n_mem, n_split, n_qtiles,
-                            (const T*)qraw, fast, st, pdl);
+                            (const T*)qraw, fast, st, pdl, wf);
     } else {
         const int lpu = score_lanes_per_unit(n_mem, D.Hkv);
         const int per = SC_THREADS / lpu;
         n_split = (n_mem + per - 1) / per;
         if (n_split > D.score_splits_max) return cudaErrorInvalidValue;
         dim3 grid(n_split, D.Hkv);
-        err = score_mode == 0 ? launch_score<T, 0>(D, lpu, grid, n_mem, n_split, n_qtiles, (const T*)qraw, fast, st, pdl)
-                              : launch_score<T, 1>(D, lpu, grid, n_mem, n_split, n_qtiles, (const T*)qraw, fast, st, pdl);
+        err = score_mode == 0
+                  ? launch_score<T, 0>(D, lpu, grid, n_mem, n_split, n_qtiles, (const T*)qraw, fast, st, pdl, wf)
+                  : launch_score<T, 1>(D, lpu, grid, n_mem, n_split, n_qtiles, (const T*)qraw, fast, st, pdl, wf);
     }
     ++*launches;
     if (err != cudaSuccess) return err;
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
     if (fast) {
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(D.Hkv);
-        cfg.blockDim = dim3(SEL_THREADS);
-        cfg.dynamicSmemBytes = 0;
-        cfg.stream = st;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[0].val.programmaticStreamSerializationAllowed = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        err = cudaLaunchKernelEx(&cfg, k_select_topk, D, n_mem, n_split);
+        err = launch_k(k_select_topk, dim3(D.Hkv), dim3(SEL_THREADS), 0, st, pdl, D, n_mem, n_split);
         ++*launches;
         return err;
     }
@@ -613,9 +604,10 @@ cudaError_t launch_select(const Dev& D, int score_mode, int n_mem, int n_qtiles,
     return cudaGetLastError();
 }
 
-template cudaError_t launch_prep<float>(const Dev&, const void*, int64_t, int, cudaStream_t);
-template cudaError_t launch_prep<__nv_bfloat16>(const Dev&, const void*, int64_t, int, cudaStream_t);
-template cudaError_t launch_select<float>(const Dev&, int, int, int, const void*, cudaStream_t, int*, bool);
-template cudaError_t launch_select<__nv_bfloat16>(const Dev&, int, int, int, const void*, cudaStream_t, int*, bool);
+template cudaError_t launch_prep<float>(const Dev&, const void*, int64_t, int, int, cudaStream_t, bool);
+template cudaError_t launch_prep<__nv_bfloat16>(const Dev&, const void*, int64_t, int, int, cudaStream_t, bool);
+template cudaError_t launch_select<float>(const Dev&, int, int, int, const void*, cudaStream_t, int*, bool, bool);
+template cudaError_t launch_select<__nv_bfloat16>(const Dev&, int, int, int, const void*, cudaStream_t, int*, bool,
+                                                  bool);
 
 }  // namespace infllm

@@ -10,8 +10,5 @@ struct TcMaps {
     CUtensorMap kraw, krot, v, qm, qw;
 };
 
-// Programmatic dependent launch: wait for the preceding kernel in the stream (no-op when the
-// kernel was launched without the attribute).
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 }  // namespace infllm

@@ -125,6 +125,19 @@ infllm_status infllm_append_chunk(infllm_ctx* ctx, const void* q, const void* k,
  * Errors: ESTATE (no matching append), EINVAL. */
 infllm_status infllm_attend_chunk(infllm_ctx* ctx, const void* q, int32_t n, void* out);
 
+/* Whole-prompt prefill: n tokens (q [n][Hq][d], k, v [n][Hkv][d], out [n][Hq][d]) in chunks
+ * of `chunk` tokens (the last one ragged), each chunk appended and then attended exactly as
+ * infllm_append_chunk + infllm_attend_chunk would, in one call.  Chunk-wise pre-filling with
+ * per-chunk unit lookup follows "InfLLM: Training-Free Long-Context Extrapolation for LLMs
+ * with an Efficient Context Memory" (OpenReview rebuttal, Q2; the guide's "Memory Efficiency"
+ * section); this entry point adds no arithmetic of its own.  Because every input is in place
+ * when the call starts, the kernels of chunk c+1 that store its keys and pack its queries are
+ * chained to (and overlap) chunk c's attention.  Results are identical to the per-chunk calls.
+ * Errors: EINVAL (null pointer with n > 0, chunk not in [1, max_chunk], n < 0), ESTATE (an
+ * appended chunk still waits for its attend), ECAPACITY (tokens + n > max_tokens). */
+infllm_status infllm_prefill(infllm_ctx* ctx, const void* q, const void* k, const void* v,
+                             int64_t n, int32_t chunk, void* out);
+
 /* One decode step: append one token (q [1][Hq][d], k, v [1][Hkv][d]) and attend it
  * (split-KV kernel with a log-sum-exp merge).  out [1][Hq][d]. */
 infllm_status infllm_decode_step(infllm_ctx* ctx, const void* q, const void* k, const void* v,
@@ -166,6 +179,12 @@ enum {
     INFLLM_PROFILE_DECODE = 64  /* decode attention (tiles and merge) */
 };
 infllm_status infllm_set_profiling(infllm_ctx* ctx, int32_t enable);
+
+/* Launch chaining (default on): inside one call, every kernel launch after the first is a
+ * programmatic dependent launch, so a kernel that does not need its predecessor's results
+ * starts while that predecessor runs; the first launch of a call always waits for the work
+ * before it on the stream.  enable = 0 launches every kernel plainly (same results). */
+infllm_status infllm_set_launch_chaining(infllm_ctx* ctx, int32_t enable);
 
 /* Human-readable description of the last error on this context ("" if none). */
 const char* infllm_last_error(infllm_ctx* ctx);
