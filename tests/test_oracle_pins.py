@@ -348,6 +348,29 @@ def test_streaming_equals_stateless_recomputation():
     assert infos[-1]["n_mem"] >= 15
 
 
+def test_batched_linear_reps_and_key_table_past_256_units():
+    # the summed-query form fetches keys 256 units at a time: more than 256 units here, against
+    # the plain double loop of the streaming layer and a direct gather of the representative keys
+    cfg = small_cfg(n_q_heads=2, n_kv_heads=1, head_dim=8, n_sink=2, window=8, unit_size=4, n_reps=2)
+    T = 2 + 4 * 300 + 8 + 4
+    q, k, v = rand_stream(cfg, T, seed=7)
+    layer = O.OracleLayer(cfg, rep_method="plain")
+    for c0 in range(0, T, 128):
+        n = min(128, T - c0)
+        layer.append_chunk(q[c0:c0 + n], k[c0:c0 + n], v[c0:c0 + n])
+    layer._evict_to(T)
+    nu = len(layer.reps)
+    assert nu > 256
+    reps, rho = O.all_reps_linear(lambda t0, n: q[t0:t0 + n], lambda t0, n: k[t0:t0 + n], T, cfg)
+    assert len(reps) == nu
+    for j in range(nu):
+        assert reps[j] == layer.reps[j]
+        assert np.max(np.abs(rho[j] - layer.rep_scores[j])) <= 1e-12 * np.max(np.abs(rho[j]))
+    table = O.rep_key_table(lambda t0, n: k[t0:t0 + n], reps, nu, cfg)
+    for j in (0, 255, 256, nu - 1):
+        assert np.array_equal(table[0, j], k[[2 + 4 * j + m for m in reps[j][0]], 0])
+
+
 def test_representatives_brute_force_ties():
     # integer-valued q/k with d=2 at positions multiple of 2*pi are not available, so force ties by
     # duplicated keys: equal keys at different positions differ only by rotation; use W so that the
