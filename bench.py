@@ -176,6 +176,25 @@ def gen_full(w, torch, device):
     return q, k, v
 
 
+ATTN_PROFILE = os.path.join(ROOT, "profiles", "k_attn_tc_mistral_128k.md")
+ATTN_SOURCE = os.path.join(ROOT, "block_memory_sparse_b200", "csrc", "attend_tc.cu")
+
+
+def attn_traffic():
+    """DRAM bytes per attention launch from the committed ncu summary, or None when the kernel
+    source has changed since the counters were taken (its sha256 is recorded in the summary)."""
+    import hashlib
+    import re
+    try:
+        txt = open(ATTN_PROFILE).read()
+        want = re.search(r"attend_tc\.cu sha256: ([0-9a-f]{64})", txt).group(1)
+        traffic = float(re.search(r"dram bytes per launch: ([0-9.eE+]+)", txt).group(1))
+    except (OSError, AttributeError, ValueError):
+        return None
+    have = hashlib.sha256(open(ATTN_SOURCE, "rb").read()).hexdigest()
+    return traffic if have == want else None
+
+
 def run_ours(args, rank, world):
     import torch
     from block_memory_sparse_b200 import InfLLMLayer
@@ -241,8 +260,10 @@ def run_ours(args, rank, world):
     if tc:
         peak = P["bf16_sust"]
         roof = {"bound": "tensor", "achieved": achieved_tf, "peak": peak, "unit": "TFLOP/s",
-                "frac": (achieved_tf / peak) if achieved_tf else None, "traffic": None,
-                "kernel": "attention (tcgen05)", "peak_source": f"{P['src']} bf16 sustained"}
+                "frac": (achieved_tf / peak) if achieved_tf else None, "traffic": attn_traffic(),
+                "kernel": "attention (tcgen05)", "peak_source": f"{P['src']} bf16 sustained",
+                "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of one steady-chunk launch "
+                                  "(profiles/k_attn_tc_mistral_128k.md); null if the kernel changed since"}
     else:
         # CUDA-core fp32 FMA path: 148 SMs x 128 FP32 lanes x 2 flop x max SM clock
         peak = 148 * 128 * 2 * P["sm_max"] * 1e6 / 1e12
@@ -365,7 +386,7 @@ def run_decode(args, torch, device, stream, local):
     fsum = torch.empty((), dtype=torch.float32, device=device)
 
     def flush_l2():  # read 256 MB (> 126 MB L2): leaves clean lines, so no write-back lands in the step
-        torch.sum(flush, out=fsum)
+        torch.sum(flush, dim=0, out=fsum)
     for mi, mode in enumerate(("reps", "repsum")):
         layer.set_score_mode(mode)
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
@@ -463,7 +484,7 @@ def run_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="mistral_128k", choices=["mistral_128k", "llama3_128k", "needle_256k"])
