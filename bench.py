@@ -366,6 +366,8 @@ def run_decode(args, torch, device, stream, local):
     single-token steps, each timed with CUDA events after an L2 flush."""
     from block_memory_sparse_b200 import InfLLMLayer
     w = synth.WORKLOADS["decode_1m"]
+    if args.decode_units:  # a smaller memory (profiling captures)
+        w = w.replace(n_tokens=w.n_sink + args.decode_units * w.unit_size + w.window)
     steps = min(w.decode_steps, args.decode_steps)
     P = peaks()
     out = {}
@@ -424,7 +426,8 @@ def run_decode(args, torch, device, stream, local):
     del qkv, flush
     torch.cuda.empty_cache()
     out["build_s"] = build_s
-    out["workload"] = (f"{w.name}: 8192 units x 128 + 128 sinks + 4096 window = {w.n_tokens} tokens built, then "
+    units = (w.n_tokens - w.n_sink - w.window) // w.unit_size
+    out["workload"] = (f"{w.name}: {units} units x 128 + 128 sinks + 4096 window = {w.n_tokens} tokens built, then "
                        f"{steps} single-token steps per scoring mode (tokens continue across modes); L2 flushed "
                        f"(256 MB read) before each timed step")
     return out
@@ -489,6 +492,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="mistral_128k", choices=["mistral_128k", "llama3_128k", "needle_256k"])
     ap.add_argument("--decode-steps", type=int, default=256)
+    ap.add_argument("--decode-units", type=int, default=0, help="memory units of the decode workload (0: 8192)")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")

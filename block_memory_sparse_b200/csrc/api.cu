@@ -53,7 +53,12 @@ struct infllm_ctx {
     // (programmatic dependent launch); the first waits for whatever precedes it on the stream
     int chaining = 1;   // infllm_set_launch_chaining
     bool chain = false; // a kernel of the current call has been launched
-    int qpar = 0;       // query buffer the next chunk's packed queries go to
+    // lookups so far: lookup L packs its queries into slot L % 3, sums them into buffer L % 2 and
+    // writes its selection to buffer L % 2 (so a lookup can run while the previous attention reads)
+    int64_t nlook = 0;
+    int last_sel = 0;   // selection buffer of the last attended chunk or token
+    int32_t* sel_base = nullptr;
+    float* qbar_base = nullptr;
     // profiling
     int profiling = 0;  // bit mask of kernel classes (1 << Kind) bracketed with events
     std::vector<EventPair> events;
@@ -171,11 +176,20 @@ infllm_status validate(const infllm_config* g, char* msg, size_t n) {
     return INFLLM_OK;
 }
 
+// The state of lookup L: its selection buffer and query-sum buffer in a copy of the device view.
+Dev lookup_dev(const infllm_ctx* c, int64_t L) {
+    Dev D = c->D;
+    D.sel = c->sel_base + (size_t)(L & 1) * D.Hkv * std::max(1, D.topk);
+    D.qbar_part = c->qbar_base + (size_t)(L & 1) * D.Hkv * D.qtiles_max * D.d;
+    return D;
+}
+
+// a1 + a2 for tokens [tokens, tokens + n): representatives of every unit that becomes eligible
+// at the chunk start (they use queries before it only), then the chunk's stores.
 template <typename T>
-infllm_status append_impl(infllm_ctx* c, const void* q, const void* k, const void* v, int32_t n) {
+infllm_status stage_store(infllm_ctx* c, const void* q, const void* k, const void* v, int32_t n) {
     const Dev& D = c->D;
     const int64_t c0 = c->tokens;
-    // representatives of every unit that becomes eligible at c0 (uses queries < c0 only)
     const int64_t target = n_mem_at(c0, D.S, D.W, D.U);
     if (target > c->units_done) {
         Prof p(c, K_REPS);
@@ -193,32 +207,73 @@ infllm_status append_impl(infllm_ctx* c, const void* q, const void* k, const voi
     p.done();
     c->launches += 1 + l;
     c->tokens = c0 + n;
-    c->pending = true;
-    c->pending_n = n;
-    c->pending_c0 = c0;
     return INFLLM_OK;
 }
 
+// Packed, rotated queries of chunk [c0, c0 + n) for lookup L, and their per-tile sums.
 template <typename T>
-infllm_status select_impl(infllm_ctx* c, int nm, int n_qtiles, const void* qraw) {
+infllm_status stage_prep(infllm_ctx* c, const void* q, int64_t c0, int32_t n, int64_t L) {
+    Prof p(c, K_PREP);
+    CK(launch_prep<T>(lookup_dev(c, L), q, c0, n, (int)(L % 3), c->stream, pdl_ok(c)));
+    c->chain = true;
+    p.done();
+    c->launches += 1;
+    return INFLLM_OK;
+}
+
+// a3: unit scores and top-k of lookup L.  wait_first: the scoring needs its predecessor's results.
+template <typename T>
+infllm_status stage_select(infllm_ctx* c, int64_t L, int nm, int n_qtiles, const void* qraw, bool wait_first) {
     int l = 0;
     Prof p(c, K_SELECT);
-    const bool pdl = pdl_ok(c);
-    CK(launch_select<T>(c->D, c->cfg.score_mode, nm, n_qtiles, qraw, c->stream, &l, pdl, /*wait_first=*/true));
+    CK(launch_select<T>(lookup_dev(c, L), c->cfg.score_mode, nm, n_qtiles, qraw, c->stream, &l, pdl_ok(c),
+                        wait_first));
     if (l > 0) c->chain = true;
     p.done();
     c->launches += l;
     return INFLLM_OK;
 }
 
-void record_attend(infllm_ctx* c, int64_t c0, int n, int nm, int kk, int64_t B) {
+void record_attend(infllm_ctx* c, int64_t L, int64_t c0, int n, int nm, int kk, int64_t B) {
     c->last_nmem = nm;
     c->last_kk = kk;
     c->last_B = B;
+    c->last_sel = (int)(L & 1);
     const int64_t t = c0 + n - 1;
     const int64_t s_eff = std::min<int64_t>(c->cfg.n_sink, t + 1);
     c->last_active = s_eff + (int64_t)kk * c->cfg.unit_size + std::max<int64_t>(0, t - B + 1);
     c->attended = true;
+}
+
+// a4: attention of chunk [c0, c0 + n) with lookup L's packed queries and selection.
+template <typename T>
+infllm_status stage_attend(infllm_ctx* c, int64_t L, int64_t c0, int32_t n, void* out) {
+    const Dev D = lookup_dev(c, L);
+    const int nm = (int)n_mem_at(c0, D.S, D.W, D.U);
+    const int kk = std::min(D.topk, nm);
+    const int64_t B = (int64_t)D.S + (int64_t)D.U * nm;
+    Prof p(c, K_ATTEND);
+    if (c->use_tc && sizeof(T) == 2) {
+        CK(launch_attend_tc(D, c0, n, kk, B, (int)(L % 3), out, c->stream, c->tmaps, pdl_ok(c)));
+    } else {
+        CK(launch_attend_simt<T>(D, c0, n, kk, B, (int)(L % 3), out, c->stream, pdl_ok(c)));
+    }
+    c->chain = true;
+    p.done();
+    c->launches += 1;
+    record_attend(c, L, c0, n, nm, kk, B);
+    return INFLLM_OK;
+}
+
+template <typename T>
+infllm_status append_impl(infllm_ctx* c, const void* q, const void* k, const void* v, int32_t n) {
+    const int64_t c0 = c->tokens;
+    infllm_status s = stage_store<T>(c, q, k, v, n);
+    if (s != INFLLM_OK) return s;
+    c->pending = true;
+    c->pending_n = n;
+    c->pending_c0 = c0;
+    return INFLLM_OK;
 }
 
 template <typename T>
@@ -227,34 +282,53 @@ infllm_status attend_impl(infllm_ctx* c, const void* q, int32_t n, void* out) {
     const int64_t c0 = c->pending_c0;
     c->pending = false;
     if (n == 0) return INFLLM_OK;
+    const int64_t L = c->nlook++;
     const int nm = (int)n_mem_at(c0, D.S, D.W, D.U);
-    const int kk = std::min(D.topk, nm);
-    const int64_t B = (int64_t)D.S + (int64_t)D.U * nm;
-    const int par = c->qpar;
-    c->qpar ^= 1;
-    {
-        Prof p(c, K_PREP);
-        CK(launch_prep<T>(D, q, c0, n, par, c->stream, pdl_ok(c)));
-        c->chain = true;
-        p.done();
-        c->launches += 1;
+    infllm_status s = stage_prep<T>(c, q, c0, n, L);
+    if (s == INFLLM_OK && std::min(D.topk, nm) > 0) s = stage_select<T>(c, L, nm, (n + D.qt - 1) / D.qt, nullptr, true);
+    if (s == INFLLM_OK) s = stage_attend<T>(c, L, c0, n, out);
+    return s;
+}
+
+// A whole prompt, one chunk ahead: after the first chunk the stream runs
+//   attend(c-1) | store + pack (c+1) | lookup (c) | attend (c) | store + pack (c+2) | ...
+// The lookup of chunk c reads only results of kernels before attend(c-1) (its representatives and
+// query sums were made a chunk earlier), so it is chained to run alongside attend(c-1); the store
+// side of chunk c+1 runs there as well.  Three query slots and two selection / query-sum buffers
+// keep the overlapping chunks apart.  Every store side after the second follows an attention (a
+// late kernel), so it starts only once the chunks before are complete; the second follows the
+// first lookup, or is a plain launch.
+template <typename T>
+infllm_status prefill_impl(infllm_ctx* c, const char* q, const char* k, const char* v, int64_t n, int32_t chunk,
+                           char* out) {
+    const Dev& D = c->D;
+    const size_t qrow = (size_t)D.Hq * D.d * c->elt, krow = (size_t)D.Hkv * D.d * c->elt;
+    const int64_t N = (n + chunk - 1) / chunk, L0 = c->nlook, t0 = c->tokens;
+    auto len = [&](int64_t i) { return (int32_t)std::min<int64_t>(chunk, n - i * chunk); };
+    auto store_pack = [&](int64_t i) {
+        const int64_t off = i * chunk;
+        infllm_status s = stage_store<T>(c, q + off * qrow, k + off * krow, v + off * krow, len(i));
+        return s == INFLLM_OK ? stage_prep<T>(c, q + off * qrow, t0 + off, len(i), L0 + i) : s;
+    };
+    auto lookup = [&](int64_t i, bool wait_first) {
+        const int64_t c0 = t0 + i * chunk;
+        const int nm = (int)n_mem_at(c0, D.S, D.W, D.U);
+        if (std::min(D.topk, nm) == 0) return INFLLM_OK;
+        return stage_select<T>(c, L0 + i, nm, (len(i) + D.qt - 1) / D.qt, nullptr, wait_first);
+    };
+    infllm_status s = store_pack(0);
+    const int64_t before = c->launches;
+    if (s == INFLLM_OK) s = lookup(0, true);
+    // chunk 1's store side (representatives from chunk 0's block sums) must see chunk 0 complete:
+    // the first lookup waited for it; without one, chunk 1's first kernel is a plain launch
+    if (c->launches == before) c->chain = false;
+    for (int64_t i = 0; i < N && s == INFLLM_OK; ++i) {
+        if (i + 1 < N) s = store_pack(i + 1);
+        if (s == INFLLM_OK && i > 0) s = lookup(i, false);
+        if (s == INFLLM_OK) s = stage_attend<T>(c, L0 + i, t0 + i * chunk, len(i), out + i * chunk * qrow);
     }
-    const int n_qtiles = (n + D.qt - 1) / D.qt;
-    if (kk > 0) {
-        infllm_status s = select_impl<T>(c, nm, n_qtiles, nullptr);
-        if (s != INFLLM_OK) return s;
-    }
-    Prof p(c, K_ATTEND);
-    if (c->use_tc && sizeof(T) == 2) {
-        CK(launch_attend_tc(D, c0, n, kk, B, par, out, c->stream, c->tmaps, pdl_ok(c)));
-    } else {
-        CK(launch_attend_simt<T>(D, c0, n, kk, B, par, out, c->stream, pdl_ok(c)));
-    }
-    c->chain = true;
-    p.done();
-    c->launches += 1;
-    record_attend(c, c0, n, nm, kk, B);
-    return INFLLM_OK;
+    c->nlook = L0 + N;
+    return s;
 }
 
 template <typename T>
@@ -287,36 +361,44 @@ infllm_status decode_impl(infllm_ctx* c, const void* q, const void* k, const voi
         s = append_impl<T>(c, q, k, v, 1);
         if (s != INFLLM_OK) return s;
     }
-    const Dev& D = c->D;
     const int64_t t = c->pending_c0;
     c->pending = false;
-    const int nm = (int)n_mem_at(t, D.S, D.W, D.U);
-    const int kk = std::min(D.topk, nm);
-    const int64_t B = (int64_t)D.S + (int64_t)D.U * nm;
-    if (D.G > 8) {  // wide groups: the chunk kernels handle a single token as well
+    if (c->D.G > 8) {  // wide groups: the chunk kernels handle a single token as well
         c->pending = true;
         return attend_impl<T>(c, q, 1, out);
     }
+    const int64_t L = c->nlook++;
+    const Dev D = lookup_dev(c, L);
+    const int nm = (int)n_mem_at(t, D.S, D.W, D.U);
+    const int kk = std::min(D.topk, nm);
+    const int64_t B = (int64_t)D.S + (int64_t)D.U * nm;
     if (sizeof(T) == 2 && c->use_tc && decode_tc_supported(D)) {
-        if (kk > 0) {
-            int l = 0;
-            Prof p(c, K_SELECT);
-            CK(launch_select<T>(D, c->cfg.score_mode, nm, 1, q, c->stream, &l, pdl_ok(c), new_reps));
-            if (l > 0) c->chain = true;
+        {   // sink and window tiles: independent of the lookup, so they run alongside it
+            Prof p(c, K_DECODE);
+            cudaError_t e = launch_decode_tc(D, q, t, kk, B, 0, c->stream, c->tmaps, pdl_ok(c));
+            if (e != cudaSuccess) return fail(c, INFLLM_ECUDA, "decode launch (sinks, window): %s", cudaGetErrorString(e));
+            c->chain = true;
             p.done();
-            c->launches += l;
+            c->launches += 1;
+        }
+        if (kk > 0) {
+            s = stage_select<T>(c, L, nm, 1, q, new_reps);
+            if (s != INFLLM_OK) return s;
         }
         Prof p(c, K_DECODE);
-        int nt = 0;
-        cudaError_t e = launch_decode_tc(D, q, t, kk, B, out, c->stream, c->tmaps, &nt, pdl_ok(c));
-        if (e != cudaSuccess) return fail(c, INFLLM_ECUDA, "decode launch (%d tiles): %s", nt, cudaGetErrorString(e));
+        if (kk > 0) {
+            cudaError_t e = launch_decode_tc(D, q, t, kk, B, 1, c->stream, c->tmaps, pdl_ok(c));
+            if (e != cudaSuccess) return fail(c, INFLLM_ECUDA, "decode launch (units): %s", cudaGetErrorString(e));
+            c->launches += 1;
+        }
+        CK(launch_decode_merge(D, t, kk, B, out, c->stream, pdl_ok(c)));
         p.done();
-        c->launches += 2;  // tiles + merge
-        record_attend(c, t, 1, nm, kk, B);
+        c->launches += 1;
+        record_attend(c, L, t, 1, nm, kk, B);
         return INFLLM_OK;
     }
     if (kk > 0) {
-        s = select_impl<T>(c, nm, 1, q);
+        s = stage_select<T>(c, L, nm, 1, q, true);
         if (s != INFLLM_OK) return s;
     }
     Prof p(c, K_DECODE);
@@ -325,14 +407,14 @@ infllm_status decode_impl(infllm_ctx* c, const void* q, const void* k, const voi
     if (e != cudaSuccess) return fail(c, INFLLM_ECUDA, "decode launch (%d splits): %s", n_split, cudaGetErrorString(e));
     p.done();
     c->launches += 1;
-    record_attend(c, t, 1, nm, kk, B);
+    record_attend(c, L, t, 1, nm, kk, B);
     return INFLLM_OK;
 }
 
 infllm_status zero_state(infllm_ctx* c) {
     CK(cudaMemsetAsync(c->D.Y, 0, sizeof(float) * (size_t)((c->D.T_max / c->D.gblk) + 2) * c->D.Hkv * c->D.d, c->stream));
     CK(cudaMemsetAsync(c->D.counters, 0, sizeof(unsigned) * 2 * c->D.Hkv, c->stream));
-    CK(cudaMemsetAsync(c->D.sel, 0xff, sizeof(int32_t) * (size_t)c->D.Hkv * std::max(1, c->D.topk), c->stream));
+    CK(cudaMemsetAsync(c->sel_base, 0xff, sizeof(int32_t) * 2 * (size_t)c->D.Hkv * std::max(1, c->D.topk), c->stream));
     c->tokens = 0;
     c->units_done = 0;
     c->pending = false;
@@ -340,7 +422,8 @@ infllm_status zero_state(infllm_ctx* c) {
     c->attended = false;
     c->last_nmem = c->last_kk = 0;
     c->last_B = c->last_active = 0;
-    c->qpar = 0;
+    c->nlook = 0;
+    c->last_sel = 0;
     return INFLLM_OK;
 }
 
@@ -405,13 +488,13 @@ infllm_status create_impl(infllm_ctx* c) {
     AL(D.rep_ids, sizeof(int32_t) * (size_t)D.Hkv * D.units_max * D.r);
     AL(D.rep_keys, (size_t)D.Hkv * D.units_max * D.r * D.d * c->elt);
     AL(D.repsum, sizeof(float) * (size_t)D.Hkv * D.units_max * D.d);
-    AL(D.sel, sizeof(int32_t) * (size_t)D.Hkv * std::max(1, D.topk));
+    AL(D.sel, sizeof(int32_t) * 2 * (size_t)D.Hkv * std::max(1, D.topk));  // two buffers
     AL(D.uscore, sizeof(float) * (size_t)D.Hkv * D.units_max);
-    AL(D.qbar_part, sizeof(float) * (size_t)D.Hkv * D.qtiles_max * D.d);
+    AL(D.qbar_part, sizeof(float) * 2 * (size_t)D.Hkv * D.qtiles_max * D.d);  // two buffers
     AL(D.cand, sizeof(uint64_t) * (size_t)D.Hkv * D.score_splits_max * 32);
     AL(D.counters, sizeof(unsigned) * 2 * D.Hkv);
-    AL(D.Qm, (size_t)D.Hkv * 2 * D.qrows_max * D.d * c->elt);  // two buffers, by chunk parity
-    AL(D.Qw, (size_t)D.Hkv * 2 * D.qrows_max * D.d * c->elt);
+    AL(D.Qm, (size_t)D.Hkv * 3 * D.qrows_max * D.d * c->elt);  // three slots
+    AL(D.Qw, (size_t)D.Hkv * 3 * D.qrows_max * D.d * c->elt);
     AL(D.cs_chunk, sizeof(float2) * (size_t)g.max_chunk * D.half);
     AL(D.dec_part, sizeof(float) * (size_t)D.Hkv * D.dec_splits_max * D.G * (D.d + 2));
     double* invf = nullptr;
@@ -444,6 +527,8 @@ infllm_status create_impl(infllm_ctx* c) {
     CK(cudaMemcpy(invf, th.data(), sizeof(double) * D.half, cudaMemcpyHostToDevice));
     CK(cudaMemcpy(cs_rel, rel.data(), sizeof(float2) * rel.size(), cudaMemcpyHostToDevice));
     CK(cudaMemcpy(cs_w, w.data(), sizeof(float2) * w.size(), cudaMemcpyHostToDevice));
+    c->sel_base = D.sel;
+    c->qbar_base = D.qbar_part;
     D.inv_freq = invf;
     D.cs_rel = cs_rel;
     D.cs_W = cs_w;
@@ -562,27 +647,17 @@ infllm_status infllm_prefill(infllm_ctx* c, const void* q, const void* k, const 
                     (long long)n, (long long)c->cfg.max_tokens);
     if (n == 0) return INFLLM_OK;
     if (!q || !k || !v || !out) return fail(c, INFLLM_EINVAL, "prefill: null pointer");
-    const size_t qrow = (size_t)c->D.Hq * c->D.d * c->elt, krow = (size_t)c->D.Hkv * c->D.d * c->elt;
-    for (int64_t t0 = 0; t0 < n; t0 += chunk) {
-        const int m = (int)std::min<int64_t>(chunk, n - t0);
-        const char* qc = (const char*)q + t0 * qrow;
-        if (c->cfg.dtype == INFLLM_BF16) {
-            s = append_impl<__nv_bfloat16>(c, qc, (const char*)k + t0 * krow, (const char*)v + t0 * krow, m);
-            if (s == INFLLM_OK) s = attend_impl<__nv_bfloat16>(c, qc, m, (char*)out + t0 * qrow);
-        } else {
-            s = append_impl<float>(c, qc, (const char*)k + t0 * krow, (const char*)v + t0 * krow, m);
-            if (s == INFLLM_OK) s = attend_impl<float>(c, qc, m, (char*)out + t0 * qrow);
-        }
-        if (s != INFLLM_OK) return s;
-    }
-    return INFLLM_OK;
+    return c->cfg.dtype == INFLLM_BF16
+               ? prefill_impl<__nv_bfloat16>(c, (const char*)q, (const char*)k, (const char*)v, n, chunk, (char*)out)
+               : prefill_impl<float>(c, (const char*)q, (const char*)k, (const char*)v, n, chunk, (char*)out);
 }
 
 infllm_status infllm_get_selection(infllm_ctx* c, int32_t* host_sel) {
     if (!c || !host_sel) return INFLLM_EINVAL;
     if (c->cfg.top_k == 0) return INFLLM_OK;
     CK(cudaStreamSynchronize(c->stream));
-    CK(cudaMemcpy(host_sel, c->D.sel, sizeof(int32_t) * (size_t)c->D.Hkv * c->D.topk, cudaMemcpyDeviceToHost));
+    CK(cudaMemcpy(host_sel, c->sel_base + (size_t)c->last_sel * c->D.Hkv * std::max(1, c->D.topk),
+                  sizeof(int32_t) * (size_t)c->D.Hkv * c->D.topk, cudaMemcpyDeviceToHost));
     // entries beyond the last chunk's selection are not rewritten by the kernels
     for (int h = 0; h < c->D.Hkv; ++h)
         for (int i = c->last_kk; i < c->D.topk; ++i) host_sel[h * c->D.topk + i] = -1;

@@ -45,8 +45,8 @@ __global__ void __launch_bounds__(256) k_attn_simt(Dev D, int64_t c0, int n, int
     const bool valid = tl < n;
     const int64_t t = c0 + tl;
     if (valid) {  // rows past the packed tiles (rows % 8 != 0) are never read
-        const T* Qm = (const T*)D.Qm + (((int64_t)hk * 2 + par) * D.qrows_max + R) * d;
-        const T* Qw = (const T*)D.Qw + (((int64_t)hk * 2 + par) * D.qrows_max + R) * d;
+        const T* Qm = (const T*)D.Qm + (((int64_t)hk * 3 + par) * D.qrows_max + R) * d;
+        const T* Qw = (const T*)D.Qw + (((int64_t)hk * 3 + par) * D.qrows_max + R) * d;
         for (int i = lane; i < d; i += 32) {
             qm_s[warp * d + i] = to_f(Qm[i]);
             qw_s[warp * d + i] = to_f(Qw[i]);

@@ -7,11 +7,21 @@
 //
 // One CTA per (128 packed query rows, KV head): the rows are G q heads x 128/G consecutive
 // queries of one KV group, so every K/V tile is read once per group.  Warp roles:
-//   warp 0      TMA producer: the two rotated query tiles once, then K and V tiles (2 stages)
-//   warp 1      MMA issuer:   S_i = Q K_i^T into TMEM (double buffered), O += P_i V_i
-//   warps 2..5  softmax:      one thread per row; masks, online softmax with lazy rescale of
-//                             O (only when the running max grows by > 2^8), P_i to shared
-//                             memory in the swizzled K-major layout, final 1/l and store.
+//   warp 0      TMA producer: K and V tiles (3-stage rings)
+//   warp 1      MMA issuer:   S_i = Q K_i^T into TMEM (double buffered), O += P_i V_i; both A
+//                             operands (Q and P) are read from TMEM
+//   warps 2..9  softmax:      two threads per row (warps w and w + 4 share a TMEM lane quarter
+//                             and split the tile's 128 columns in halves); the row max is
+//                             combined through shared memory, each exponentiates its own 64: online
+//                             softmax with lazy rescale of O (only when the running max grows by
+//                             > 2^8), P_i as bf16 into the TMEM columns of S_i; at the end the
+//                             two halves' row sums are added and each thread stores 64 outputs.
+// The two rotated query tiles (R(W)q for sinks and memory, R(t)q for the window) are stored into
+// TMEM once by the softmax warps, which frees shared memory for 3-stage K/V rings.  Each softmax
+// warp writes its half of P_i over the first 32 columns of its own half of S_i (it has read them;
+// the partner warp never reads them), so S_i and P_i share a buffer, double buffered: the
+// exponentials of tile i overlap the PV product of tile i - 1, and QK of tile i + 2 (same buffer)
+// is issued after PV(i) -- the tensor pipe executes one thread's MMAs in issue order.
 // Sinks and memory tiles use R(W) q with raw keys; window tiles use R(t) q with R(n) k.
 #include <cuda.h>
 #include <math.h>
@@ -28,29 +38,35 @@ namespace {
 constexpr int BM = 128;  // packed query rows per CTA
 constexpr int BN = 128;  // keys per tile
 constexpr int HD = 128;  // head dim handled here
-constexpr int NTHREADS = 192;
+constexpr int NTHREADS = 320;  // producer warp, MMA warp, 8 softmax warps
+constexpr int NSOFT = 256;     // softmax threads
 constexpr uint32_t TILE = BN * HD * 2;  // bytes of one bf16 128 x 128 tile
 constexpr uint32_t HALF = TILE / 2;     // one 64-column swizzle block (128 rows x 128 B)
-constexpr int OFF_QM = 0;
-constexpr int OFF_QW = OFF_QM + (int)TILE;
-constexpr int OFF_K = OFF_QW + (int)TILE;      // 2 stages
-constexpr int OFF_V = OFF_K + 2 * (int)TILE;   // 2 stages
-constexpr int OFF_P = OFF_V + 2 * (int)TILE;
-constexpr int OFF_BAR = OFF_P + (int)TILE;
-constexpr int OFF_SEL = OFF_BAR + 256;             // selected unit ids of this KV head
+constexpr int NSTAGE = 3;                      // K and V ring depth
+constexpr int OFF_K = 0;
+constexpr int OFF_V = OFF_K + NSTAGE * (int)TILE;
+constexpr int OFF_BAR = OFF_V + NSTAGE * (int)TILE;
+constexpr int OFF_LSUM = OFF_BAR + 256;            // [2][128] row sums of the two column halves
+constexpr int OFF_MXS = OFF_LSUM + 2 * 128 * 4;    // [2 tile parities][2 halves][128] half-maxima
+constexpr int OFF_SEL = OFF_MXS + 2 * 2 * 128 * 4; // selected unit ids of this KV head
 constexpr int MAX_SEL = 256;
 constexpr int SMEM_BYTES = OFF_SEL + MAX_SEL * 4 + 1024;  // + alignment slack
-constexpr uint32_t TMEM_COLS = 512;              // S0 [0,128) S1 [128,256) O [256,384)
+constexpr uint32_t TMEM_COLS = 512;  // S0 / P0 [0,128), S1 / P1 [128,256), O [256,384), Qm [384,448), Qw [448,512)
 constexpr uint32_t TM_O = 256;
+constexpr uint32_t TM_QM = 384;  // R(W) q, bf16 pairs
+constexpr uint32_t TM_QW = 448;  // R(t) q, bf16 pairs
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float RESCALE_LOG2 = 8.0f;
 constexpr int ERR_TIMEOUT = 16;
 
 struct Bars {
-    uint64_t q, kfull[2], kempty[2], vfull[2], vempty[2], sfull[2], sfree[2], pfull, pvdone;
+    uint64_t q, kfull[NSTAGE], kempty[NSTAGE], vfull[NSTAGE], vempty[NSTAGE], sfull[2], pfull, pvdone;
+    uint64_t mx[4];  // per TMEM lane quarter: both softmax warps of the rows posted their half-max
     uint32_t tmem;
     int abort;
 };
+
+static_assert(sizeof(Bars) <= 256, "barrier block overflows its shared-memory slot");
 
 struct TileInfo {
     int kind;  // 0 sink, 1 memory unit, 2 window
@@ -93,28 +109,20 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Bars* b
 }
 
 __device__ void producer(const TcMaps& maps, const Plan& P, const Dev& D, uint8_t* sm, Bars* bars) {
-    ptx::prefetch_tmap(&maps.qm);
-    ptx::prefetch_tmap(&maps.qw);
     ptx::prefetch_tmap(&maps.kraw);
     ptx::prefetch_tmap(&maps.krot);
     ptx::prefetch_tmap(&maps.v);
-    const int y = P.par * (int)D.qrows_max + P.a * BM;
-    ptx::mbar_expect_tx(&bars->q, 4 * HALF);
-    ptx::tma_load_3d(sm + OFF_QM, &maps.qm, &bars->q, 0, y, P.hk);
-    ptx::tma_load_3d(sm + OFF_QM + HALF, &maps.qm, &bars->q, 64, y, P.hk);
-    ptx::tma_load_3d(sm + OFF_QW, &maps.qw, &bars->q, 0, y, P.hk);
-    ptx::tma_load_3d(sm + OFF_QW + HALF, &maps.qw, &bars->q, 64, y, P.hk);
     int issued = 0;
     for (int i = 0; i < P.NT; ++i) {
-        const int s = i & 1;
-        const uint32_t use = (uint32_t)(i >> 1);
-        if (i >= 2 && !wait_bar(&bars->kempty[s], (use - 1) & 1, bars, D)) break;
+        const int s = i % NSTAGE;
+        const uint32_t use = (uint32_t)(i / NSTAGE);
+        if (i >= NSTAGE && !wait_bar(&bars->kempty[s], (use - 1) & 1, bars, D)) break;
         const TileInfo T = P.tile(D, i);
         const CUtensorMap* km = T.kind == 2 ? &maps.krot : &maps.kraw;
         ptx::mbar_expect_tx(&bars->kfull[s], TILE);
         ptx::tma_load_3d(sm + OFF_K + s * TILE, km, &bars->kfull[s], 0, (int)T.y0, P.hk);
         ptx::tma_load_3d(sm + OFF_K + s * TILE + HALF, km, &bars->kfull[s], 64, (int)T.y0, P.hk);
-        if (i >= 2 && !wait_bar(&bars->vempty[s], (use - 1) & 1, bars, D)) {
+        if (i >= NSTAGE && !wait_bar(&bars->vempty[s], (use - 1) & 1, bars, D)) {
             issued = i + 1;
             break;
         }
@@ -125,52 +133,48 @@ __device__ void producer(const TcMaps& maps, const Plan& P, const Dev& D, uint8_
     }
     if (*(volatile int*)&bars->abort) {
         // let the copies already in flight land before the CTA exits (bounded)
-        for (int i = issued - 2 < 0 ? 0 : issued - 2; i < issued; ++i) {
-            ptx::mbar_wait(&bars->kfull[i & 1], (uint32_t)(i >> 1) & 1, 1ll << 28);
-            ptx::mbar_wait(&bars->vfull[i & 1], (uint32_t)(i >> 1) & 1, 1ll << 28);
+        for (int i = issued - NSTAGE < 0 ? 0 : issued - NSTAGE; i < issued; ++i) {
+            ptx::mbar_wait(&bars->kfull[i % NSTAGE], (uint32_t)(i / NSTAGE) & 1, 1ll << 28);
+            ptx::mbar_wait(&bars->vfull[i % NSTAGE], (uint32_t)(i / NSTAGE) & 1, 1ll << 28);
         }
-        ptx::mbar_wait(&bars->q, 0, 1ll << 28);
     }
 }
 
 __device__ void mma_issuer(const Plan& P, const Dev& D, uint8_t* sm, Bars* bars, uint32_t tmem) {
     constexpr uint32_t IDESC_QK = ptx::idesc_bf16_f32(BM, BN, false, false);
     constexpr uint32_t IDESC_PV = ptx::idesc_bf16_f32(BM, HD, false, true);
-    if (!wait_bar(&bars->q, 0, bars, D)) return;
+    if (!wait_bar(&bars->q, 0, bars, D)) return;  // the query tiles are in TMEM
     ptx::tc_fence_after();
-    const uint32_t qm = ptx::smem_u32(sm + OFF_QM), qw = ptx::smem_u32(sm + OFF_QW);
-    const uint32_t kb = ptx::smem_u32(sm + OFF_K), vb = ptx::smem_u32(sm + OFF_V), pb = ptx::smem_u32(sm + OFF_P);
+    const uint32_t kb = ptx::smem_u32(sm + OFF_K), vb = ptx::smem_u32(sm + OFF_V);
     for (int i = 0; i <= P.NT; ++i) {
         if (i < P.NT) {
-            const int s = i & 1;
-            const uint32_t use = (uint32_t)(i >> 1);
-            if (!wait_bar(&bars->kfull[s], use & 1, bars, D)) return;
-            if (i >= 2 && !wait_bar(&bars->sfree[s], (use - 1) & 1, bars, D)) return;
+            // S_i into buffer i & 1, which held P_{i-2}: PV(i - 2) was issued in the previous
+            // iteration, before this MMA, and same-thread MMAs execute in order
+            const int s = i % NSTAGE, b = i & 1;
+            if (!wait_bar(&bars->kfull[s], (uint32_t)(i / NSTAGE) & 1, bars, D)) return;
             ptx::tc_fence_after();
-            const uint32_t qa = P.tile(D, i).kind == 2 ? qw : qm;
+            const uint32_t qa = tmem + (P.tile(D, i).kind == 2 ? TM_QW : TM_QM);
             const uint32_t ka = kb + s * TILE;
 #pragma unroll
             for (int ks = 0; ks < HD / 16; ++ks) {
                 const uint32_t off = (uint32_t)(ks >> 2) * HALF + (uint32_t)(ks & 3) * 32;
-                ptx::mma_bf16(tmem + s * BN, ptx::sdesc_sw128(qa + off, 16, 1024), ptx::sdesc_sw128(ka + off, 16, 1024),
-                              IDESC_QK, ks > 0 ? 1u : 0u);
+                ptx::mma_bf16_ts(tmem + b * BN, qa + (uint32_t)ks * 8, ptx::sdesc_sw128(ka + off, 16, 1024), IDESC_QK,
+                                 ks > 0 ? 1u : 0u);
             }
-            ptx::mma_commit(&bars->sfull[s]);
+            ptx::mma_commit(&bars->sfull[b]);
             ptx::mma_commit(&bars->kempty[s]);
         }
         if (i >= 1) {
-            const int j = i - 1, sj = j & 1;
+            const int j = i - 1, sj = j % NSTAGE, bj = j & 1;
             if (!wait_bar(&bars->pfull, (uint32_t)j & 1, bars, D)) return;
-            if (!wait_bar(&bars->vfull[sj], (uint32_t)(j >> 1) & 1, bars, D)) return;
+            if (!wait_bar(&bars->vfull[sj], (uint32_t)(j / NSTAGE) & 1, bars, D)) return;
             ptx::tc_fence_after();
             const uint32_t va = vb + sj * TILE;
 #pragma unroll
-            for (int ks = 0; ks < BN / 16; ++ks) {
-                const uint32_t aoff = (uint32_t)(ks >> 2) * HALF + (uint32_t)(ks & 3) * 32;
-                ptx::mma_bf16(tmem + TM_O, ptx::sdesc_sw128(pb + aoff, 16, 1024),
-                              ptx::sdesc_sw128(va + (uint32_t)ks * 2048, HALF, 1024), IDESC_PV,
-                              (j > 0 || ks > 0) ? 1u : 0u);
-            }
+            for (int ks = 0; ks < BN / 16; ++ks)  // keys 16 ks ..: half ks / 4 of P_j, 8 columns per step
+                ptx::mma_bf16_ts(tmem + TM_O, tmem + bj * BN + (uint32_t)(ks >> 2) * 64 + (uint32_t)(ks & 3) * 8,
+                                 ptx::sdesc_sw128(va + (uint32_t)ks * 2048, HALF, 1024), IDESC_PV,
+                                 (j > 0 || ks > 0) ? 1u : 0u);
             ptx::mma_commit(&bars->pvdone);
             ptx::mma_commit(&bars->vempty[sj]);
         }
@@ -188,19 +192,47 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
-__device__ void softmax_role(const Plan& P, const Dev& D, uint8_t* sm, Bars* bars, uint32_t tmem, int64_t c0, int n,
-                             __nv_bfloat16* __restrict__ out, int warp, int lane) {
-    const int quarter = warp & 3;  // TMEM lanes this warp may access
+// PV completions are consumed strictly in order, and never more than one phase late: a parity
+// wait on an mbarrier that has completed two phases past the awaited one would wait for a third.
+// Tile i consumes PV(i - 1) before it releases P_i; PV(i) cannot have been issued by then.
+struct PvTrack {
+    int seen = 0;  // PV products known complete: tiles [0, seen)
+    __device__ __forceinline__ bool upto(int j, Bars* bars, const Dev& D) {
+        while (seen <= j) {
+            if (!warp_wait(&bars->pvdone, (uint32_t)seen & 1, bars, D)) return false;
+            ++seen;
+        }
+        return true;
+    }
+};
+
+__device__ void softmax_role(const Plan& P, const Dev& D, Bars* bars, float* lsum, float* mxs, uint32_t tmem,
+                             int64_t c0, int n, __nv_bfloat16* __restrict__ out, int warp, int lane) {
+    const int quarter = warp & 3;        // TMEM lanes this warp may access
+    const int half = (warp - 2) >> 2;    // columns [64 half, 64 half + 64) of every tile are this thread's
     const int row = quarter * 32 + lane;
     const uint32_t tl_addr = tmem + ((uint32_t)(quarter * 32) << 16);
     const int hg = row / D.qt, tl = P.a * D.qt + row % D.qt;
     const bool valid = tl < n;
     const int64_t t = c0 + tl;
     const float sc = D.inv_sqrt_d * LOG2E;  // logits in log2 units: s * sc
-    float m_used = -INFINITY, l = 0.f;      // running max (log2 units) and sum
-    float s[BN];
-    uint8_t* prow = sm + OFF_P + row * 128;
+    float m_used = -INFINITY, l = 0.f;      // running max (log2 units) and this half's sum
+    float s[64];
+    PvTrack pv;
     bool ok = true;
+    {   // this thread's query row into TMEM: half 0 stores R(W) q, half 1 stores R(t) q
+        const __nv_bfloat16* src = (const __nv_bfloat16*)(half == 0 ? D.Qm : D.Qw) +
+                                   (((int64_t)P.hk * 3 + P.par) * D.qrows_max + (int64_t)P.a * BM + row) * HD;
+        uint4 qv[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) qv[c] = __ldg(reinterpret_cast<const uint4*>(src) + c);
+        const uint32_t qcol = tl_addr + (half == 0 ? TM_QM : TM_QW);
+        ptx::tmem_st32(qcol, reinterpret_cast<const float*>(qv));
+        ptx::tmem_st32(qcol + 32, reinterpret_cast<const float*>(qv + 8));
+        ptx::tmem_wait_st();
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(&bars->q);
+    }
     for (int i = 0; i < P.NT; ++i) {
         const int b = i & 1;
         if (!warp_wait(&bars->sfull[b], (uint32_t)(i >> 1) & 1, bars, D)) {
@@ -208,11 +240,10 @@ __device__ void softmax_role(const Plan& P, const Dev& D, uint8_t* sm, Bars* bar
             break;
         }
         ptx::tc_fence_after();
-#pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) ptx::tmem_ld32(tl_addr + b * BN + c4 * 32, s + c4 * 32);
+        const uint32_t sbase = tl_addr + b * BN;
+        ptx::tmem_ld32(sbase + half * 64, s);
+        ptx::tmem_ld32(sbase + half * 64 + 32, s + 32);
         ptx::tmem_wait_ld();
-        ptx::tc_fence_before();
-        ptx::mbar_arrive(&bars->sfree[b]);
         // columns [0, lim) of this tile are attended by this row (causal limit on sinks and window)
         const TileInfo T = P.tile(D, i);
         int lim = T.nv;
@@ -220,85 +251,102 @@ __device__ void softmax_role(const Plan& P, const Dev& D, uint8_t* sm, Bars* bar
             const int64_t c = t - T.y0 + 1;
             lim = c < (int64_t)lim ? (int)(c < 0 ? 0 : c) : lim;
         }
-        float mx = -INFINITY;
-        if (__all_sync(0xffffffffu, lim >= BN)) {
+        const int own = lim - half * 64;  // valid columns of this half
+        float mq[8];                       // independent partial maxima (short dependency chains)
 #pragma unroll
-            for (int c = 0; c < BN; ++c) mx = fmaxf(mx, s[c]);
+        for (int e = 0; e < 8; ++e) mq[e] = -INFINITY;
+        if (__all_sync(0xffffffffu, own >= 64)) {
+#pragma unroll
+            for (int c = 0; c < 64; ++c) mq[c & 7] = fmaxf(mq[c & 7], s[c]);
         } else {
 #pragma unroll
-            for (int c = 0; c < BN; ++c) {
-                s[c] = c < lim ? s[c] : -INFINITY;
-                mx = fmaxf(mx, s[c]);
+            for (int c = 0; c < 64; ++c) {
+                s[c] = c < own ? s[c] : -INFINITY;
+                mq[c & 7] = fmaxf(mq[c & 7], s[c]);
             }
         }
+        float mx = fmaxf(fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])), fmaxf(fmaxf(mq[4], mq[5]), fmaxf(mq[6], mq[7])));
+        // the row max over both halves: post this half's, wait (bounded) until the partner warp
+        // posted its own for this tile, read it.  Slots alternate by tile parity; a warp reaches
+        // tile i + 2 only after its partner arrived for tile i + 1, i.e. after it read slot i.
+        mxs[((i & 1) * 2 + half) * 128 + row] = mx;
+        ptx::mbar_arrive(&bars->mx[quarter]);
+        if (!warp_wait(&bars->mx[quarter], (uint32_t)i & 1, bars, D)) {
+            ok = false;
+            break;
+        }
+        mx = fmaxf(mx, mxs[((i & 1) * 2 + (1 - half)) * 128 + row]);
         const float mt = mx * sc;
         const bool need = mt > m_used + RESCALE_LOG2;
         const float m_new = need ? mt : m_used;
-        if (i >= 1) {
-            if (!warp_wait(&bars->pvdone, (uint32_t)(i - 1) & 1, bars, D)) {
+        if (i >= 1 && __any_sync(0xffffffffu, need)) {  // O must hold every earlier product first
+            if (!pv.upto(i - 1, bars, D)) {
                 ok = false;
                 break;
             }
             ptx::tc_fence_after();
-            if (__any_sync(0xffffffffu, need)) {
-                const float f = need ? ex2(m_used - m_new) : 1.f;
-                l *= f;
+            const float f = need ? ex2(m_used - m_new) : 1.f;
+            l *= f;
 #pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4) {
-                    float o[32];
-                    ptx::tmem_ld32(tl_addr + TM_O + c4 * 32, o);
-                    ptx::tmem_wait_ld();
+            for (int c4 = 0; c4 < 2; ++c4) {
+                float o[32];
+                ptx::tmem_ld32(tl_addr + TM_O + half * 64 + c4 * 32, o);
+                ptx::tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) o[e] *= f;
-                    ptx::tmem_st32(tl_addr + TM_O + c4 * 32, o);
-                }
-                ptx::tmem_wait_st();
+                for (int e = 0; e < 32; ++e) o[e] *= f;
+                ptx::tmem_st32(tl_addr + TM_O + half * 64 + c4 * 32, o);
             }
         }
         m_used = m_new;
         const float nref = m_used == -INFINITY ? 0.f : -m_used;
-        float rs0 = 0.f, rs1 = 0.f;
+        float rs[8];
 #pragma unroll
-        for (int cb = 0; cb < 2; ++cb) {
+        for (int e = 0; e < 8; ++e) rs[e] = 0.f;
+        uint32_t w[32];  // this half's 64 keys as 32 columns of packed bf16 pairs
 #pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
-                uint32_t w[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int c = cb * 64 + ch * 8 + 2 * e;
-                    const float p0 = ex2(fmaf(s[c], sc, nref)), p1 = ex2(fmaf(s[c + 1], sc, nref));
-                    rs0 += p0;
-                    rs1 += p1;
-                    __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
-                    w[e] = *reinterpret_cast<uint32_t*>(&h);
-                }
-                *reinterpret_cast<uint4*>(prow + cb * HALF + ((ch ^ (row & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
-            }
+        for (int e = 0; e < 32; ++e) {
+            const float p0 = ex2(fmaf(s[2 * e], sc, nref)), p1 = ex2(fmaf(s[2 * e + 1], sc, nref));
+            rs[(2 * e) & 7] += p0;
+            rs[(2 * e + 1) & 7] += p1;
+            __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
+            w[e] = *reinterpret_cast<uint32_t*>(&h);
         }
-        l += rs0 + rs1;
-        ptx::fence_proxy_async_smem();
+        ptx::tmem_st32(sbase + half * 64, reinterpret_cast<const float*>(w));  // over this half's own S columns
+        l += ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
+        ptx::tmem_wait_st();
+        // PV(i - 1) ran during this tile's exponentials; consume its completion before P_i is
+        // released (PV(i) is issued only after the arrival below)
+        if (i >= 1 && !pv.upto(i - 1, bars, D)) {
+            ok = false;
+            break;
+        }
         ptx::tc_fence_before();
         ptx::mbar_arrive(&bars->pfull);
     }
-    if (!ok || !warp_wait(&bars->pvdone, (uint32_t)(P.NT - 1) & 1, bars, D)) return;
+    ok = ok && pv.upto(P.NT - 1, bars, D);
+    // the two halves' sums of this row (every softmax thread reaches this barrier: all waits above
+    // are bounded)
+    lsum[half * 128 + row] = l;
+    asm volatile("bar.sync 1, %0;" ::"n"(NSOFT) : "memory");
+    if (!__all_sync(0xffffffffu, ok)) return;
     ptx::tc_fence_after();
-    const float inv = 1.f / l;
-    __nv_bfloat16* orow = out + ((int64_t)tl * D.Hq + P.hk * D.G + hg) * HD;
+    const float inv = 1.f / (l + lsum[(1 - half) * 128 + row]);
+    __nv_bfloat16* orow = out + ((int64_t)tl * D.Hq + P.hk * D.G + hg) * HD + half * 64;
 #pragma unroll
-    for (int c4 = 0; c4 < 4; ++c4) {
+    for (int c4 = 0; c4 < 2; ++c4) {
         float o[32];
-        ptx::tmem_ld32(tl_addr + TM_O + c4 * 32, o);
+        ptx::tmem_ld32(tl_addr + TM_O + half * 64 + c4 * 32, o);
         ptx::tmem_wait_ld();
         if (valid) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                uint32_t w[4];
+                uint32_t w4[4];
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     __nv_bfloat162 h = __floats2bfloat162_rn(o[e * 8 + 2 * q] * inv, o[e * 8 + 2 * q + 1] * inv);
-                    w[q] = *reinterpret_cast<uint32_t*>(&h);
+                    w4[q] = *reinterpret_cast<uint32_t*>(&h);
                 }
-                *reinterpret_cast<uint4*>(orow + c4 * 32 + e * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+                *reinterpret_cast<uint4*>(orow + c4 * 32 + e * 8) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
             }
         }
     }
@@ -333,17 +381,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     int* sel_s = reinterpret_cast<int*>(sm + OFF_SEL);
     P.sel = sel_s;
     if (threadIdx.x == 0) {
-        ptx::mbar_init(&bars->q, 1);
-        for (int s = 0; s < 2; ++s) {
+        ptx::mbar_init(&bars->q, NSOFT);
+        for (int s = 0; s < NSTAGE; ++s) {
             ptx::mbar_init(&bars->kfull[s], 1);
             ptx::mbar_init(&bars->kempty[s], 1);
             ptx::mbar_init(&bars->vfull[s], 1);
             ptx::mbar_init(&bars->vempty[s], 1);
-            ptx::mbar_init(&bars->sfull[s], 1);
-            ptx::mbar_init(&bars->sfree[s], 128);
         }
-        ptx::mbar_init(&bars->pfull, 128);
+        for (int b = 0; b < 2; ++b) ptx::mbar_init(&bars->sfull[b], 1);
+        ptx::mbar_init(&bars->pfull, NSOFT);
         ptx::mbar_init(&bars->pvdone, 1);
+        for (int qd = 0; qd < 4; ++qd) ptx::mbar_init(&bars->mx[qd], 64);
         bars->abort = 0;
         ptx::mbar_fence_init();
     }
@@ -374,7 +422,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         } else if (warp == 1) {
             if (lane == 0) mma_issuer(P, D, sm, bars, tmem);
         } else {
-            softmax_role(P, D, sm, bars, tmem, c0, n, out, warp, lane);
+            softmax_role(P, D, bars, reinterpret_cast<float*>(sm + OFF_LSUM), reinterpret_cast<float*>(sm + OFF_MXS),
+                         tmem, c0, n, out, warp, lane);
         }
     }
     ptx::tc_fence_before();
@@ -429,8 +478,8 @@ bool make_tc_maps(const Dev& D, void* out) {
     return encode_3d(&m->kraw, D.Kraw, (uint64_t)D.T_max, (uint64_t)D.Hkv) &&
            encode_3d(&m->krot, D.Krot, (uint64_t)D.T_max, (uint64_t)D.Hkv) &&
            encode_3d(&m->v, D.V, (uint64_t)D.T_max, (uint64_t)D.Hkv) &&
-           encode_3d(&m->qm, D.Qm, 2 * (uint64_t)D.qrows_max, (uint64_t)D.Hkv) &&
-           encode_3d(&m->qw, D.Qw, 2 * (uint64_t)D.qrows_max, (uint64_t)D.Hkv);
+           encode_3d(&m->qm, D.Qm, 3 * (uint64_t)D.qrows_max, (uint64_t)D.Hkv) &&
+           encode_3d(&m->qw, D.Qw, 3 * (uint64_t)D.qrows_max, (uint64_t)D.Hkv);
 }
 
 cudaError_t launch_attend_tc(const Dev& D, int64_t c0, int n, int kk, int64_t B, int par, void* out, cudaStream_t st,

@@ -28,13 +28,13 @@ struct Dev {
     void* rep_keys;       // [Hkv][units_max][r][d] raw keys (context dtype)
     float* repsum;        // [Hkv][units_max][d] fp32 sum of the r raw keys
     // lookup
-    int32_t* sel;         // [Hkv][topk] ascending ids, -1 padded
+    int32_t* sel;         // [Hkv][topk] ascending ids, -1 padded (the current lookup's of two buffers)
     float* uscore;        // [Hkv][units_max] last chunk's unit scores
-    float* qbar_part;     // [Hkv][qtiles_max][d] per-tile raw query sums
+    float* qbar_part;     // [Hkv][qtiles_max][d] per-tile raw query sums (the current lookup's of two)
     uint64_t* cand;       // [Hkv][score_splits_max][32] top-k candidate lists
-    unsigned* counters;   // [Hkv] arrival counters (last-block-done)
-    // rotated, packed queries of a chunk: [Hkv][2][qrows_max][d] (two buffers alternating by chunk
-    // parity, so the next chunk's queries can be prepared while this chunk's attention runs)
+    unsigned* counters;   // [2][Hkv] arrival counters (last CTA done): unit selection, CUDA-core decode merge
+    // rotated, packed queries of a chunk: [Hkv][3][qrows_max][d] (three slots, so later chunks'
+    // queries can be packed while an earlier chunk's attention runs)
     void* Qm;             // R(W) q  (sink / memory frame)
     void* Qw;             // R(t) q  (window frame)
     int64_t qrows_max;    // rows per buffer and kv head

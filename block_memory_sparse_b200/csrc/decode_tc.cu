@@ -7,9 +7,13 @@
 // the sum l of exp(s - m) and the unnormalised output over its 128 keys; the last CTA of each
 // KV head rescales every partial by exp(m_s - M) and divides by the total sum.
 //
-// Launch sequence of one step: k_decode_append (plain launch) -> unit scoring + top-k
-// (programmatic dependent launch: it reads only the representative pool and the query, so it
-// overlaps the store) -> k_decode_attn (programmatic dependent launch; waits for both).
+// Launch sequence of one step (programmatic dependent launches after the first):
+//   k_decode_append           store the token (early kernel)
+//   k_decode_attn, part 0     sink and window tiles: need the store, not the selection
+//   unit scoring + top-k      reads only the representative pool and the query, so it runs
+//                             alongside part 0 (it holds its completion until part 0 is done)
+//   k_decode_attn, part 1     the selected units' tiles (waits for the selection)
+//   k_decode_merge            log-sum-exp merge of every tile's partial
 #include <cuda.h>
 #include <math.h>
 
@@ -148,24 +152,28 @@ __device__ __forceinline__ uint32_t tile_chunk(uint32_t base, int j, int c) {
 // (mma.sync m16n8k16, bf16 in, fp32 accumulate): S = Q K^T, then O = P V with P kept in
 // registers; softmax statistics are combined across the four warps through shared memory.
 __global__ void __launch_bounds__(DTHREADS) k_decode_attn(const __grid_constant__ TcMaps maps, Dev D,
-                                                          const __nv_bfloat16* __restrict__ q,
-                                                          __nv_bfloat16* __restrict__ out, int64_t t, int kk, int64_t B,
-                                                          int NT) {
+                                                          const __nv_bfloat16* __restrict__ q, int64_t t, int kk,
+                                                          int64_t B, int part) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     float* red = reinterpret_cast<float*>(sm + OFF_RED);  // [2][4 warps][8 rows]
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + OFF_MISC);
-    const int hk = blockIdx.y, ti = blockIdx.x;
+    const int hk = blockIdx.y;
+    // tile index in the working context (sinks, units, window): part 0 takes sinks and window,
+    // part 1 the selected units
+    const int nst = ((D.S < t + 1 ? D.S : (int)(t + 1)) + DK - 1) / DK;
+    const int nut = kk * ((D.U + DK - 1) / DK);
+    const int ti = part == 1 ? nst + (int)blockIdx.x : ((int)blockIdx.x < nst ? (int)blockIdx.x : (int)blockIdx.x + nut);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, tg = lane & 3;
     const int G = D.G;
-    pdl_trigger();  // the merge kernel may start its prologue
+    pdl_trigger();  // the next kernel reads nothing this one writes before the merge
     if (tid == 0) {
         ptx::mbar_init(bar, 1);
         ptx::mbar_fence_init();
     }
     __syncthreads();
-    pdl_wait();  // the token's store, its (cos, sin) and the selection are ready past this point
+    pdl_wait();  // the token's store, its (cos, sin) and (part 1) the selection are ready past this point
     const DTile T = decode_tile(D, hk, ti, t, kk, B);
     if (tid == 0) {
         const CUtensorMap* km = T.kind == 2 ? &maps.krot : &maps.kraw;
@@ -283,15 +291,15 @@ __global__ void __launch_bounds__(DTHREADS) k_decode_attn(const __grid_constant_
         obuf[(warp * 8 + g) * DHD + 8 * nt + 2 * tg + 1] = oacc[nt][1];
     }
     __syncthreads();
-    float* part = D.dec_part + ((int64_t)hk * D.dec_splits_max + ti) * G * (DHD + 2);
+    float* pout = D.dec_part + ((int64_t)hk * D.dec_splits_max + ti) * G * (DHD + 2);
     for (int h = 0; h < G; ++h) {
         const float o = obuf[(0 * 8 + h) * DHD + tid] + obuf[(1 * 8 + h) * DHD + tid] + obuf[(2 * 8 + h) * DHD + tid] +
                         obuf[(3 * 8 + h) * DHD + tid];
-        part[h * (DHD + 2) + 2 + tid] = o;
+        pout[h * (DHD + 2) + 2 + tid] = o;
         if (tid == 0) {
             const float mh = fmaxf(fmaxf(red[h], red[8 + h]), fmaxf(red[16 + h], red[24 + h]));
-            part[h * (DHD + 2) + 0] = mh == -INFINITY ? -INFINITY : mh * D.inv_sqrt_d;  // natural-log units
-            part[h * (DHD + 2) + 1] = red[32 + h] + red[40 + h] + red[48 + h] + red[56 + h];
+            pout[h * (DHD + 2) + 0] = mh == -INFINITY ? -INFINITY : mh * D.inv_sqrt_d;  // natural-log units
+            pout[h * (DHD + 2) + 1] = red[32 + h] + red[40 + h] + red[48 + h] + red[56 + h];
         }
     }
 }
@@ -357,23 +365,27 @@ cudaError_t launch_decode_append(const Dev& D, const void* q, const void* k, con
                     (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, t);
 }
 
-cudaError_t launch_decode_tc(const Dev& D, const void* q, int64_t t, int kk, int64_t B, void* out, cudaStream_t st,
-                             const void* tmaps, int* n_tiles_out, bool pdl) {
+cudaError_t launch_decode_tc(const Dev& D, const void* q, int64_t t, int kk, int64_t B, int part, cudaStream_t st,
+                             const void* tmaps, bool pdl) {
     const int S_eff = (int)(D.S < t + 1 ? D.S : t + 1);
     const int64_t win = t - B + 1;
-    const int NT = (S_eff + DK - 1) / DK + kk * ((D.U + DK - 1) / DK) + (int)((win + DK - 1) / DK);
-    *n_tiles_out = NT;
-    if (NT > D.dec_splits_max || NT > MERGE_SLICES * MERGE_BATCH) return cudaErrorInvalidValue;
+    const int nst = (S_eff + DK - 1) / DK, nut = kk * ((D.U + DK - 1) / DK), nwt = (int)((win + DK - 1) / DK);
+    if (nst + nut + nwt > D.dec_splits_max || nst + nut + nwt > MERGE_SLICES * MERGE_BATCH) return cudaErrorInvalidValue;
+    const int tiles = part == 1 ? nut : nst + nwt;
+    if (tiles == 0) return cudaSuccess;
     static bool attr_set = false;
     if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(k_decode_attn, cudaFuncAttributeMaxDynamicSharedMemorySize, DSMEM);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    cudaError_t e = launch_k(k_decode_attn, dim3(NT, D.Hkv), dim3(DTHREADS), DSMEM, st, pdl,
-                             *reinterpret_cast<const TcMaps*>(tmaps), D, (const __nv_bfloat16*)q, (__nv_bfloat16*)out,
-                             t, kk, B, NT);
-    if (e != cudaSuccess) return e;
+    return launch_k(k_decode_attn, dim3(tiles, D.Hkv), dim3(DTHREADS), DSMEM, st, pdl,
+                    *reinterpret_cast<const TcMaps*>(tmaps), D, (const __nv_bfloat16*)q, t, kk, B, part);
+}
+
+cudaError_t launch_decode_merge(const Dev& D, int64_t t, int kk, int64_t B, void* out, cudaStream_t st, bool pdl) {
+    const int S_eff = (int)(D.S < t + 1 ? D.S : t + 1);
+    const int NT = (S_eff + DK - 1) / DK + kk * ((D.U + DK - 1) / DK) + (int)((t - B + 1 + DK - 1) / DK);
     return launch_k(k_decode_merge, dim3(D.G, D.Hkv), dim3(MERGE_SLICES * DHD), 0, st, pdl, D, (__nv_bfloat16*)out, NT);
 }
 

@@ -15,7 +15,7 @@ cudaError_t launch_ysum(const Dev& D, const void* q, int64_t c0, int n, cudaStre
 template <typename T>
 cudaError_t launch_reps(const Dev& D, int64_t j0, int64_t j1, cudaStream_t st, bool pdl);
 
-// Rotated, packed queries of the chunk into query buffer `par` (0 or 1) + per-tile raw query sums.
+// Rotated, packed queries of the chunk into query slot `par` (0..2) + per-tile raw query sums.
 template <typename T>
 cudaError_t launch_prep(const Dev& D, const void* q, int64_t c0, int n, int par, cudaStream_t st, bool pdl);
 
@@ -46,12 +46,15 @@ cudaError_t launch_decode(const Dev& D, const void* q, int64_t t, int kk, int64_
 
 int decode_split_keys(int elt_bytes);
 
-// Decode on the TMA path (bf16, head dim 128, G <= 8): store the token, then (after the lookup)
-// split-KV attention over 128-key tiles with a last-CTA log-sum-exp merge.
+// Decode on the TMA path (bf16, head dim 128, G <= 8): store the token, split-KV attention over
+// 128-key tiles (sinks and window alongside the lookup, the selected units after it), then a
+// log-sum-exp merge.
 bool decode_tc_supported(const Dev& D);
 cudaError_t launch_decode_append(const Dev& D, const void* q, const void* k, const void* v, int64_t t, cudaStream_t st,
                                  bool pdl);
-cudaError_t launch_decode_tc(const Dev& D, const void* q, int64_t t, int kk, int64_t B, void* out, cudaStream_t st,
-                             const void* tmaps, int* n_tiles_out, bool pdl);
+// part 0: sink and window tiles (no selection needed); part 1: the selected units' tiles.
+cudaError_t launch_decode_tc(const Dev& D, const void* q, int64_t t, int kk, int64_t B, int part, cudaStream_t st,
+                             const void* tmaps, bool pdl);
+cudaError_t launch_decode_merge(const Dev& D, int64_t t, int kk, int64_t B, void* out, cudaStream_t st, bool pdl);
 
 }  // namespace infllm

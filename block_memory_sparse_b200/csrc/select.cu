@@ -19,8 +19,8 @@ namespace infllm {
 // queries [a*qt, a*qt + qt); row r of a tile is (head hg = r / qt, query a*qt + r % qt).
 // Thread = (vector v: elements [vV, vV+V) of each half, row group): 16-byte loads and stores,
 // four rows per load batch.  Also writes each tile's raw query sum over its rows
-// (fixed-order reduction).  An early kernel: it may run while the previous chunk's attention
-// reads the other query buffer, and while this chunk's keys are stored, so it takes the
+// (fixed-order reduction).  An early kernel: it may run while an earlier chunk's attention
+// reads another query slot, and while this chunk's keys are stored, so it takes the
 // (cos, sin)(t theta_i) of its queries from the fp64 digit tables itself.
 template <typename T>
 __global__ void __launch_bounds__(256) k_prep(Dev D, const T* __restrict__ q, int64_t c0, int n, int par) {
@@ -40,7 +40,7 @@ __global__ void __launch_bounds__(256) k_prep(Dev D, const T* __restrict__ q, in
         cs_sh[x] = tl < n ? cs_abs(D.cs_abs3, D.half, c0 + tl, x % D.half) : make_float2(1.f, 0.f);
     }
     __syncthreads();
-    const int64_t qbase = ((int64_t)hk * 2 + par) * D.qrows_max + (int64_t)a * rows;
+    const int64_t qbase = ((int64_t)hk * 3 + par) * D.qrows_max + (int64_t)a * rows;
     T* Qm = (T*)D.Qm + qbase * D.d;
     T* Qw = (T*)D.Qw + qbase * D.d;
     float2 cw[V];
@@ -128,9 +128,71 @@ template <> struct Vec16<float> {
     }
 };
 
+// Top-k of one KV head from the scoring CTAs' top-32 lists (composite keys, descending), run by
+// the last scoring CTA of that head: warp w merges lists w, w + nw, ... (loads of a batch issued
+// together), then the warp lists are merged pairwise in shared memory; the k ids are written in
+// ascending order.  Ties go to the lower unit index.  Valid for k <= 32.
+__device__ void merge_select(const Dev& D, int hk, int n_mem, int n_split, uint64_t (*lists)[32], int nw) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint64_t* cb = D.cand + (int64_t)hk * D.score_splits_max * 32 + lane;
+    uint64_t m = 0;
+    for (int s0 = warp; s0 < n_split; s0 += nw * 4) {
+        uint64_t b[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int sp = s0 + nw * u;
+            b[u] = sp < n_split ? __ldcg(cb + (int64_t)sp * 32) : 0ull;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (s0 + nw * u < n_split) m = warp_merge_desc(m, b[u]);
+    }
+    __syncthreads();  // the caller's use of lists[] is over
+    lists[warp][lane] = m;
+    for (int stride = 1; stride < nw; stride *= 2) {
+        __syncthreads();
+        if ((warp % (2 * stride)) == 0 && warp + stride < nw)
+            lists[warp][lane] = warp_merge_desc(lists[warp][lane], lists[warp + stride][lane]);
+    }
+    __syncthreads();
+    if (warp == 0) {
+        const int kk = min(D.topk, n_mem);
+        uint64_t sk = (lane < kk) ? (uint64_t)(0xffffffffu - key_index(lists[0][lane])) : 0ull;
+        sk = warp_sort_desc(sk);  // ascending ids
+        if (lane < D.topk) {
+            int o = -1;
+            if (lane < kk) {
+                o = (int)(0xffffffffu - (uint32_t)sk);
+                if (o < 0 || o >= n_mem) {
+                    set_err(D, ERR_SEL_RANGE);
+                    o = 0;
+                }
+            }
+            D.sel[hk * D.topk + lane] = o;
+        }
+    }
+}
+
+// This CTA's top-32 list of KV head hk goes to D.cand; the last CTA of the head to finish (device
+// counter, threadfence pattern: no CTA waits for another) merges all lists into the selection and
+// re-arms the counter for the next launch.
+__device__ void publish_and_select(const Dev& D, int hk, int split, int n_mem, int n_split, uint64_t (*lists)[32],
+                                   int nw) {
+    __shared__ int is_last;
+    if (threadIdx.x < 32) D.cand[((int64_t)hk * D.score_splits_max + split) * 32 + threadIdx.x] = lists[0][threadIdx.x];
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) is_last = atomicAdd(&D.counters[hk], 1u) == (unsigned)(n_split - 1);
+    __syncthreads();
+    if (!is_last) return;
+    __threadfence();
+    merge_select(D, hk, n_mem, n_split, lists, nw);
+    if (threadIdx.x == 0) D.counters[hk] = 0u;
+}
+
 // Grid (n_split, Hkv), 512 threads.  Each unit is scored by a group of LPU lanes that split
 // its operand (16-byte loads issued in batches of 8), reduced inside the group; PER = 512 / LPU
-// units per CTA.  Writes the unit scores; the selection kernel picks the top-k.
+// units per CTA.  Writes the unit scores and, with do_select, the top-k (last CTA per head).
 constexpr int SC_THREADS = 512;
 constexpr int SC_WARPS = SC_THREADS / 32;
 
@@ -139,7 +201,7 @@ __global__ void __launch_bounds__(SC_THREADS, 2) k_score_topk(Dev D, int n_mem, 
                                                            const T* qraw, int do_select, int wait_first) {
     __shared__ float qb[128];
     if (wait_first) pdl_wait();  // the query sums (and the representatives) come from the kernels before
-    pdl_trigger();               // the selection kernel may start its prologue
+    pdl_trigger();               // the attention kernel may start its prologue
     const int split = blockIdx.x, hk = blockIdx.y;
     for (int i = threadIdx.x; i < D.half; i += blockDim.x) {
         float a = 0.f, b = 0.f;
@@ -235,7 +297,7 @@ __global__ void __launch_bounds__(SC_THREADS, 2) k_score_topk(Dev D, int n_mem, 
         D.uscore[(int64_t)hk * D.units_max + j] = sc;
         cand = make_key(sc, (uint32_t)j);
     }
-    if (do_select) {  // this CTA's top-32 (composite keys, descending) for the selection kernel
+    if (do_select) {  // this CTA's top-32 (composite keys, descending), then the head's selection
         __shared__ uint64_t lists[SC_WARPS][32];
         lists[warp][lane] = warp_sort_desc(cand);
 #pragma unroll
@@ -245,7 +307,7 @@ __global__ void __launch_bounds__(SC_THREADS, 2) k_score_topk(Dev D, int n_mem, 
                 lists[warp][lane] = warp_merge_desc(lists[warp][lane], lists[warp + stride][lane]);
         }
         __syncthreads();
-        if (warp == 0) D.cand[((int64_t)hk * D.score_splits_max + split) * 32 + lane] = lists[0][lane];
+        publish_and_select(D, hk, split, n_mem, n_split, lists, SC_WARPS);
     }
     // Without wait_first this grid may run while the preceding kernel runs (the scores do not
     // depend on it), but it must not complete before it: the kernels after rely on both.
@@ -287,13 +349,46 @@ __device__ __forceinline__ void rotated_query_sum(const Dev& D, int hk, int n_qt
     }
 }
 
+// One stage of the scoring pipeline: UB units' operand rows (C 16-byte chunks per lane each).
+template <int UB, int C>
+__device__ __forceinline__ void load_units(uint4 (&r)[UB][C], const uint4* base, int ub, int valid, int lane) {
+#pragma unroll
+    for (int u = 0; u < UB; ++u)
+#pragma unroll
+        for (int k = 0; k < C; ++k)
+            r[u][k] = (ub + u < valid) ? __ldg(base + (int64_t)(ub + u) * 32 * C + k * 32 + lane) : make_uint4(0, 0, 0, 0);
+}
+template <typename T, int MODE, int UB, int C, int V>
+__device__ __forceinline__ void dot_units(const uint4 (&r)[UB][C], const float (&qr)[C][V], float* acc) {
+#pragma unroll
+    for (int u = 0; u < UB; ++u) {
+        float a = 0.f;
+#pragma unroll
+        for (int k = 0; k < C; ++k) {
+            if (MODE == 0 && sizeof(T) == 2) {
+                const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&r[u][k]);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const float2 f = __bfloat1622float2(h2[c]);
+                    a += f.x * qr[k][2 * c] + f.y * qr[k][2 * c + 1];
+                }
+            } else {
+                const float* f = reinterpret_cast<const float*>(&r[u][k]);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) a += f[c] * qr[k][c];
+            }
+        }
+        acc[u] = a;
+    }
+}
+
 // Warp-per-32-units scoring.  Grid (n_split, Hkv), 32 * WPC threads; warp w of CTA s scores units
 // [(s * WPC + w) * 32, +32).  Lane l loads 16-byte chunks l, l + 32, ... (C per unit) of every
 // unit's operand -- consecutive lanes read consecutive 16 bytes, so each load instruction reads
 // 512 contiguous bytes -- and multiplies them with the matching slice of the rotated query sum,
 // held in registers.  The 32 partial sums of the warp's 32 units are then transposed across the
 // warp (recursive halving, 31 shuffles) so that lane u ends with unit u's score.  Writes the scores
-// and this CTA's top-32 list for the selection kernel.
+// and, with do_select, the top-k (see publish_and_select).
 template <typename T, int MODE, int C>
 __global__ void __launch_bounds__(256, 2) k_score_wpu(Dev D, int n_mem, int n_split, int n_qtiles, const T* qraw,
                                                       int do_select, int wait_first) {
@@ -302,10 +397,21 @@ __global__ void __launch_bounds__(256, 2) k_score_wpu(Dev D, int n_mem, int n_sp
     if (wait_first) pdl_wait();  // as in k_score_topk
     pdl_trigger();
     const int split = blockIdx.x, hk = blockIdx.y;
-    rotated_query_sum<T>(D, hk, n_qtiles, qraw, qb);
-    __syncthreads();
     constexpr int V = MODE == 0 ? (int)(16 / sizeof(T)) : 4;  // elements per 16-byte chunk
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    const int u0 = (split * nw + warp) * 32;
+    const uint4* base = MODE == 0
+        ? reinterpret_cast<const uint4*>((const T*)D.rep_keys + ((int64_t)hk * D.units_max + u0) * D.r * D.d)
+        : reinterpret_cast<const uint4*>(D.repsum + ((int64_t)hk * D.units_max + u0) * D.d);
+    // two register stages of UB units: the loads of one stage are in flight while the other is
+    // multiplied; the first stage is issued before the query sum, which it does not need
+    constexpr int UB = C >= 4 ? 2 : 4;
+    constexpr int NB = 32 / UB;
+    const int valid = n_mem - u0;
+    uint4 ra[UB][C], rb[UB][C];
+    load_units<UB, C>(ra, base, 0, valid, lane);
+    rotated_query_sum<T>(D, hk, n_qtiles, qraw, qb);
+    __syncthreads();
     float qr[C][V];
 #pragma unroll
     for (int k = 0; k < C; ++k) {
@@ -313,41 +419,13 @@ __global__ void __launch_bounds__(256, 2) k_score_wpu(Dev D, int n_mem, int n_sp
 #pragma unroll
         for (int v = 0; v < V; ++v) qr[k][v] = qb[i0 + v];
     }
-    const int u0 = (split * nw + warp) * 32;
-    const uint4* base = MODE == 0
-        ? reinterpret_cast<const uint4*>((const T*)D.rep_keys + ((int64_t)hk * D.units_max + u0) * D.r * D.d)
-        : reinterpret_cast<const uint4*>(D.repsum + ((int64_t)hk * D.units_max + u0) * D.d);
     float acc[32];
-    constexpr int UB = C >= 4 ? 4 : 8;  // units per load batch
 #pragma unroll
-    for (int ub = 0; ub < 32; ub += UB) {
-        uint4 raw[UB][C];
-#pragma unroll
-        for (int u = 0; u < UB; ++u)
-#pragma unroll
-            for (int k = 0; k < C; ++k)
-                raw[u][k] = (u0 + ub + u < n_mem) ? __ldg(base + (int64_t)(ub + u) * 32 * C + k * 32 + lane)
-                                                  : make_uint4(0, 0, 0, 0);
-#pragma unroll
-        for (int u = 0; u < UB; ++u) {
-            float a = 0.f;
-#pragma unroll
-            for (int k = 0; k < C; ++k) {
-                if (MODE == 0 && sizeof(T) == 2) {
-                    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw[u][k]);
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const float2 f = __bfloat1622float2(h2[c]);
-                        a += f.x * qr[k][2 * c] + f.y * qr[k][2 * c + 1];
-                    }
-                } else {
-                    const float* f = reinterpret_cast<const float*>(&raw[u][k]);
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) a += f[c] * qr[k][c];
-                }
-            }
-            acc[ub + u] = a;
-        }
+    for (int bi = 0; bi < NB; bi += 2) {
+        if (bi + 1 < NB) load_units<UB, C>(rb, base, (bi + 1) * UB, valid, lane);
+        dot_units<T, MODE, UB, C, V>(ra, qr, acc + bi * UB);
+        if (bi + 2 < NB) load_units<UB, C>(ra, base, (bi + 2) * UB, valid, lane);
+        if (bi + 1 < NB) dot_units<T, MODE, UB, C, V>(rb, qr, acc + (bi + 1) * UB);
     }
     // transpose-reduce: afterwards acc[0] of lane l is the full dot product of unit u0 + l
 #pragma unroll
@@ -375,59 +453,9 @@ __global__ void __launch_bounds__(256, 2) k_score_wpu(Dev D, int n_mem, int n_sp
                 lists[warp][lane] = warp_merge_desc(lists[warp][lane], lists[warp + stride][lane]);
         }
         __syncthreads();
-        if (warp == 0) D.cand[((int64_t)hk * D.score_splits_max + split) * 32 + lane] = lists[0][lane];
+        publish_and_select(D, hk, split, n_mem, n_split, lists, nw);
     }
     if (!wait_first) pdl_hold();  // this grid must not complete before its predecessor (see k_score_topk)
-}
-
-// Top-k of one KV head from the scoring CTAs' top-32 lists: one CTA of 1024 threads per KV
-// head; warp w merges lists w, w + 32, ... (loads of a batch issued together), then the 32
-// warp lists are merged pairwise in shared memory.  Ties go to the lower unit index (composite
-// keys).  Valid for k <= 32.
-constexpr int SEL_THREADS = 1024;
-constexpr int SEL_WARPS = SEL_THREADS / 32;
-
-__global__ void __launch_bounds__(SEL_THREADS) k_select_topk(Dev D, int n_mem, int n_split) {
-    __shared__ uint64_t lists[SEL_WARPS][32];
-    pdl_trigger();  // the attention kernel after this one is a late kernel as well
-    pdl_wait();     // the candidate lists are complete past this point
-    const int hk = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const uint64_t* cb = D.cand + (int64_t)hk * D.score_splits_max * 32 + lane;
-    uint64_t m = 0;
-    for (int s0 = warp; s0 < n_split; s0 += SEL_WARPS * 4) {
-        uint64_t b[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int s = s0 + SEL_WARPS * u;
-            b[u] = s < n_split ? __ldcg(cb + (int64_t)s * 32) : 0ull;
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-            if (s0 + SEL_WARPS * u < n_split) m = warp_merge_desc(m, b[u]);
-    }
-    lists[warp][lane] = m;
-#pragma unroll
-    for (int stride = 1; stride < SEL_WARPS; stride *= 2) {
-        __syncthreads();
-        if ((warp % (2 * stride)) == 0) lists[warp][lane] = warp_merge_desc(lists[warp][lane], lists[warp + stride][lane]);
-    }
-    __syncthreads();
-    if (warp == 0) {
-        const int kk = min(D.topk, n_mem);
-        uint64_t sk = (lane < kk) ? (uint64_t)(0xffffffffu - key_index(lists[0][lane])) : 0ull;
-        sk = warp_sort_desc(sk);  // ascending ids
-        if (lane < D.topk) {
-            int o = -1;
-            if (lane < kk) {
-                o = (int)(0xffffffffu - (uint32_t)sk);
-                if (o < 0 || o >= n_mem) {
-                    set_err(D, ERR_SEL_RANGE);
-                    o = 0;
-                }
-            }
-            D.sel[hk * D.topk + lane] = o;
-        }
-    }
 }
 
 // Selection for top_k > 32: one CTA per kv head sorts every unit's composite key in shared
@@ -567,8 +595,10 @@ cudaError_t launch_select(const Dev& D, int score_mode, int n_mem, int n_qtiles,
     int n_split;
     cudaError_t err;
     if (C == 1 || C == 2 || C == 4) {
-        int wpc = 8;  // warps per CTA: fewer when that still gives at least one CTA per SM
-        while (wpc > 1 && (int64_t)((n_mem + 32 * wpc - 1) / (32 * wpc)) * D.Hkv < 148) wpc /= 2;
+        // warps per CTA: 8, or 4 when that gives more CTAs for a wave of 148 SMs (not fewer than
+        // 4: the last CTA of a head merges the lists of the others)
+        int wpc = 8;
+        if ((int64_t)((n_mem + 255) / 256) * D.Hkv < 148) wpc = 4;
         n_split = (n_mem + 32 * wpc - 1) / (32 * wpc);
         if (n_split > D.score_splits_max) return cudaErrorInvalidValue;
         err = launch_wpu<T>(D, score_mode, C, dim3(n_split, D.Hkv), 32 * wpc, n_mem, n_split, n_qtiles,
@@ -587,11 +617,7 @@ cudaError_t launch_select(const Dev& D, int score_mode, int n_mem, int n_qtiles,
     if (err != cudaSuccess) return err;
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
-    if (fast) {
-        err = launch_k(k_select_topk, dim3(D.Hkv), dim3(SEL_THREADS), 0, st, pdl, D, n_mem, n_split);
-        ++*launches;
-        return err;
-    }
+    if (fast) return cudaSuccess;  // the scoring kernel's last CTA per head selected already
     int p2 = 1;
     while (p2 < n_mem) p2 <<= 1;  // n_mem <= 16384 (checked at create when top_k > 32)
     const size_t smem = (size_t)p2 * sizeof(uint64_t);
