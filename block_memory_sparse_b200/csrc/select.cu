@@ -449,7 +449,7 @@ __global__ void __launch_bounds__(256, 2) k_score_wpu(Dev D, int n_mem, int n_sp
         lists[warp][lane] = warp_sort_desc(cand);
         for (int stride = 1; stride < nw; stride *= 2) {
             __syncthreads();
-            if ((warp % (2 * stride)) == 0)
+            if ((warp % (2 * stride)) == 0 && warp + stride < nw)
                 lists[warp][lane] = warp_merge_desc(lists[warp][lane], lists[warp + stride][lane]);
         }
         __syncthreads();
@@ -595,10 +595,20 @@ cudaError_t launch_select(const Dev& D, int score_mode, int n_mem, int n_qtiles,
     int n_split;
     cudaError_t err;
     if (C == 1 || C == 2 || C == 4) {
-        // warps per CTA: 8, or 4 when that gives more CTAs for a wave of 148 SMs (not fewer than
-        // 4: the last CTA of a head merges the lists of the others)
+        // warps per CTA (4..8, each warp scores 32 units): the one whose CTA count fills the
+        // waves of 2 CTAs per SM on 148 SMs best, the larger on ties (fewer lists to merge); not
+        // fewer than 4 warps, as the last CTA of a head merges the lists of the others
         int wpc = 8;
-        if ((int64_t)((n_mem + 255) / 256) * D.Hkv < 148) wpc = 4;
+        double best = -1.0;
+        for (int w = 8; w >= 4; --w) {
+            const int64_t ctas = (int64_t)((n_mem + 32 * w - 1) / (32 * w)) * D.Hkv;
+            const int64_t waves = (ctas + 295) / 296;
+            const double eff = (double)ctas / (double)(waves * 296);
+            if (eff > best + 1e-9) {
+                best = eff;
+                wpc = w;
+            }
+        }
         n_split = (n_mem + 32 * wpc - 1) / (32 * wpc);
         if (n_split > D.score_splits_max) return cudaErrorInvalidValue;
         err = launch_wpu<T>(D, score_mode, C, dim3(n_split, D.Hkv), 32 * wpc, n_mem, n_split, n_qtiles,
