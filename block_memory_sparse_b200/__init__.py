@@ -63,6 +63,7 @@ SIGNATURES = {
     "infllm_decode_step": (ctypes.c_int, [_P, _P, _P, _P, _P]),
     "infllm_prefill": (ctypes.c_int, [_P, _P, _P, _P, ctypes.c_int64, ctypes.c_int32, _P]),
     "infllm_set_launch_chaining": (ctypes.c_int, [_P, ctypes.c_int32]),
+    "infllm_set_prefill_lookup": (ctypes.c_int, [_P, ctypes.c_int32]),
     "infllm_get_selection": (ctypes.c_int, [_P, _P]),
     "infllm_get_unit_scores": (ctypes.c_int, [_P, _P, ctypes.c_int32, ctypes.POINTER(ctypes.c_int32)]),
     "infllm_get_reps": (ctypes.c_int, [_P, ctypes.c_int32, ctypes.c_int32, _P]),
@@ -183,6 +184,10 @@ class InfLLMLayer:
         op = _dev_ptr(out, self.dtype, (n, self.Hq, self.d), "out")
         self._check(self.L.infllm_prefill(self.h, qp, kp, vp, n, int(chunk), op), "infllm_prefill")
         return out
+
+    def set_prefill_lookup(self, on: bool):
+        """off: chunks attend to sinks + window only (representatives still built); decode looks up."""
+        self._check(self.L.infllm_set_prefill_lookup(self.h, 1 if on else 0), "infllm_set_prefill_lookup")
 
     def set_launch_chaining(self, on: bool):
         self._check(self.L.infllm_set_launch_chaining(self.h, 1 if on else 0), "infllm_set_launch_chaining")

@@ -52,6 +52,7 @@ struct infllm_ctx {
     // launch chaining: within one API call every launch after the first may start early
     // (programmatic dependent launch); the first waits for whatever precedes it on the stream
     int chaining = 1;   // infllm_set_launch_chaining
+    int prefill_lookup = 1;  // infllm_set_prefill_lookup: unit lookup for chunks (decode always looks up)
     bool chain = false; // a kernel of the current call has been launched
     // lookups so far: lookup L packs its queries into slot L % 3, sums them into buffer L % 2 and
     // writes its selection to buffer L % 2 (so a lookup can run while the previous attention reads)
@@ -247,10 +248,10 @@ void record_attend(infllm_ctx* c, int64_t L, int64_t c0, int n, int nm, int kk, 
 
 // a4: attention of chunk [c0, c0 + n) with lookup L's packed queries and selection.
 template <typename T>
-infllm_status stage_attend(infllm_ctx* c, int64_t L, int64_t c0, int32_t n, void* out) {
+infllm_status stage_attend(infllm_ctx* c, int64_t L, int64_t c0, int32_t n, void* out, bool lookup) {
     const Dev D = lookup_dev(c, L);
     const int nm = (int)n_mem_at(c0, D.S, D.W, D.U);
-    const int kk = std::min(D.topk, nm);
+    const int kk = lookup ? std::min(D.topk, nm) : 0;  // without lookup: sinks and window only
     const int64_t B = (int64_t)D.S + (int64_t)D.U * nm;
     Prof p(c, K_ATTEND);
     if (c->use_tc && sizeof(T) == 2) {
@@ -277,16 +278,18 @@ infllm_status append_impl(infllm_ctx* c, const void* q, const void* k, const voi
 }
 
 template <typename T>
-infllm_status attend_impl(infllm_ctx* c, const void* q, int32_t n, void* out) {
+infllm_status attend_impl(infllm_ctx* c, const void* q, int32_t n, void* out, bool decoding = false) {
     const Dev& D = c->D;
     const int64_t c0 = c->pending_c0;
     c->pending = false;
     if (n == 0) return INFLLM_OK;
     const int64_t L = c->nlook++;
     const int nm = (int)n_mem_at(c0, D.S, D.W, D.U);
+    const bool lookup = decoding || c->prefill_lookup;
     infllm_status s = stage_prep<T>(c, q, c0, n, L);
-    if (s == INFLLM_OK && std::min(D.topk, nm) > 0) s = stage_select<T>(c, L, nm, (n + D.qt - 1) / D.qt, nullptr, true);
-    if (s == INFLLM_OK) s = stage_attend<T>(c, L, c0, n, out);
+    if (s == INFLLM_OK && lookup && std::min(D.topk, nm) > 0)
+        s = stage_select<T>(c, L, nm, (n + D.qt - 1) / D.qt, nullptr, true);
+    if (s == INFLLM_OK) s = stage_attend<T>(c, L, c0, n, out, lookup);
     return s;
 }
 
@@ -310,10 +313,11 @@ infllm_status prefill_impl(infllm_ctx* c, const char* q, const char* k, const ch
         infllm_status s = stage_store<T>(c, q + off * qrow, k + off * krow, v + off * krow, len(i));
         return s == INFLLM_OK ? stage_prep<T>(c, q + off * qrow, t0 + off, len(i), L0 + i) : s;
     };
+    const bool lk = c->prefill_lookup != 0;
     auto lookup = [&](int64_t i, bool wait_first) {
         const int64_t c0 = t0 + i * chunk;
         const int nm = (int)n_mem_at(c0, D.S, D.W, D.U);
-        if (std::min(D.topk, nm) == 0) return INFLLM_OK;
+        if (!lk || std::min(D.topk, nm) == 0) return INFLLM_OK;
         return stage_select<T>(c, L0 + i, nm, (len(i) + D.qt - 1) / D.qt, nullptr, wait_first);
     };
     infllm_status s = store_pack(0);
@@ -325,7 +329,7 @@ infllm_status prefill_impl(infllm_ctx* c, const char* q, const char* k, const ch
     for (int64_t i = 0; i < N && s == INFLLM_OK; ++i) {
         if (i + 1 < N) s = store_pack(i + 1);
         if (s == INFLLM_OK && i > 0) s = lookup(i, false);
-        if (s == INFLLM_OK) s = stage_attend<T>(c, L0 + i, t0 + i * chunk, len(i), out + i * chunk * qrow);
+        if (s == INFLLM_OK) s = stage_attend<T>(c, L0 + i, t0 + i * chunk, len(i), out + i * chunk * qrow, lk);
     }
     c->nlook = L0 + N;
     return s;
@@ -365,7 +369,7 @@ infllm_status decode_impl(infllm_ctx* c, const void* q, const void* k, const voi
     c->pending = false;
     if (c->D.G > 8) {  // wide groups: the chunk kernels handle a single token as well
         c->pending = true;
-        return attend_impl<T>(c, q, 1, out);
+        return attend_impl<T>(c, q, 1, out, /*decoding=*/true);
     }
     const int64_t L = c->nlook++;
     const Dev D = lookup_dev(c, L);
@@ -721,6 +725,12 @@ infllm_status infllm_set_score_mode(infllm_ctx* c, int32_t mode) {
     if (!c) return INFLLM_EINVAL;
     if (mode != INFLLM_SCORE_REPS && mode != INFLLM_SCORE_REPSUM) return fail(c, INFLLM_EINVAL, "unknown score_mode %d", mode);
     c->cfg.score_mode = mode;
+    return INFLLM_OK;
+}
+
+infllm_status infllm_set_prefill_lookup(infllm_ctx* c, int32_t enable) {
+    if (!c) return INFLLM_EINVAL;
+    c->prefill_lookup = enable ? 1 : 0;
     return INFLLM_OK;
 }
 

@@ -180,6 +180,14 @@ enum {
 };
 infllm_status infllm_set_profiling(infllm_ctx* ctx, int32_t enable);
 
+/* Unit lookup while pre-filling (default on).  enable = 0: chunks (infllm_attend_chunk,
+ * infllm_prefill) attend to sinks and the local window only, while representatives are still
+ * built for every evicted unit; infllm_decode_step always looks up.  This is the ablation
+ * "memory lookup during both encoding and decoding instead of decoding only" of "InfLLM:
+ * Training-Free Long-Context Extrapolation for LLMs with an Efficient Context Memory" (research-map
+ * summary, "Measured effects"), run with lookup during decoding only. */
+infllm_status infllm_set_prefill_lookup(infllm_ctx* ctx, int32_t enable);
+
 /* Launch chaining (default on): inside one call, every kernel launch after the first is a
  * programmatic dependent launch, so a kernel that does not need its predecessor's results
  * starts while that predecessor runs; the first launch of a call always waits for the work

@@ -92,6 +92,7 @@ def test_null_arguments(lib):
     assert lib.infllm_decode_step(None, None, None, None, None) == 1
     assert lib.infllm_prefill(None, None, None, None, 0, 1, None) == 1
     assert lib.infllm_set_launch_chaining(None, 1) == 1
+    assert lib.infllm_set_prefill_lookup(None, 0) == 1
     assert lib.infllm_get_selection(None, None) == 1
     assert lib.infllm_get_stats(None, None) == 1
     assert lib.infllm_last_error(None) == b"null context"

@@ -129,6 +129,62 @@ def test_decode_matches_oracle(cuda_ok):
     glayer.close()
 
 
+def test_lookup_while_decoding_only(cuda_ok):
+    """Ablation of lookup during pre-filling (research-map summary, "Measured effects"): chunks attend
+    to sinks + window only, the representatives are still built, decode steps look up as usual."""
+    import torch
+    w = synth.SMALL["small_decode"]
+    cfg = w.as_config()
+    glayer = make_layer(w)
+    glayer.set_prefill_lookup(False)
+    src = Source(w)
+    olayer = O.OracleLayer(dict(cfg, top_k=0), rep_method="linear")  # representatives do not depend on k
+    tol = TOL[w.dtype]
+    T0 = w.n_tokens
+    for c0 in range(0, T0, w.build_chunk):
+        n = min(w.build_chunk, T0 - c0)
+        q, k, v = (to_torch(x) for x in synth.gen_chunk(w, c0, n))
+        glayer.append_chunk(q, k, v)
+        out = glayer.attend_chunk(q)
+        olayer.append_chunk(src.q(c0, n), src.k(c0, n), src.v(c0, n))
+        ref = olayer.attend_chunk()
+        torch.cuda.synchronize()
+        assert float(np.max(np.abs(to_np64(out) - ref))) <= tol, c0
+        assert glayer.stats()["n_selected"] == 0 and bool((glayer.selection() < 0).all())
+    assert glayer.stats()["units_with_reps"] == O.n_mem(T0 - n, w.n_sink, w.window, w.unit_size)
+    olayer.cfg = dict(cfg)  # decoding looks up with the configured k
+    for s in range(6):
+        t = T0 + s
+        q, k, v = synth.gen_chunk(w, t, 1)
+        out = glayer.decode_step(to_torch(q), to_torch(k), to_torch(v))
+        olayer.append_chunk(src.q(t, 1), src.k(t, 1), src.v(t, 1))
+        gsel = glayer.selection()
+        nm = O.n_mem(t, w.n_sink, w.window, w.unit_size)
+        assert glayer.stats()["n_selected"] == min(w.top_k, nm) > 0
+        greps = glayer.reps(0, nm)
+        saved = olayer.reps
+        olayer.reps = [[list(greps[h, j]) for h in range(w.n_kv_heads)] for j in range(nm)]
+        ref = olayer.attend_chunk(sel_override=[[int(x) for x in gsel[h] if x >= 0] for h in range(w.n_kv_heads)])
+        compare_selection(gsel, olayer.last["sigma"], w.top_k)
+        olayer.reps = saved
+        torch.cuda.synchronize()
+        assert float(np.max(np.abs(to_np64(out) - ref))) <= tol, s
+    # the whole-prompt entry point obeys the switch too
+    layer2 = make_layer(w)
+    layer2.set_prefill_lookup(False)
+    q, k, v = (to_torch(x) for x in synth.gen_chunk(w, 0, T0))
+    o2 = layer2.prefill(q, k, v, w.build_chunk)
+    torch.cuda.synchronize()
+    olayer2 = O.OracleLayer(dict(cfg, top_k=0), rep_method="linear")
+    for c0 in range(0, T0, w.build_chunk):
+        n = min(w.build_chunk, T0 - c0)
+        olayer2.append_chunk(src.q(c0, n), src.k(c0, n), src.v(c0, n))
+        ref = olayer2.attend_chunk()
+        assert float(np.max(np.abs(to_np64(o2[c0:c0 + n]) - ref))) <= tol, c0
+    glayer.close()
+    layer2.close()
+
+
 def test_needle_selected_on_gpu(cuda_ok):
     w = synth.SMALL["small_needle"]
     j_star = synth.needle_info(w)[0]
