@@ -29,7 +29,7 @@ import numpy as np  # noqa: E402
 
 import synth  # noqa: E402
 
-METRIC = "prefill tok/s and decode us/step at 128K-1M ctx; % of HBM / TC roofline"
+METRIC = "prefill tok/s and decode \u00b5s/step at 128K\u20131M ctx; % of HBM / TC roofline"
 
 
 def peaks():
@@ -195,6 +195,15 @@ def attn_traffic():
     return traffic if have == want else None
 
 
+def workload_config(w, world):
+    """The `config` object of the JSON line (the same for both arms)."""
+    return {"workload": f"{w.name}: {w.n_q_heads}q/{w.n_kv_heads}kv heads, d={w.head_dim}, "
+                        f"{w.n_tokens} tokens in {w.chunk}-token chunks, W={w.window}, S={w.n_sink}, "
+                        f"U={w.unit_size}, r={w.n_reps}, k={w.top_k}, base={w.rope_base:g}",
+            "global_batch": 1 * world, "seq_len": w.n_tokens, "parallelism": f"replicas x{world}",
+            "l2": "inputs larger than L2 (1.6 GB of Q/K/V per step)"}
+
+
 def run_ours(args, rank, world):
     import torch
     from block_memory_sparse_b200 import InfLLMLayer
@@ -276,11 +285,7 @@ def run_ours(args, rank, world):
     res = {"metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world, "steps": args.steps,
            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
            "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded Philox normals, K channel bias N(0,4))",
-           "config": {"workload": f"{w.name}: {w.n_q_heads}q/{w.n_kv_heads}kv heads, d={w.head_dim}, "
-                                  f"{w.n_tokens} tokens in {w.chunk}-token chunks, W={w.window}, S={w.n_sink}, "
-                                  f"U={w.unit_size}, r={w.n_reps}, k={w.top_k}, base={w.rope_base:g}",
-                      "global_batch": 1 * world, "seq_len": w.n_tokens, "parallelism": f"replicas x{world}",
-                      "l2": "inputs larger than L2 (1.6 GB of Q/K/V per step)"},
+           "config": workload_config(w, world),
            "roofline": roof, "gpu_launches": launches,
            "clocks": clk.summary(),
            "time_split_ms_per_step": {k: split[f"ms_{k}"]
@@ -468,18 +473,17 @@ def run_reference(args, rank, world):
     if rank != 0:
         return None
     times = []
-    for i in range(args.warmup + args.steps):
+    for i in range(args.warmup + max(1, args.steps)):
         n, s, what = oracle_sample(args.workload)
         if i >= args.warmup:
             times.append(s)
     tot = sum(times)
     w = synth.WORKLOADS[args.workload]
     v = n * len(times) / tot
-    return {"impl": "reference", "metric": METRIC, "value": v, "unit": "tok/s", "n_gpus": 1, "steps": args.steps,
+    return {"impl": "reference", "metric": METRIC, "value": v, "unit": "tok/s", "n_gpus": 1, "steps": len(times),
             "warmup": args.warmup, "ms_per_step": tot / len(times) * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded Philox normals)",
-            "config": {"workload": f"{w.name} (oracle on one steady chunk per step)", "global_batch": 1,
-                       "seq_len": w.n_tokens, "parallelism": "host cores"},
+            "config": workload_config(w, 1),
             "cpu_baseline": {"value": v, "unit": "tok/s", "cores": cpu_threads(), "kind": "oracle", "sample": what},
             "e2e": {"value": v, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
