@@ -180,19 +180,26 @@ ATTN_PROFILE = os.path.join(ROOT, "profiles", "k_attn_tc_mistral_128k.md")
 ATTN_SOURCE = os.path.join(ROOT, "block_memory_sparse_b200", "csrc", "attend_tc.cu")
 
 
-def attn_traffic():
-    """DRAM bytes per attention launch from the committed ncu summary, or None when the kernel
-    source has changed since the counters were taken (its sha256 is recorded in the summary)."""
+def attn_device_hash():
+    """sha256 of the attention kernel's device code: attend_tc.cu up to its host-side part (the
+    tensor-map encoding and the launcher), which does not change what the kernel moves."""
     import hashlib
+    src = open(ATTN_SOURCE, "rb").read()
+    cut = src.find(b"typedef CUresult (*EncodeTiledFn)")
+    return hashlib.sha256(src if cut < 0 else src[:cut]).hexdigest()
+
+
+def attn_traffic():
+    """DRAM bytes per attention launch from the committed ncu summary, or None when the kernel's
+    device code has changed since the counters were taken (its sha256 is recorded there)."""
     import re
     try:
         txt = open(ATTN_PROFILE).read()
-        want = re.search(r"attend_tc\.cu sha256: ([0-9a-f]{64})", txt).group(1)
+        want = re.search(r"attend_tc\.cu device-code sha256: ([0-9a-f]{64})", txt).group(1)
         traffic = float(re.search(r"dram bytes per launch: ([0-9.eE+]+)", txt).group(1))
     except (OSError, AttributeError, ValueError):
         return None
-    have = hashlib.sha256(open(ATTN_SOURCE, "rb").read()).hexdigest()
-    return traffic if have == want else None
+    return traffic if attn_device_hash() == want else None
 
 
 def workload_config(w, world):

@@ -485,12 +485,9 @@ bool make_tc_maps(const Dev& D, void* out) {
 cudaError_t launch_attend_tc(const Dev& D, int64_t c0, int n, int kk, int64_t B, int par, void* out, cudaStream_t st,
                              const void* tmaps, bool pdl) {
     if (n <= 0) return cudaSuccess;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(k_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    static std::atomic<unsigned long long> attr_done{0};
+    cudaError_t e = smem_limit_once(k_attn_tc, SMEM_BYTES, attr_done);
+    if (e != cudaSuccess) return e;
     const int tiles = (n + D.qt - 1) / D.qt;
     return launch_k(k_attn_tc, dim3(tiles, D.Hkv), dim3(NTHREADS), SMEM_BYTES, st, pdl,
                     *reinterpret_cast<const TcMaps*>(tmaps), D, c0, n, kk, B, par, (__nv_bfloat16*)out);

@@ -1,6 +1,8 @@
 // Shared device-side definitions for the InfLLM layer kernels (sm_100a).
 #pragma once
 
+#include <atomic>
+
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -179,6 +181,20 @@ __device__ __forceinline__ float2 cs_abs(const double2* tab, int half, int64_t t
 __host__ __device__ __forceinline__ int64_t n_mem_at(int64_t c0, int S, int W, int U) {
     int64_t x = c0 - (int64_t)W - (int64_t)S;
     return x > 0 ? x / U : 0;
+}
+
+// Raise `kernel`'s dynamic shared-memory limit to `bytes` once per device (the attribute is per
+// device; `done` holds one bit per device ordinal, ordinals >= 64 are set on every call).
+template <typename... KArgs>
+inline cudaError_t smem_limit_once(void (*kernel)(KArgs...), int bytes, std::atomic<unsigned long long>& done) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const unsigned long long bit = dev < 64 ? 1ull << dev : 0ull;
+    if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
+    return e;
 }
 
 // Launch `kernel` on `st`, with programmatic dependent launch when `pdl` is set.

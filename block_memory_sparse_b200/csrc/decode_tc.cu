@@ -373,12 +373,9 @@ cudaError_t launch_decode_tc(const Dev& D, const void* q, int64_t t, int kk, int
     if (nst + nut + nwt > D.dec_splits_max || nst + nut + nwt > MERGE_SLICES * MERGE_BATCH) return cudaErrorInvalidValue;
     const int tiles = part == 1 ? nut : nst + nwt;
     if (tiles == 0) return cudaSuccess;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(k_decode_attn, cudaFuncAttributeMaxDynamicSharedMemorySize, DSMEM);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    static std::atomic<unsigned long long> attr_done{0};
+    cudaError_t e = smem_limit_once(k_decode_attn, DSMEM, attr_done);
+    if (e != cudaSuccess) return e;
     return launch_k(k_decode_attn, dim3(tiles, D.Hkv), dim3(DTHREADS), DSMEM, st, pdl,
                     *reinterpret_cast<const TcMaps*>(tmaps), D, (const __nv_bfloat16*)q, t, kk, B, part);
 }

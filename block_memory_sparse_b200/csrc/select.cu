@@ -525,12 +525,9 @@ cudaError_t launch_prep(const Dev& D, const void* q, int64_t c0, int n, int par,
     const int threads = 256;
     const int nv = D.half / (16 / (int)sizeof(T));
     const size_t smem = (threads / nv) * D.d * sizeof(float) + (size_t)D.qt * D.half * sizeof(float2);
-    static bool attr_set = false;  // up to 80 KB (one KV head per q head: 128 queries a tile)
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(k_prep<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    static std::atomic<unsigned long long> attr_done{0};  // up to 80 KB (one q head per KV head: 128 queries a tile)
+    cudaError_t e = smem_limit_once(k_prep<T>, 96 * 1024, attr_done);
+    if (e != cudaSuccess) return e;
     return launch_k(k_prep<T>, dim3(tiles, D.Hkv), dim3(threads), smem, st, pdl, D, (const T*)q, c0, n, par);
 }
 
