@@ -76,7 +76,7 @@ typedef struct {
     int32_t n_reps;      /* r in [1, min(U, 32)]: representative tokens per unit */
     int32_t top_k;       /* k >= 0: units attended per chunk and kv head */
     int32_t max_chunk;   /* largest n accepted by append/attend */
-    int64_t max_tokens;  /* capacity of the token stream */
+    int64_t max_tokens;  /* capacity of the token stream; max_tokens / unit_size + 1 <= 16384 units */
     double rope_base;    /* RoPE base (> 1) */
     int32_t dtype;       /* infllm_dtype of q/k/v/out */
     int32_t score_mode;  /* infllm_score_mode */
