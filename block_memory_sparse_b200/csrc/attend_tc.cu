@@ -7,21 +7,23 @@
 //
 // One CTA per (128 packed query rows, KV head): the rows are G q heads x 128/G consecutive
 // queries of one KV group, so every K/V tile is read once per group.  Warp roles:
-//   warp 0      TMA producer: K and V tiles (3-stage rings)
-//   warp 1      MMA issuer:   S_i = Q K_i^T into TMEM (double buffered), O += P_i V_i; both A
-//                             operands (Q and P) are read from TMEM
+//   warp 0      TMA producer: the two query tiles once, then K and V tiles (2-stage rings)
+//   warp 1      MMA issuer:   S_i = Q K_i^T into TMEM (double buffered, Q and K from shared
+//                             memory); O_h += P_i[:, half h] V_i[half h] with P read from TMEM
 //   warps 2..9  softmax:      two threads per row (warps w and w + 4 share a TMEM lane quarter
-//                             and split the tile's 128 columns in halves); the row max is
-//                             combined through shared memory, each exponentiates its own 64: online
-//                             softmax with lazy rescale of O (only when the running max grows by
-//                             > 2^8), P_i as bf16 into the TMEM columns of S_i; at the end the
-//                             two halves' row sums are added and each thread stores 64 outputs.
-// The two rotated query tiles (R(W)q for sinks and memory, R(t)q for the window) are stored into
-// TMEM once by the softmax warps, which frees shared memory for 3-stage K/V rings.  Each softmax
-// warp writes its half of P_i over the first 32 columns of its own half of S_i (it has read them;
-// the partner warp never reads them), so S_i and P_i share a buffer, double buffered: the
-// exponentials of tile i overlap the PV product of tile i - 1, and QK of tile i + 2 (same buffer)
-// is issued after PV(i) -- the tensor pipe executes one thread's MMAs in issue order.
+//                             and split the tile's 128 columns in halves).  Each half runs its own
+//                             online softmax over its columns of every tile -- its own running
+//                             max, sum and accumulator O_h -- so the two never wait for each
+//                             other inside the loop; O_h is rescaled lazily (only when the half's
+//                             max grows by > 2^8).  P_i goes as bf16 into the TMEM columns of S_i.
+//                             After the last tile the halves exchange (max, sum) once through
+//                             shared memory and each thread stores 64 outputs of the merged row.
+// Splitting a row's keys in two and merging the partial softmaxes at the end is exact (up to
+// rounding): it is the log-sum-exp combination of two disjoint key sets.  Each softmax warp writes
+// its half of P_i over the first 32 columns of its own half of S_i (it has read them; the partner
+// warp never reads them), so S_i and P_i share a buffer, double buffered: the exponentials of tile
+// i overlap the PV product of tile i - 1, and QK of tile i + 2 (same buffer) is issued after
+// PV(i) -- the tensor pipe executes one thread's MMAs in issue order.
 // Sinks and memory tiles use R(W) q with raw keys; window tiles use R(t) q with R(n) k.
 #include <cuda.h>
 #include <math.h>
@@ -42,26 +44,25 @@ constexpr int NTHREADS = 320;  // producer warp, MMA warp, 8 softmax warps
 constexpr int NSOFT = 256;     // softmax threads
 constexpr uint32_t TILE = BN * HD * 2;  // bytes of one bf16 128 x 128 tile
 constexpr uint32_t HALF = TILE / 2;     // one 64-column swizzle block (128 rows x 128 B)
-constexpr int NSTAGE = 3;                      // K and V ring depth
-constexpr int OFF_K = 0;
+constexpr int NSTAGE = 2;                      // K and V ring depth
+constexpr int OFF_QM = 0;                      // R(W) q tile (sinks and memory units)
+constexpr int OFF_QW = OFF_QM + (int)TILE;     // R(t) q tile (window)
+constexpr int OFF_K = OFF_QW + (int)TILE;
 constexpr int OFF_V = OFF_K + NSTAGE * (int)TILE;
 constexpr int OFF_BAR = OFF_V + NSTAGE * (int)TILE;
-constexpr int OFF_LSUM = OFF_BAR + 256;            // [2][128] row sums of the two column halves
-constexpr int OFF_MXS = OFF_LSUM + 2 * 128 * 4;    // [2 tile parities][2 halves][128] half-maxima
-constexpr int OFF_SEL = OFF_MXS + 2 * 2 * 128 * 4; // selected unit ids of this KV head
+constexpr int OFF_LSUM = OFF_BAR + 256;            // [2 halves][128] row sums
+constexpr int OFF_MREF = OFF_LSUM + 2 * 128 * 4;   // [2 halves][128] reference maxima (log2 units)
+constexpr int OFF_SEL = OFF_MREF + 2 * 128 * 4;    // selected unit ids of this KV head
 constexpr int MAX_SEL = 256;
 constexpr int SMEM_BYTES = OFF_SEL + MAX_SEL * 4 + 1024;  // + alignment slack
-constexpr uint32_t TMEM_COLS = 512;  // S0 / P0 [0,128), S1 / P1 [128,256), O [256,384), Qm [384,448), Qw [448,512)
-constexpr uint32_t TM_O = 256;
-constexpr uint32_t TM_QM = 384;  // R(W) q, bf16 pairs
-constexpr uint32_t TM_QW = 448;  // R(t) q, bf16 pairs
+constexpr uint32_t TMEM_COLS = 512;  // S0 / P0 [0,128), S1 / P1 [128,256), O_0 [256,384), O_1 [384,512)
+constexpr uint32_t TM_O = 256;       // O_h: the products with the keys of column half h of every tile
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float RESCALE_LOG2 = 8.0f;
 constexpr int ERR_TIMEOUT = 16;
 
 struct Bars {
     uint64_t q, kfull[NSTAGE], kempty[NSTAGE], vfull[NSTAGE], vempty[NSTAGE], sfull[2], pfull, pvdone;
-    uint64_t mx[4];  // per TMEM lane quarter: both softmax warps of the rows posted their half-max
     uint32_t tmem;
     int abort;
 };
@@ -109,9 +110,19 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Bars* b
 }
 
 __device__ void producer(const TcMaps& maps, const Plan& P, const Dev& D, uint8_t* sm, Bars* bars) {
+    ptx::prefetch_tmap(&maps.qm);
+    ptx::prefetch_tmap(&maps.qw);
     ptx::prefetch_tmap(&maps.kraw);
     ptx::prefetch_tmap(&maps.krot);
     ptx::prefetch_tmap(&maps.v);
+    {   // both rotated query tiles of this CTA's 128 packed rows (slot par of the query buffers)
+        const int y = P.par * (int)D.qrows_max + P.a * BM;
+        ptx::mbar_expect_tx(&bars->q, 2 * TILE);
+        ptx::tma_load_3d(sm + OFF_QM, &maps.qm, &bars->q, 0, y, P.hk);
+        ptx::tma_load_3d(sm + OFF_QM + HALF, &maps.qm, &bars->q, 64, y, P.hk);
+        ptx::tma_load_3d(sm + OFF_QW, &maps.qw, &bars->q, 0, y, P.hk);
+        ptx::tma_load_3d(sm + OFF_QW + HALF, &maps.qw, &bars->q, 64, y, P.hk);
+    }
     int issued = 0;
     for (int i = 0; i < P.NT; ++i) {
         const int s = i % NSTAGE;
@@ -137,14 +148,16 @@ __device__ void producer(const TcMaps& maps, const Plan& P, const Dev& D, uint8_
             ptx::mbar_wait(&bars->kfull[i % NSTAGE], (uint32_t)(i / NSTAGE) & 1, 1ll << 28);
             ptx::mbar_wait(&bars->vfull[i % NSTAGE], (uint32_t)(i / NSTAGE) & 1, 1ll << 28);
         }
+        ptx::mbar_wait(&bars->q, 0, 1ll << 28);
     }
 }
 
 __device__ void mma_issuer(const Plan& P, const Dev& D, uint8_t* sm, Bars* bars, uint32_t tmem) {
     constexpr uint32_t IDESC_QK = ptx::idesc_bf16_f32(BM, BN, false, false);
     constexpr uint32_t IDESC_PV = ptx::idesc_bf16_f32(BM, HD, false, true);
-    if (!wait_bar(&bars->q, 0, bars, D)) return;  // the query tiles are in TMEM
+    if (!wait_bar(&bars->q, 0, bars, D)) return;  // the query tiles have landed
     ptx::tc_fence_after();
+    const uint32_t qm = ptx::smem_u32(sm + OFF_QM), qw = ptx::smem_u32(sm + OFF_QW);
     const uint32_t kb = ptx::smem_u32(sm + OFF_K), vb = ptx::smem_u32(sm + OFF_V);
     for (int i = 0; i <= P.NT; ++i) {
         if (i < P.NT) {
@@ -153,13 +166,13 @@ __device__ void mma_issuer(const Plan& P, const Dev& D, uint8_t* sm, Bars* bars,
             const int s = i % NSTAGE, b = i & 1;
             if (!wait_bar(&bars->kfull[s], (uint32_t)(i / NSTAGE) & 1, bars, D)) return;
             ptx::tc_fence_after();
-            const uint32_t qa = tmem + (P.tile(D, i).kind == 2 ? TM_QW : TM_QM);
+            const uint32_t qa = P.tile(D, i).kind == 2 ? qw : qm;
             const uint32_t ka = kb + s * TILE;
 #pragma unroll
             for (int ks = 0; ks < HD / 16; ++ks) {
                 const uint32_t off = (uint32_t)(ks >> 2) * HALF + (uint32_t)(ks & 3) * 32;
-                ptx::mma_bf16_ts(tmem + b * BN, qa + (uint32_t)ks * 8, ptx::sdesc_sw128(ka + off, 16, 1024), IDESC_QK,
-                                 ks > 0 ? 1u : 0u);
+                ptx::mma_bf16(tmem + b * BN, ptx::sdesc_sw128(qa + off, 16, 1024), ptx::sdesc_sw128(ka + off, 16, 1024),
+                              IDESC_QK, ks > 0 ? 1u : 0u);
             }
             ptx::mma_commit(&bars->sfull[b]);
             ptx::mma_commit(&bars->kempty[s]);
@@ -171,10 +184,11 @@ __device__ void mma_issuer(const Plan& P, const Dev& D, uint8_t* sm, Bars* bars,
             ptx::tc_fence_after();
             const uint32_t va = vb + sj * TILE;
 #pragma unroll
-            for (int ks = 0; ks < BN / 16; ++ks)  // keys 16 ks ..: half ks / 4 of P_j, 8 columns per step
-                ptx::mma_bf16_ts(tmem + TM_O, tmem + bj * BN + (uint32_t)(ks >> 2) * 64 + (uint32_t)(ks & 3) * 8,
+            for (int ks = 0; ks < BN / 16; ++ks)  // keys 16 ks ..: half h = ks / 4 of P_j into O_h
+                ptx::mma_bf16_ts(tmem + TM_O + (uint32_t)(ks >> 2) * HD,
+                                 tmem + bj * BN + (uint32_t)(ks >> 2) * 64 + (uint32_t)(ks & 3) * 8,
                                  ptx::sdesc_sw128(va + (uint32_t)ks * 2048, HALF, 1024), IDESC_PV,
-                                 (j > 0 || ks > 0) ? 1u : 0u);
+                                 (j > 0 || (ks & 3) > 0) ? 1u : 0u);
             ptx::mma_commit(&bars->pvdone);
             ptx::mma_commit(&bars->vempty[sj]);
         }
@@ -206,33 +220,23 @@ struct PvTrack {
     }
 };
 
-__device__ void softmax_role(const Plan& P, const Dev& D, Bars* bars, float* lsum, float* mxs, uint32_t tmem,
+__device__ void softmax_role(const Plan& P, const Dev& D, Bars* bars, float* lsum, float* mref, uint32_t tmem,
                              int64_t c0, int n, __nv_bfloat16* __restrict__ out, int warp, int lane) {
     const int quarter = warp & 3;        // TMEM lanes this warp may access
     const int half = (warp - 2) >> 2;    // columns [64 half, 64 half + 64) of every tile are this thread's
     const int row = quarter * 32 + lane;
     const uint32_t tl_addr = tmem + ((uint32_t)(quarter * 32) << 16);
+    const uint32_t o_addr = tl_addr + TM_O + (uint32_t)half * HD;  // this thread's row of O_half
     const int hg = row / D.qt, tl = P.a * D.qt + row % D.qt;
     const bool valid = tl < n;
     const int64_t t = c0 + tl;
     const float sc = D.inv_sqrt_d * LOG2E;  // logits in log2 units: s * sc
-    float m_used = -INFINITY, l = 0.f;      // running max (log2 units) and this half's sum
+    // This half's own online softmax: reference max (log2 units), sum, and O_half; the two
+    // halves of a row meet once, after the last tile.
+    float m_used = -INFINITY, l = 0.f;
     float s[64];
     PvTrack pv;
     bool ok = true;
-    {   // this thread's query row into TMEM: half 0 stores R(W) q, half 1 stores R(t) q
-        const __nv_bfloat16* src = (const __nv_bfloat16*)(half == 0 ? D.Qm : D.Qw) +
-                                   (((int64_t)P.hk * 3 + P.par) * D.qrows_max + (int64_t)P.a * BM + row) * HD;
-        uint4 qv[16];
-#pragma unroll
-        for (int c = 0; c < 16; ++c) qv[c] = __ldg(reinterpret_cast<const uint4*>(src) + c);
-        const uint32_t qcol = tl_addr + (half == 0 ? TM_QM : TM_QW);
-        ptx::tmem_st32(qcol, reinterpret_cast<const float*>(qv));
-        ptx::tmem_st32(qcol + 32, reinterpret_cast<const float*>(qv + 8));
-        ptx::tmem_wait_st();
-        ptx::tc_fence_before();
-        ptx::mbar_arrive(&bars->q);
-    }
     for (int i = 0; i < P.NT; ++i) {
         const int b = i & 1;
         if (!warp_wait(&bars->sfull[b], (uint32_t)(i >> 1) & 1, bars, D)) {
@@ -265,21 +269,11 @@ __device__ void softmax_role(const Plan& P, const Dev& D, Bars* bars, float* lsu
                 mq[c & 7] = fmaxf(mq[c & 7], s[c]);
             }
         }
-        float mx = fmaxf(fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])), fmaxf(fmaxf(mq[4], mq[5]), fmaxf(mq[6], mq[7])));
-        // the row max over both halves: post this half's, wait (bounded) until the partner warp
-        // posted its own for this tile, read it.  Slots alternate by tile parity; a warp reaches
-        // tile i + 2 only after its partner arrived for tile i + 1, i.e. after it read slot i.
-        mxs[((i & 1) * 2 + half) * 128 + row] = mx;
-        ptx::mbar_arrive(&bars->mx[quarter]);
-        if (!warp_wait(&bars->mx[quarter], (uint32_t)i & 1, bars, D)) {
-            ok = false;
-            break;
-        }
-        mx = fmaxf(mx, mxs[((i & 1) * 2 + (1 - half)) * 128 + row]);
+        const float mx = fmaxf(fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])), fmaxf(fmaxf(mq[4], mq[5]), fmaxf(mq[6], mq[7])));
         const float mt = mx * sc;
         const bool need = mt > m_used + RESCALE_LOG2;
         const float m_new = need ? mt : m_used;
-        if (i >= 1 && __any_sync(0xffffffffu, need)) {  // O must hold every earlier product first
+        if (i >= 1 && __any_sync(0xffffffffu, need)) {  // O_half must hold every earlier product first
             if (!pv.upto(i - 1, bars, D)) {
                 ok = false;
                 break;
@@ -288,13 +282,13 @@ __device__ void softmax_role(const Plan& P, const Dev& D, Bars* bars, float* lsu
             const float f = need ? ex2(m_used - m_new) : 1.f;
             l *= f;
 #pragma unroll
-            for (int c4 = 0; c4 < 2; ++c4) {
+            for (int c4 = 0; c4 < HD / 32; ++c4) {
                 float o[32];
-                ptx::tmem_ld32(tl_addr + TM_O + half * 64 + c4 * 32, o);
+                ptx::tmem_ld32(o_addr + c4 * 32, o);
                 ptx::tmem_wait_ld();
 #pragma unroll
                 for (int e = 0; e < 32; ++e) o[e] *= f;
-                ptx::tmem_st32(tl_addr + TM_O + half * 64 + c4 * 32, o);
+                ptx::tmem_st32(o_addr + c4 * 32, o);
             }
         }
         m_used = m_new;
@@ -324,18 +318,25 @@ __device__ void softmax_role(const Plan& P, const Dev& D, Bars* bars, float* lsu
         ptx::mbar_arrive(&bars->pfull);
     }
     ok = ok && pv.upto(P.NT - 1, bars, D);
-    // the two halves' sums of this row (every softmax thread reaches this barrier: all waits above
-    // are bounded)
+    // the two halves of the row meet: O = (2^(m_0 - M) O_0 + 2^(m_1 - M) O_1) / (same weights on
+    // l_0, l_1), M = max(m_0, m_1).  Every softmax thread reaches this barrier: all waits above
+    // are bounded.
     lsum[half * 128 + row] = l;
+    mref[half * 128 + row] = m_used;
     asm volatile("bar.sync 1, %0;" ::"n"(NSOFT) : "memory");
     if (!__all_sync(0xffffffffu, ok)) return;
     ptx::tc_fence_after();
-    const float inv = 1.f / (l + lsum[(1 - half) * 128 + row]);
+    const float m0 = mref[row], m1 = mref[128 + row];
+    const float M = fmaxf(m0, m1);
+    const float f0 = m0 == -INFINITY ? 0.f : ex2(m0 - M), f1 = m1 == -INFINITY ? 0.f : ex2(m1 - M);
+    const float inv = 1.f / (lsum[row] * f0 + lsum[128 + row] * f1);
+    const float g0 = f0 * inv, g1 = f1 * inv;
     __nv_bfloat16* orow = out + ((int64_t)tl * D.Hq + P.hk * D.G + hg) * HD + half * 64;
-#pragma unroll
+#pragma unroll 1
     for (int c4 = 0; c4 < 2; ++c4) {
-        float o[32];
-        ptx::tmem_ld32(tl_addr + TM_O + half * 64 + c4 * 32, o);
+        float o0[32], o1[32];
+        ptx::tmem_ld32(tl_addr + TM_O + half * 64 + c4 * 32, o0);
+        ptx::tmem_ld32(tl_addr + TM_O + HD + half * 64 + c4 * 32, o1);
         ptx::tmem_wait_ld();
         if (valid) {
 #pragma unroll
@@ -343,7 +344,9 @@ __device__ void softmax_role(const Plan& P, const Dev& D, Bars* bars, float* lsu
                 uint32_t w4[4];
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    __nv_bfloat162 h = __floats2bfloat162_rn(o[e * 8 + 2 * q] * inv, o[e * 8 + 2 * q + 1] * inv);
+                    const int k = e * 8 + 2 * q;
+                    __nv_bfloat162 h = __floats2bfloat162_rn(fmaf(o0[k], g0, o1[k] * g1),
+                                                             fmaf(o0[k + 1], g0, o1[k + 1] * g1));
                     w4[q] = *reinterpret_cast<uint32_t*>(&h);
                 }
                 *reinterpret_cast<uint4*>(orow + c4 * 32 + e * 8) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
@@ -381,7 +384,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     int* sel_s = reinterpret_cast<int*>(sm + OFF_SEL);
     P.sel = sel_s;
     if (threadIdx.x == 0) {
-        ptx::mbar_init(&bars->q, NSOFT);
+        ptx::mbar_init(&bars->q, 1);
         for (int s = 0; s < NSTAGE; ++s) {
             ptx::mbar_init(&bars->kfull[s], 1);
             ptx::mbar_init(&bars->kempty[s], 1);
@@ -391,7 +394,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int b = 0; b < 2; ++b) ptx::mbar_init(&bars->sfull[b], 1);
         ptx::mbar_init(&bars->pfull, NSOFT);
         ptx::mbar_init(&bars->pvdone, 1);
-        for (int qd = 0; qd < 4; ++qd) ptx::mbar_init(&bars->mx[qd], 64);
         bars->abort = 0;
         ptx::mbar_fence_init();
     }
@@ -422,7 +424,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         } else if (warp == 1) {
             if (lane == 0) mma_issuer(P, D, sm, bars, tmem);
         } else {
-            softmax_role(P, D, bars, reinterpret_cast<float*>(sm + OFF_LSUM), reinterpret_cast<float*>(sm + OFF_MXS),
+            softmax_role(P, D, bars, reinterpret_cast<float*>(sm + OFF_LSUM), reinterpret_cast<float*>(sm + OFF_MREF),
                          tmem, c0, n, out, warp, lane);
         }
     }
