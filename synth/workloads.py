@@ -102,6 +102,11 @@ SMALL = {
                              needle=True),
     "small_decode": Workload("small_decode", 8, 2, 128, 16, 512, 64, 4, 4, 1, 2048, 1e4, "bf16", seed=20,
                              decode_steps=200, build_chunk=512),
+    # eight q heads per KV head: 16 queries per packed 128-row tile (smallest tensor-core tile)
+    "small_g8": Workload("small_g8", 16, 2, 128, 32, 512, 128, 4, 4, 256, 2600, 1e6, "bf16", seed=21,
+                         k_bias_var=4.0),
+    "small_decode_g8": Workload("small_decode_g8", 16, 2, 128, 16, 512, 64, 4, 4, 1, 2048, 1e6, "bf16", seed=22,
+                                decode_steps=64, build_chunk=512),
 }
 
 ALL = {**WORKLOADS, **SMALL}

@@ -18,7 +18,7 @@ from tests._source import Source
 pytestmark = pytest.mark.gpu
 
 SMALL_PREFILL = ["small_gqa", "small_g4", "small_d64", "small_u256", "small_nosink", "small_streaming",
-                 "small_allunits", "small_f32", "small_needle"]
+                 "small_allunits", "small_f32", "small_needle", "small_g8"]
 
 
 def _stream_oracle(w):
@@ -33,8 +33,8 @@ def _stream_oracle(w):
 @pytest.mark.parametrize("score_mode", ["reps", "repsum"])
 def test_prefill_stream_matches_oracle(cuda_ok, name, score_mode):
     w = synth.SMALL[name]
-    if score_mode == "repsum" and name not in ("small_gqa", "small_g4", "small_f32"):
-        pytest.skip("repsum covered on three shapes")
+    if score_mode == "repsum" and name not in ("small_gqa", "small_g4", "small_f32", "small_g8"):
+        pytest.skip("repsum covered on four shapes")
     glayer, res = run_prefill(w, score_mode=score_mode)
     olayer, q, k, v = _stream_oracle(w)
     tol = TOL[w.dtype]
@@ -97,9 +97,10 @@ def test_chunked_equals_stateless_on_gpu_reps(cuda_ok):
     glayer.close()
 
 
-def test_decode_matches_oracle(cuda_ok):
+@pytest.mark.parametrize("name", ["small_decode", "small_decode_g8"])
+def test_decode_matches_oracle(cuda_ok, name):
     import torch
-    w = synth.SMALL["small_decode"]
+    w = synth.SMALL[name]
     glayer = make_layer(w)
     src = Source(w)
     olayer = O.OracleLayer(w.as_config(), rep_method="linear")
