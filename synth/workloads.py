@@ -105,6 +105,9 @@ SMALL = {
     # eight q heads per KV head: 16 queries per packed 128-row tile (smallest tensor-core tile)
     "small_g8": Workload("small_g8", 16, 2, 128, 32, 512, 128, 4, 4, 256, 2600, 1e6, "bf16", seed=21,
                          k_bias_var=4.0),
+    # two q heads per KV head: 64 queries per packed tile; chunks of 2.5 tiles
+    "small_g2": Workload("small_g2", 4, 2, 128, 64, 256, 64, 4, 3, 160, 2000, 1e4, "bf16", seed=23,
+                         k_bias_var=4.0),
     "small_decode_g8": Workload("small_decode_g8", 16, 2, 128, 16, 512, 64, 4, 4, 1, 2048, 1e6, "bf16", seed=22,
                                 decode_steps=64, build_chunk=512),
 }

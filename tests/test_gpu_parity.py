@@ -18,7 +18,8 @@ from tests._source import Source
 pytestmark = pytest.mark.gpu
 
 SMALL_PREFILL = ["small_gqa", "small_g4", "small_d64", "small_u256", "small_nosink", "small_streaming",
-                 "small_allunits", "small_f32", "small_needle", "small_g8"]
+                 "small_allunits", "small_f32", "small_needle", "small_g8",
+                 "small_g2"]
 
 
 def _stream_oracle(w):
