@@ -642,7 +642,6 @@ infllm_status infllm_prefill(infllm_ctx* c, const void* q, const void* k, const 
     c->chain = false;
     infllm_status s = check_device_error(c);
     if (s != INFLLM_OK) return s;
-    if (c->pending && c->pending_n > 0) return fail(c, INFLLM_ESTATE, "prefill: an appended chunk waits for attend");
     if (n < 0) return fail(c, INFLLM_EINVAL, "prefill: n = %lld < 0", (long long)n);
     if (chunk < 1 || chunk > c->cfg.max_chunk)
         return fail(c, INFLLM_EINVAL, "prefill: chunk = %d not in [1, max_chunk = %d]", chunk, c->cfg.max_chunk);
@@ -651,6 +650,7 @@ infllm_status infllm_prefill(infllm_ctx* c, const void* q, const void* k, const 
                     (long long)n, (long long)c->cfg.max_tokens);
     if (n == 0) return INFLLM_OK;
     if (!q || !k || !v || !out) return fail(c, INFLLM_EINVAL, "prefill: null pointer");
+    c->pending = false;  // a chunk appended and not attended stays in the context without its outputs
     return c->cfg.dtype == INFLLM_BF16
                ? prefill_impl<__nv_bfloat16>(c, (const char*)q, (const char*)k, (const char*)v, n, chunk, (char*)out)
                : prefill_impl<float>(c, (const char*)q, (const char*)k, (const char*)v, n, chunk, (char*)out);

@@ -8,6 +8,7 @@
 // static device array of fixed size, which every GPU that loads the library holds until the
 // process exits.  The InfLLM pages have no counterpart to this entry point; it computes the
 // same unit scores and selection as the lookup step of infllm_decode_step.
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <math.h>
 
@@ -36,6 +37,33 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[sizeof(NoallocS
 
 std::mutex g_mu;
 void* g_addr[NA_MAX_DEVICES] = {nullptr};
+unsigned long long g_ctx[NA_MAX_DEVICES] = {0};  // id of the context g_addr[dev] was resolved in
+
+// Unique id (for the process lifetime) of the calling thread's current CUDA context, 0 if none.  A
+// device reset replaces the primary context and reloads the module, which moves the scratch array;
+// a new id tells the entry point to look its address up again.
+unsigned long long current_context_id() {
+    typedef CUresult (*GetCurrentFn)(CUcontext*);
+    typedef CUresult (*GetIdFn)(CUcontext, unsigned long long*);
+    static GetCurrentFn get_current = nullptr;
+    static GetIdFn get_id = nullptr;
+    if (!get_current || !get_id) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = (GetCurrentFn)p;
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = (GetIdFn)p;
+        if (!get_current || !get_id) return 0;
+    }
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
 
 template <typename T>
 __global__ void __launch_bounds__(256) k_select_noalloc(NoallocScratch* scr, const T* __restrict__ rep_keys,
@@ -64,17 +92,42 @@ __global__ void __launch_bounds__(256) k_select_noalloc(NoallocScratch* scr, con
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int u0 = split * NA_UNITS_PER_CTA;
     const int u1 = min(n_units, u0 + NA_UNITS_PER_CTA);
+    // A unit's row (r * d elements) is read by the whole warp in 16-byte pieces, consecutive lanes
+    // on consecutive pieces; the warp takes four units at a time, all their loads issued first.
+    constexpr int V = 16 / sizeof(T);
+    const int cpr = r * d / V;  // 16-byte pieces per row (a multiple of 4)
     uint64_t list = 0;
     for (int jb = u0 + warp * 32; jb < u1; jb += 8 * 32) {
-        const int j = jb + lane;
         uint64_t cand = 0;
-        if (j < u1) {
-            const T* p = rep_keys + ((int64_t)hk * n_units + j) * r * d;
-            float acc = 0.f;
-            for (int e = 0; e < r * d; ++e) acc += to_f(p[e]) * qb[e % d];
-            const float s = acc * inv_sqrt_d;
-            if (scores) scores[(int64_t)hk * n_units + j] = s;
-            cand = make_key(s, (uint32_t)j);
+        for (int jj = 0; jj < 32 && jb + jj < u1; jj += 4) {  // warp-uniform
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int c0 = 0; c0 < cpr; c0 += 32) {
+                const int c = c0 + lane;
+                uint4 raw[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int j = jb + jj + u;
+                    raw[u] = (c < cpr && j < u1)
+                                 ? __ldg(reinterpret_cast<const uint4*>(rep_keys + ((int64_t)hk * n_units + j) * r * d) + c)
+                                 : make_uint4(0, 0, 0, 0);
+                }
+                const int i0 = (c * V) % d;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const T* e = reinterpret_cast<const T*>(&raw[u]);
+#pragma unroll
+                    for (int v = 0; v < V; ++v) acc[u] += c < cpr ? to_f(e[v]) * qb[i0 + v] : 0.f;
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float s = warp_sum(acc[u]) * inv_sqrt_d;
+                const int j = jb + jj + u;
+                if (j < u1 && lane == jj + u) {
+                    if (scores) scores[(int64_t)hk * n_units + j] = s;
+                    cand = make_key(s, (uint32_t)j);
+                }
+            }
         }
         list = warp_topk_insert(list, cand);
     }
@@ -117,6 +170,7 @@ extern "C" infllm_status infllm_select_units_noalloc(const void* rep_keys, const
     if (top_k < 1 || top_k > 32) return INFLLM_EINVAL;
     if (dtype != INFLLM_F32 && dtype != INFLLM_BF16) return INFLLM_EINVAL;
     if (n_units > 0 && !rep_keys) return INFLLM_EINVAL;
+    if ((uintptr_t)rep_keys % 16 != 0) return INFLLM_EINVAL;  // read in 16-byte pieces
     // beyond the fixed scratch area
     if (n_kv_heads > NA_MAX_HKV || n_units > NA_MAX_UNITS) return INFLLM_ECAPACITY;
     cudaStream_t st = (cudaStream_t)cuda_stream;
@@ -128,11 +182,14 @@ extern "C" infllm_status infllm_select_units_noalloc(const void* rep_keys, const
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= NA_MAX_DEVICES) return INFLLM_ECUDA;
     void* base = nullptr;
     {
+        // the current device's runtime context exists from here on (cudaGetSymbolAddress creates it)
         std::lock_guard<std::mutex> lk(g_mu);
-        if (!g_addr[dev]) {  // once per device, with that device current
+        unsigned long long ctx = current_context_id();
+        if (!g_addr[dev] || ctx == 0 || ctx != g_ctx[dev]) {  // once per device and context, that device current
             void* p = nullptr;
             if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return INFLLM_ECUDA;
             g_addr[dev] = p;
+            g_ctx[dev] = ctx != 0 ? ctx : current_context_id();
         }
         base = g_addr[dev];
     }

@@ -99,47 +99,73 @@ typedef struct {
 
 typedef struct infllm_ctx infllm_ctx; /* opaque */
 
-/* Create a context: validates cfg, allocates every pool for max_tokens / max_chunk on
- * the current CUDA device, and records `cuda_stream` (a cudaStream_t; NULL = legacy
- * default stream) for all later work.  On failure *out is NULL. */
+/* Create a context: validates cfg, allocates every pool for max_tokens / max_chunk on the
+ * current CUDA device (the K/V stores, the representative pool, the packed-query and lookup
+ * buffers), and records `cuda_stream` (a cudaStream_t; NULL = legacy default stream) for all
+ * later work.  The pools hold the three parts of the context that "InfLLM Guide: Training-Free
+ * Long-Context Memory Units", "Core Innovation 1: Structured Context Partitioning", names:
+ * initial (sink) tokens, memory units of unit_size tokens, and the local window.
+ * Errors: EINVAL (cfg out of range, message on stderr), ECUDA (allocation failed).  On failure
+ * *out is NULL and nothing stays allocated.  The caller owns the context until infllm_destroy. */
 infllm_status infllm_create(const infllm_config* cfg, void* cuda_stream, infllm_ctx** out);
 
-/* Free everything.  Waits for the context's pending work.  NULL is accepted. */
+/* Free everything the context owns.  Waits for the context's pending work.  NULL is accepted. */
 infllm_status infllm_destroy(infllm_ctx* ctx);
 
 /* Start a new token stream in the same context (keeps allocations). */
 infllm_status infllm_reset(infllm_ctx* ctx);
 
-/* Append tokens [t, t+n) where t = tokens so far.  Before storing them, every unit that
- * becomes eligible at t (its last token at least `window` tokens before t) gets its
- * representatives, scored against the `window` queries that follow it.  q [n][Hq][d] is
- * used for those later scores; k, v [n][Hkv][d] are stored.  n == 0 is a no-op.
+/* Append tokens [t, t+n) where t = tokens so far.  First, every unit that becomes eligible at t
+ * (its last token at least `window` tokens before t) is turned into a memory unit: its n_reps
+ * representative tokens are the ones with the largest attention logit summed over the `window`
+ * queries that follow the unit and the q heads of the group ("InfLLM: Training-Free Long-Context
+ * Extrapolation for LLMs with an Efficient Context Memory", research-map summary, "Approach":
+ * units represented by representative tokens chosen by attention scores; ties to the lower
+ * token).  Then the chunk's k and v are stored and its queries are kept (as block sums) for
+ * later representative scores.
+ *   q [n][Hq][d] device, k, v [n][Hkv][d] device, all in the context dtype; read during the call's
+ *   kernels only (the caller may reuse them once the stream has passed this call).
+ * n == 0 is a no-op.  A chunk that is appended and not attended before the next append, decode
+ * step or prefill stays in the context without outputs of its own: that is how a memory is built
+ * from a prompt whose outputs are not needed.
  * Errors: EINVAL (null pointer with n > 0, n > max_chunk, n < 0), ECAPACITY (tokens + n >
- * max_tokens). */
+ * max_tokens), EDEVICE (an earlier kernel's check failed). */
 infllm_status infllm_append_chunk(infllm_ctx* ctx, const void* q, const void* k, const void* v,
                                   int32_t n);
 
-/* Attention output of the chunk just appended (same n): score every eligible unit, keep
- * the top min(top_k, n_mem) per kv head (ties to the lower unit index), then
- * out[n][Hq][d] = softmax over sinks (n < S, causal) U selected units U window [B, t].
- * Errors: ESTATE (no matching append), EINVAL. */
+/* Attention output of the chunk just appended (same n), the chunk-wise lookup of the OpenReview
+ * rebuttal (paperhub.cn), Q2 "Comparison to Well-trained Long LLM".  Unit lookup: every eligible
+ * unit's score is the scaled logit q . r / sqrt(d) summed over the chunk's queries, the group's q
+ * heads and the unit's representatives, with every memory token at relative distance `window`
+ * ("InfLLM Guide...", "Core Innovation 2", item 2 "Query-Aware Top-K Scoring and Loading"); the top
+ * min(top_k, n_mem) per kv head are kept, ties to the lower unit index.  Then one exact softmax
+ * over sinks (n < S, causal) U selected units U window [B, t] (same page, item 3 "Exact Attention
+ * Evaluation").
+ *   q [n][Hq][d] device (the chunk's queries again); out [n][Hq][d] device, written by the call's
+ *   kernels.
+ * Errors: ESTATE (no matching append), EINVAL (null pointer), EDEVICE. */
 infllm_status infllm_attend_chunk(infllm_ctx* ctx, const void* q, int32_t n, void* out);
 
-/* Whole-prompt prefill: n tokens (q [n][Hq][d], k, v [n][Hkv][d], out [n][Hq][d]) in chunks
+/* Whole-prompt prefill: n tokens (q [n][Hq][d], k, v [n][Hkv][d], out [n][Hq][d], device) in chunks
  * of `chunk` tokens (the last one ragged), each chunk appended and then attended exactly as
  * infllm_append_chunk + infllm_attend_chunk would, in one call.  Chunk-wise pre-filling with
- * per-chunk unit lookup follows "InfLLM: Training-Free Long-Context Extrapolation for LLMs
- * with an Efficient Context Memory" (OpenReview rebuttal, Q2; the guide's "Memory Efficiency"
- * section); this entry point adds no arithmetic of its own.  Because every input is in place
- * when the call starts, the kernels of chunk c+1 that store its keys and pack its queries are
- * chained to (and overlap) chunk c's attention.  Results are identical to the per-chunk calls.
- * Errors: EINVAL (null pointer with n > 0, chunk not in [1, max_chunk], n < 0), ESTATE (an
- * appended chunk still waits for its attend), ECAPACITY (tokens + n > max_tokens). */
+ * per-chunk unit lookup follows the OpenReview rebuttal (paperhub.cn), Q2 "Comparison to
+ * Well-trained Long LLM", and "InfLLM Guide...", "Memory Efficiency"; this entry point adds no
+ * arithmetic of its own.  Because every input is in place when the call starts, the kernels of
+ * chunk c+1 that store its keys and pack its queries are chained to (and overlap) chunk c's
+ * attention.  Results are identical, bit for bit, to the per-chunk calls.
+ * Errors: EINVAL (null pointer with n > 0, chunk not in [1, max_chunk], n < 0), ECAPACITY (tokens
+ * + n > max_tokens), EDEVICE. */
 infllm_status infllm_prefill(infllm_ctx* ctx, const void* q, const void* k, const void* v,
                              int64_t n, int32_t chunk, void* out);
 
-/* One decode step: append one token (q [1][Hq][d], k, v [1][Hkv][d]) and attend it
- * (split-KV kernel with a log-sum-exp merge).  out [1][Hq][d]. */
+/* One decode step: append one token (q [1][Hq][d], k, v [1][Hkv][d], device) and attend it; out
+ * [1][Hq][d] device.  Per generated token: lookup over every eligible unit and exact attention
+ * over sinks U top-k units U window, as for a one-token chunk ("InfLLM Guide...", "Core Innovation
+ * 2", items 2 and 3; lookup at every decoding step: "InfLLM: Training-Free Long-Context
+ * Extrapolation...", research-map summary, "Approach").  The attention is split over key tiles
+ * whose partial softmaxes are merged by log-sum-exp (exact).
+ * Errors: EINVAL (null pointer), ECAPACITY (tokens + 1 > max_tokens), EDEVICE. */
 infllm_status infllm_decode_step(infllm_ctx* ctx, const void* q, const void* k, const void* v,
                                  void* out);
 
@@ -211,6 +237,7 @@ const char* infllm_last_error(infllm_ctx* ctx);
  *
  *   rep_keys  device [n_kv_heads][n_units][n_reps][head_dim], `dtype`: raw keys of every unit's
  *             representative tokens
+ *             (16-byte aligned)
  *   q         device [n_q_heads][head_dim], `dtype`: the query token, before RoPE
  *   sel       device out [n_kv_heads][top_k] int32: ascending ids of the top min(top_k, n_units)
  *             units of each kv head (ties to the lower id), padded with -1
@@ -220,8 +247,10 @@ const char* infllm_last_error(infllm_ctx* ctx);
  * INFLLM_ECAPACITY before anything is enqueued.  Other bad arguments (top_k outside [1, 32],
  * head_dim not 64/128, ...) return INFLLM_EINVAL.  Work is enqueued on `cuda_stream`, which must
  * belong to the current device.
- * The first call on a device looks up the device address of the scratch array (once per device,
- * with that device current); make that first call before any stream capture.  Every call shares
+ * The first call on a device looks up the device address of the scratch array (once per device
+ * and CUDA context, with that device current); make that first call before any stream capture.  A
+ * device reset (cudaDeviceReset) gives the device a new context, and the next call looks the
+ * address up again.  Every call shares
  * the scratch area and keeps the last call's contents (the call clears what must start at zero):
  * calls whose work overlaps on the GPU -- on different streams or from different host threads --
  * race and can return wrong results, so serialise them. */

@@ -1,6 +1,6 @@
 """The tcgen05 prefill attention kernel's barrier protocol, modelled and explored on the CPU.
 
-compute-sanitizer is not available for this kernel, so its synchronisation is checked on a model
+No compute-sanitizer run of this kernel exists, so its synchronisation is checked on a model
 instead: the roles of `k_attn_tc` (attend_tc.cu) as coroutines that a seeded scheduler
 interleaves at random, with exact mbarrier parity semantics.
 - TMA producer: two query tiles, then K and V tiles through 2-stage rings.

@@ -1,9 +1,17 @@
-"""Parity at the full sizes of the four large workloads, in the launch configuration the bench
-times: the whole token stream runs through the C ABI on the GPU; the fp64 oracle recomputes
-sampled chunks (or decode steps) statelessly from the full prefix with its OWN representatives
-and selection.  Indices must be bit-exact wherever the oracle's fp64 score gap exceeds 1e-3
-relative; where a near-tie makes several choices correct, the GPU's choice must lie inside the
-band and the outputs are checked on the GPU's selection.  Outputs within 2e-2 max-abs (bf16).
+"""Parity at the full sizes of the four large workloads.
+
+Prefill workloads run twice through the C ABI: once through infllm_prefill, the whole prompt in
+one call -- the entry point and launch configuration the benchmark times (one-chunk lookahead,
+three query slots, two selection buffers) -- and once through append_chunk + attend_chunk per
+chunk.  The two outputs must be equal bit for bit over the whole stream, as must the final
+selection, unit scores and representatives.  The per-chunk run records the selection and unit
+scores of sampled chunks, and the fp64 oracle recomputes those chunks statelessly from the full
+prefix with its OWN representatives and selection.  Decode runs through infllm_decode_step, one
+call per token, as the benchmark times it.
+
+Indices must be bit-exact wherever the oracle's fp64 score gap exceeds 1e-3 relative; where a
+near-tie makes several choices correct, the GPU's choice must be a valid one inside the band
+and the outputs are checked on the GPU's selection.  Outputs within 2e-2 max-abs (bf16).
 """
 from __future__ import annotations
 
@@ -12,7 +20,7 @@ import pytest
 
 import synth
 from oracle import infllm_oracle as O
-from tests._parity import TOL, compare_reps, compare_selection, make_layer, run_prefill, to_np64, to_torch
+from tests._parity import TOL, compare_reps, compare_selection, make_layer, to_np64, to_torch
 from tests._source import Source
 
 pytestmark = pytest.mark.gpu
@@ -41,13 +49,46 @@ def _check_chunk(w, src, cfg, oreps, rep_keys, c0, n, g_out, g_sel, g_scores, g_
     return info, n_dec
 
 
+def _prefill_both_paths(w, sample):
+    """The whole stream through infllm_prefill and through per-chunk calls (bit-equal outputs and
+    final state).  Returns (per-chunk layer, prefill output as float64 numpy, {chunk: record})."""
+    import torch
+    q, k, v = synth.gen_chunk(w, 0, w.n_tokens)
+    qd, kd, vd = to_torch(q), to_torch(k), to_torch(v)
+    del q, k, v
+    glayer = make_layer(w)
+    outs = torch.empty_like(qd)
+    rec = {}
+    for ci, (c0, n) in enumerate(synth.chunk_bounds(w)):
+        glayer.append_chunk(qd[c0:c0 + n], kd[c0:c0 + n], vd[c0:c0 + n])
+        glayer.attend_chunk(qd[c0:c0 + n], out=outs[c0:c0 + n])
+        if ci in sample:
+            torch.cuda.synchronize()
+            rec[ci] = dict(c0=c0, n=n, sel=glayer.selection().copy(), scores=glayer.unit_scores().copy())
+    player = make_layer(w)
+    outp = player.prefill(qd, kd, vd, w.chunk)
+    torch.cuda.synchronize()
+    assert torch.equal(outp, outs), "infllm_prefill differs from the per-chunk calls"
+    assert player.selection().tolist() == glayer.selection().tolist()
+    assert np.array_equal(player.unit_scores(), glayer.unit_scores())
+    nu = glayer.stats()["units_with_reps"]
+    assert player.stats()["units_with_reps"] == nu
+    assert np.array_equal(player.reps(0, nu), glayer.reps(0, nu))
+    player.close()
+    for ci, r in rec.items():
+        r["out"] = to_np64(outp[r["c0"]:r["c0"] + r["n"]])
+    del outs, outp, qd, kd, vd
+    torch.cuda.empty_cache()
+    return glayer, rec
+
+
 @pytest.mark.parametrize("name", ["mistral_128k", "llama3_128k"])
 def test_prefill_stream_fullsize(cuda_ok, name):
     w = synth.WORKLOADS[name]
     cfg, src = w.as_config(), Source(w)
     chunks = synth.chunk_bounds(w)
     sample = {64, 160, len(chunks) - 1}
-    glayer, res = run_prefill(w, record=sample)
+    glayer, res = _prefill_both_paths(w, sample)
     last_c0 = chunks[-1][0]
     nu = O.n_mem(last_c0, w.n_sink, w.window, w.unit_size)
     g_reps = glayer.reps(0, nu)
@@ -67,7 +108,7 @@ def test_needle_256k_fullsize(cuda_ok):
     chunks = synth.chunk_bounds(w)
     last = len(chunks) - 1
     j_star = synth.needle_info(w)[0]
-    glayer, res = run_prefill(w, record={last})
+    glayer, res = _prefill_both_paths(w, {last})
     g = res[last]
     nu = O.n_mem(g["c0"], w.n_sink, w.window, w.unit_size)
     g_reps = glayer.reps(0, nu)

@@ -30,12 +30,14 @@ def _stream_oracle(w):
     return layer, q, k, v
 
 
-@pytest.mark.parametrize("name", SMALL_PREFILL)
-@pytest.mark.parametrize("score_mode", ["reps", "repsum"])
+# every shape with the representative keys; the fp32 sum of them (REPSUM) on four shapes
+PREFILL_CASES = [(n, "reps") for n in SMALL_PREFILL] + [(n, "repsum") for n in
+                                                       ("small_gqa", "small_g4", "small_f32", "small_g8")]
+
+
+@pytest.mark.parametrize("name,score_mode", PREFILL_CASES)
 def test_prefill_stream_matches_oracle(cuda_ok, name, score_mode):
     w = synth.SMALL[name]
-    if score_mode == "repsum" and name not in ("small_gqa", "small_g4", "small_f32", "small_g8"):
-        pytest.skip("repsum covered on four shapes")
     glayer, res = run_prefill(w, score_mode=score_mode)
     olayer, q, k, v = _stream_oracle(w)
     tol = TOL[w.dtype]

@@ -126,13 +126,22 @@ def test_prefill_errors(cuda_ok):
         layer.prefill(q, k, v, 200)
     assert e.value.status == 2
     assert layer.stats()["tokens"] == 0
+    # a chunk appended without its attend joins the context with no outputs of its own (how a memory
+    # is built from a prompt whose outputs are not needed); a later attend no longer refers to it
     layer.append_chunk(q[:100].contiguous(), k[:100].contiguous(), v[:100].contiguous())
-    with pytest.raises(InfLLMError) as e:  # an appended chunk waits for its attend
-        layer.prefill(q[100:200].contiguous(), k[100:200].contiguous(), v[100:200].contiguous(), 100)
-    assert e.value.status == 3
-    layer.attend_chunk(q[:100].contiguous())
     out = layer.prefill(q[100:600].contiguous(), k[100:600].contiguous(), v[100:600].contiguous(), 200)
     torch.cuda.synchronize()
     assert out.shape == (500, w.n_q_heads, w.head_dim)
     assert layer.stats()["tokens"] == 600
+    with pytest.raises(InfLLMError) as e:
+        layer.attend_chunk(q[:100].contiguous())
+    assert e.value.status == 3
+    # the same context as appending the first 100 tokens and prefilling the rest from scratch
+    ref = make_layer(w, max_tokens=600, max_chunk=200)
+    ref.append_chunk(q[:100].contiguous(), k[:100].contiguous(), v[:100].contiguous())
+    ref.attend_chunk(q[:100].contiguous())
+    ref_out = ref.prefill(q[100:600].contiguous(), k[100:600].contiguous(), v[100:600].contiguous(), 200)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref_out)
+    ref.close()
     layer.close()
