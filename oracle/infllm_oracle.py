@@ -24,6 +24,11 @@ Sources (the method as described on the InfLLM pages):
        encoding (chunked prefill) and decoding.
   [R1] OpenReview rebuttal (paperhub.cn), Q2 "Comparison to Well-trained Long
        LLM" -- lookup during pre-filling is done per block (chunk).
+  [S3] same summary page as [S1], "Measured effects" row "Use selected
+       representative tokens instead of mean key-vector representations" and
+       "Surprising findings" -- the mean of a unit's keys as the alternative unit
+       representation; [G2]'s listing ("Step-by-Step Implementation",
+       append_context_block) builds it by mean pooling the unit's keys.
 
 Readings taken where the pages leave a step open (each is listed with its
 reason in the design notes of the repository):
@@ -41,6 +46,10 @@ reason in the design notes of the repository):
     [B, t] with B = S + U * n_mem(c0); sinks are tokens n < S with n <= t.
   * Sinks and memory tokens sit at relative distance W (query rotated by
     R(W), key raw); window pairs use true relative distance t - n.
+  * The mean-of-keys representation of a unit is the mean of its U raw keys,
+    stored in the layer's dtype (rounded to nearest, ties to even), like the
+    listing's mean of a key block in the model's dtype; a unit's score is then
+    the same scaled logit with that one vector as the unit's only key.
 
 Parity pins for every function live in tests/test_oracle_pins.py.
 """
@@ -144,6 +153,41 @@ def select_reps(rho: np.ndarray, n_reps: int) -> list[int]:
 
 
 # --------------------------------------------------------------------------------------------
+# mean-of-keys unit representation  [S3]
+
+
+def round_to_dtype(x, dtype: str) -> np.ndarray:
+    """Round float64 values to the nearest value of `dtype` ("f64": unchanged; "f32": float32;
+    "bf16": 8 significant bits), ties to even, returned as float64.  Normal numbers only for bf16."""
+    x = np.asarray(x, dtype=np.float64)
+    if dtype == "f64":
+        return x.copy()
+    if dtype == "f32":
+        return x.astype(np.float32).astype(np.float64)
+    assert dtype == "bf16", dtype
+    m, e = np.frexp(x)  # x = m * 2^e, 0.5 <= |m| < 1: 8 significant bits keep m * 2^8 integral
+    return np.ldexp(np.rint(m * 256.0) / 256.0, e)
+
+
+def unit_mean_key(k_unit: np.ndarray, dtype: str) -> np.ndarray:
+    """The unit's representation as the mean of its raw keys: k_unit [U, d] -> [d] in `dtype`."""
+    return round_to_dtype(k_unit.sum(axis=0) / k_unit.shape[0], dtype)
+
+
+def mean_key_table(ksrc: Callable, n_units: int, cfg: dict) -> np.ndarray:
+    """Mean key of every unit < n_units: [Hkv, n_units, d] (keys fetched 256 units at a time)."""
+    S, U, Hkv, d = cfg["n_sink"], cfg["unit_size"], cfg["n_kv_heads"], cfg["head_dim"]
+    out = np.zeros((Hkv, n_units, d))
+    for j0 in range(0, n_units, 256):
+        nb = min(256, n_units - j0)
+        kb = ksrc(S + j0 * U, nb * U)
+        for j in range(j0, j0 + nb):
+            for hk in range(Hkv):
+                out[hk, j] = unit_mean_key(kb[(j - j0) * U:(j - j0 + 1) * U, hk], cfg["dtype"])
+    return out
+
+
+# --------------------------------------------------------------------------------------------
 # unit lookup  [G2] item 2, [R1]
 
 
@@ -212,6 +256,8 @@ class OracleLayer:
     Keeps every token's q/k/v in float64 (small streams only).  Representatives of a unit are
     computed when the unit becomes eligible, from the W queries that follow it.
     `rep_method` "plain" uses the explicit double loop, "linear" the summed-query form.
+    cfg["unit_repr"] = "meankey" scores units by the mean of their keys instead of their
+    representatives (default "reps").
     """
 
     def __init__(self, cfg: dict, rep_method: str = "plain"):
@@ -274,7 +320,11 @@ class OracleLayer:
         for hk in range(c["n_kv_heads"]):
             qg = self.q[c0:c0 + n, hk * G:(hk + 1) * G]
             if nm > 0 and k > 0:
-                rk = np.stack([self.k[[S + j * U + m for m in self.reps[j][hk]], hk] for j in range(nm)])
+                if c.get("unit_repr", "reps") == "meankey":
+                    rk = np.stack([unit_mean_key(self.k[S + j * U:S + (j + 1) * U, hk], c["dtype"])[None]
+                                   for j in range(nm)])
+                else:
+                    rk = np.stack([self.k[[S + j * U + m for m in self.reps[j][hk]], hk] for j in range(nm)])
                 sigma = unit_scores(qg, rk, W, c["rope_base"])
                 sel = topk_stable(sigma, min(k, nm))
             else:
@@ -372,7 +422,9 @@ def chunk_stateless(qsrc: Callable, ksrc: Callable, vsrc: Callable, c0: int, n: 
     """Recompute chunk [c0, c0+n) from scratch: reps of all eligible units, lookup, attention.
 
     `reps` may be passed in (e.g. the GPU's own representatives, to check the later steps on
-    them); `sel_override` likewise for the selection.  Returns (out [n, Hq, d], info dict).
+    them); `sel_override` likewise for the selection; `rep_keys` [Hkv, n_units, r, d] the units'
+    scoring vectors.  cfg["unit_repr"] = "meankey" scores by mean keys.  Returns (out [n, Hq, d],
+    info dict).
     """
     S, W, U, k, base = cfg["n_sink"], cfg["window"], cfg["unit_size"], cfg["top_k"], cfg["rope_base"]
     Hq, Hkv, d = cfg["n_q_heads"], cfg["n_kv_heads"], cfg["head_dim"]
@@ -402,7 +454,10 @@ def chunk_stateless(qsrc: Callable, ksrc: Callable, vsrc: Callable, c0: int, n: 
         return res
 
     if k > 0 and rep_keys is None:
-        rep_keys = rep_key_table(ksrc, reps, nm, cfg)  # raw keys of every unit's representatives
+        if cfg.get("unit_repr", "reps") == "meankey":
+            rep_keys = mean_key_table(ksrc, nm, cfg)[:, :, None, :]  # one vector per unit
+        else:
+            rep_keys = rep_key_table(ksrc, reps, nm, cfg)  # raw keys of every unit's representatives
     elif rep_keys is not None:
         rep_keys = rep_keys[:, :nm]
     for hk in range(Hkv):

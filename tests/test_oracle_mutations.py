@@ -37,6 +37,9 @@ MUTATIONS = {
     "key_batch_not_refetched": ("if kbatch is None or j >= kb0 + kbatch.shape[0] // U:", "if kbatch is None:"),
     "gqa_groups_transposed": ("qg = self.q[c0:c0 + n, hk * G:(hk + 1) * G]",
                               "qg = self.q[c0:c0 + n, hk::self.cfg['n_kv_heads']]"),
+    "mean_key_is_sum": ("return round_to_dtype(k_unit.sum(axis=0) / k_unit.shape[0], dtype)",
+                        "return round_to_dtype(k_unit.sum(axis=0), dtype)"),
+    "bf16_keeps_nine_bits": ("np.rint(m * 256.0) / 256.0", "np.rint(m * 512.0) / 512.0"),
 }
 
 

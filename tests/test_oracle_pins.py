@@ -421,3 +421,61 @@ def test_generator_is_counter_based_and_normal():
     np.testing.assert_array_equal(bf, synth.round_bf16(a))
     big = synth.normal(3, 2, 0, 4096, 8, 128, dtype="f32").ravel()
     assert abs(big.mean()) < 0.01 and abs(big.std() - 1) < 0.01
+
+
+# ------------------------------------------------------------------------------------------
+# 8. the mean-of-keys unit representation ("InfLLM: Training-Free Long-Context Extrapolation
+#    ...", research-map summary, "Measured effects", row "Use selected representative tokens
+#    instead of mean key-vector representations")
+
+
+def test_bf16_rounding_hand_values():
+    # bf16 keeps 8 significant bits: the grid next to 1 is 1 + k 2^-7; halfway cases go to even k
+    x = [1.0 + 2 ** -9, 1.0 + 3 * 2 ** -9, 1.0 + 3 * 2 ** -8, -(1.0 + 3 * 2 ** -8), 3.0, 0.1, 1.0 + 2 ** -8]
+    want = [1.0, 1.0 + 2 ** -7, 1.0 + 2 ** -6, -(1.0 + 2 ** -6), 3.0, 0.10009765625, 1.0]
+    assert O.round_to_dtype(x, "bf16").tolist() == want
+    assert O.round_to_dtype([0.1], "f32")[0] == float(np.float32(0.1))
+
+
+def test_mean_key_of_constant_and_hand_units():
+    c = O.round_to_dtype(rng.standard_normal(16), "bf16")
+    for U in (1, 3, 128):
+        np.testing.assert_array_equal(O.unit_mean_key(np.tile(c, (U, 1)), "bf16"), c)
+    np.testing.assert_array_equal(O.unit_mean_key(np.array([[1.0, 2.0], [3.0, 4.0]]), "f64"), [2.0, 3.0])
+    # (0.5 + 1.0 + 2.0) / 3 = 7/6 -> bf16 1.1640625 (7/6 = 1.00101010..b: 8 bits 1.0010101 then 0 1 0...)
+    assert O.unit_mean_key(np.array([[0.5], [1.0], [2.0]]), "bf16")[0] == 1.1640625
+
+
+def test_mean_key_score_is_the_all_token_score_over_u():
+    """Scored with its mean key (unrounded), a unit's score is the score it gets with all of its U tokens
+    as representatives, divided by U -- the sum over representatives is linear in the keys."""
+    C, G, U, n_units, d, W = 5, 4, 16, 6, 32, 300
+    q = rng.standard_normal((C, G, d))
+    keys = rng.standard_normal((n_units, U, d)) + 2.0
+    all_tok = O.unit_scores(q, keys, W, 1e4)
+    means = np.stack([O.unit_mean_key(keys[j], "f64") for j in range(n_units)])[:, None, :]
+    np.testing.assert_allclose(O.unit_scores(q, means, W, 1e4), all_tok / U, rtol=1e-12, atol=1e-12)
+
+
+def test_mean_key_layer_streaming_equals_stateless():
+    w = synth.SMALL["small_gqa"].replace(n_tokens=1300, window=256, chunk=170)
+    cfg = dict(w.as_config(), unit_repr="meankey")
+    src = Source(w)
+    T = w.n_tokens
+    q, k, v = src.q(0, T), src.k(0, T), src.v(0, T)
+    layer, outs, infos = run_stream(cfg, q, k, v, chunk=w.chunk, rep_method="linear")
+    table = O.mean_key_table(src.k, O.n_mem(T, w.n_sink, w.window, w.unit_size), cfg)
+    for hk in range(w.n_kv_heads):
+        for j in range(table.shape[1]):
+            u = k[w.n_sink + j * w.unit_size:w.n_sink + (j + 1) * w.unit_size, hk]
+            np.testing.assert_array_equal(table[hk, j], O.round_to_dtype(u.mean(axis=0), "bf16"))
+    n_cmp = 0
+    for o, inf in zip(outs, infos):
+        ref, rinfo = O.chunk_stateless(src.q, src.k, src.v, inf["c0"], inf["n"], cfg)
+        assert rinfo["sel"] == inf["sel"]
+        np.testing.assert_allclose(o, ref, rtol=0, atol=1e-12)
+        n_cmp += inf["n_mem"] > w.top_k
+    assert n_cmp >= 3
+    # the mean-key selection is a different one than the representatives' on this stream
+    rep_layer, _, rep_infos = run_stream(w.as_config(), q, k, v, chunk=w.chunk, rep_method="linear")
+    assert any(a["sel"] != b["sel"] for a, b in zip(infos, rep_infos))
