@@ -151,8 +151,8 @@ def decode_bytes(w, t, score_mode):
     B = S + U * nm
     keys = min(S, t + 1) + kk * U + (t - B + 1)
     elt = 2 if w.dtype == "bf16" else 4
-    score = nm * Hkv * (w.n_reps * d * elt if score_mode == "reps" else d * 4)
-    return score + keys * Hkv * d * elt * 2
+    per_unit = {"reps": w.n_reps * d * elt, "repsum": d * 4, "meankey": d * elt}[score_mode]
+    return nm * Hkv * per_unit + keys * Hkv * d * elt * 2
 
 
 # ------------------------------------------------------------------------------------------------
@@ -202,60 +202,121 @@ def attn_traffic():
     return traffic if attn_device_hash() == want else None
 
 
-def workload_config(w, world):
+def workload_config(w, world, big=True, in_bytes=None):
     """The `config` object of the JSON line (the same for both arms)."""
+    if in_bytes is None:
+        elt = 2 if w.dtype == "bf16" else 4
+        in_bytes = w.n_tokens * (w.n_q_heads + 2 * w.n_kv_heads) * w.head_dim * elt
+    l2 = (f"inputs larger than L2 ({in_bytes / 1e9:.2f} GB of Q/K/V per step)" if big else
+          f"inputs ({in_bytes / 1e6:.1f} MB) smaller than L2: L2 flushed (256 MB read) before every step, "
+          "steps timed one by one, median")
     return {"workload": f"{w.name}: {w.n_q_heads}q/{w.n_kv_heads}kv heads, d={w.head_dim}, "
                         f"{w.n_tokens} tokens in {w.chunk}-token chunks, W={w.window}, S={w.n_sink}, "
-                        f"U={w.unit_size}, r={w.n_reps}, k={w.top_k}, base={w.rope_base:g}",
-            "global_batch": 1 * world, "seq_len": w.n_tokens, "parallelism": f"replicas x{world}",
-            "l2": "inputs larger than L2 (1.6 GB of Q/K/V per step)"}
+                        f"U={w.unit_size}, r={w.n_reps}, k={w.top_k}, base={w.rope_base:g}, {w.dtype}",
+            "global_batch": 1 * world, "seq_len": w.n_tokens, "parallelism": f"replicas x{world}", "l2": l2}
 
 
-def run_ours(args, rank, world):
-    import torch
+L2_BYTES = 126 * 1024 * 1024
+
+
+def attn_roofline(w, st, flops, P, clk):
+    """Roofline object of the chunk-attention kernel from its event-timed launches.  The tcgen05 kernel
+    is a bf16 contraction: its peak is the measured bf16 GEMM rate, burst when the clocks sampled over
+    the attention-only pass sat at their maximum with no power cap (the kernel then runs as a short
+    burst), else sustained; both fractions are reported.  The fp32 CUDA-core kernel is bound by FP32
+    FMA issue: 148 SMs x 128 lanes x 2 flops x the maximum SM clock."""
+    att_ms, n_att = st["ms_attend"], st["n_attend"]
+    achieved = flops / (att_ms / 1e3) / 1e12 if att_ms > 0 else None
+    if st["attend_path"] == 1:
+        c = clk.summary()
+        capped = "sw_power_cap" in c["reasons"]
+        at_max = c["sm_mhz"] is not None and c["sm_max_mhz"] and c["sm_mhz"] >= 0.95 * c["sm_max_mhz"]
+        burst = bool(at_max and not capped)
+        peak = P["bf16"] if burst else P["bf16_sust"]
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": (achieved / peak) if achieved else None,
+                "frac_of_burst": (achieved / P["bf16"]) if achieved else None,
+                "frac_of_sustained": (achieved / P["bf16_sust"]) if achieved else None,
+                "traffic": attn_traffic() if w.name == "mistral_128k" else None,
+                "kernel": "attention (tcgen05)",
+                "peak_source": f"{P['src']} bf16 {'burst' if burst else 'sustained'} (clocks over the attention pass: "
+                               f"median {c['sm_mhz']} of {c['sm_max_mhz']} MHz, reasons {c['reasons']})",
+                "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of one steady-chunk launch "
+                                  "(profiles/k_attn_tc_mistral_128k.md); null if the kernel changed since, or for "
+                                  "another workload"}
+    else:
+        peak = 148 * 128 * 2 * P["sm_max"] * 1e6 / 1e12
+        roof = {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": (achieved / peak) if achieved else None, "traffic": None,
+                "kernel": "attention (CUDA cores, fp32)", "peak_source": "148 SMs x 128 FP32 lanes x 2 x max SM clock"}
+    roof["avg_launch_ms"] = att_ms / n_att if n_att else None
+    roof["launches"] = n_att
+    roof["timing"] = "CUDA events around each attention launch, over a repeat of the timed steps"
+    return roof
+
+
+def time_prefill(args, w, torch, device, stream, local, world, P, plan=None):
+    """The whole-prompt prefill of workload w (reset + infllm_prefill per step).  Inputs larger than L2 are
+    timed as K back-to-back steps; smaller ones step by step, each after an L2 flush (median reported).
+    With a KV-head shard plan, this rank runs its heads' slice of the layer (strong scaling: all ranks
+    together process the prompt once; the output gather is the model's tensor-parallel step, outside).
+    Returns (fields of the JSON line, layer, host inputs)."""
     from block_memory_sparse_b200 import InfLLMLayer
-
-    _, _, local = dist_env()
-    torch.cuda.set_device(local)
-    device = torch.device("cuda", local)
-    w = synth.WORKLOADS[args.workload]
-    if args.tokens:
-        w = w.replace(n_tokens=min(args.tokens, w.n_tokens))
-    P = peaks()
     chunks = synth.chunk_bounds(w)
     q_h, k_h, v_h = gen_full(w, torch, device)
+    if plan is not None:
+        q_h = np.ascontiguousarray(q_h[:, plan.q0:plan.q1])
+        k_h = np.ascontiguousarray(k_h[:, plan.kv0:plan.kv1])
+        v_h = np.ascontiguousarray(v_h[:, plan.kv0:plan.kv1])
+        w = w.replace(n_q_heads=plan.q1 - plan.q0, n_kv_heads=plan.kv1 - plan.kv0)
     Q, K, V = (to_dev(a, torch, device) for a in (q_h, k_h, v_h))
     OUT = torch.empty_like(Q)
-    stream = torch.cuda.current_stream(device)
+    in_bytes = q_h.nbytes + k_h.nbytes + v_h.nbytes
+    big = in_bytes > L2_BYTES
     layer = InfLLMLayer.from_workload(w, max_tokens=w.n_tokens, max_chunk=w.chunk)
 
     def one_step():  # the whole prompt, chunk by chunk, in one call of the public API
         layer.reset()
         layer.prefill(Q, K, V, w.chunk, out=OUT)
 
+    flush = None if big else torch.ones(256 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
+    fsum = torch.empty((), dtype=torch.float32, device=device)
     for _ in range(args.warmup):
         one_step()
     torch.cuda.synchronize()
     layer.set_profiling(False)  # no events in the timed steps: they would break launch chaining
     barrier()
     torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
-        e0.record(stream)
-        for _ in range(args.steps):
-            one_step()
-        e1.record(stream)
-        torch.cuda.synchronize()
+        if big:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(args.steps):
+                one_step()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ms_step = e0.elapsed_time(e1) / args.steps
+        else:
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+            for a, b2 in evs:
+                torch.sum(flush, dim=0, out=fsum)  # read 256 MB (> L2) before every step
+                a.record(stream)
+                one_step()
+                b2.record(stream)
+            torch.cuda.synchronize()
+            ms_step = float(np.median([a.elapsed_time(b2) for a, b2 in evs]))
     barrier()
-    ms = e0.elapsed_time(e1)
-    ms = max_over_ranks(ms, device)
+    ms_step = max_over_ranks(ms_step, device)
     launches = layer.stats()["kernel_launches"]
     # the attention kernel's own duration: the same steps again with CUDA events around each
     # attention launch on the layer's stream (outside the timed region: events serialise it)
     layer.set_profiling(["attend"])
-    for _ in range(args.steps):
-        one_step()
-    torch.cuda.synchronize()
+    with ClockSampler(local) as clk_att:
+        for _ in range(args.steps):
+            if not big:
+                torch.sum(flush, dim=0, out=fsum)
+            one_step()
+        torch.cuda.synchronize()
     st = layer.stats()
     # where a step's time goes: one more step with events around every launch (diagnostic only;
     # the events break launch overlap, so these sum to more than the timed step)
@@ -264,51 +325,64 @@ def run_ours(args, rank, world):
     torch.cuda.synchronize()
     split = layer.stats()
     layer.set_profiling(False)
-    tokens_all = w.n_tokens * args.steps * world
-    value = tokens_all / (ms / 1e3)
-
-    # dominant kernel: the attention kernel (tensor-bound on the tcgen05 path)
     flops = sum(chunk_flops(w, c0, n) for c0, n in chunks) * args.steps
-    att_ms = st["ms_attend"]
-    n_att = st["n_attend"]
-    achieved_tf = flops / (att_ms / 1e3) / 1e12 if att_ms > 0 else None
-    tc = st["attend_path"] == 1
-    if tc:
-        peak = P["bf16_sust"]
-        roof = {"bound": "tensor", "achieved": achieved_tf, "peak": peak, "unit": "TFLOP/s",
-                "frac": (achieved_tf / peak) if achieved_tf else None, "traffic": attn_traffic(),
-                "kernel": "attention (tcgen05)", "peak_source": f"{P['src']} bf16 sustained",
-                "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of one steady-chunk launch "
-                                  "(profiles/k_attn_tc_mistral_128k.md); null if the kernel changed since"}
-    else:
-        # CUDA-core fp32 FMA path: 148 SMs x 128 FP32 lanes x 2 flop x max SM clock
-        peak = 148 * 128 * 2 * P["sm_max"] * 1e6 / 1e12
-        roof = {"bound": "alu", "achieved": achieved_tf, "peak": peak, "unit": "TFLOP/s",
-                "frac": (achieved_tf / peak) if achieved_tf else None, "traffic": None,
-                "kernel": "attention (SIMT fp32)", "peak_source": "148 SMs x 128 FP32 x 2 x max clock"}
-    roof["avg_launch_ms"] = att_ms / n_att if n_att else None
-    roof["launches"] = n_att
-    roof["timing"] = "CUDA events around each attention launch, over a repeat of the timed steps"
-    res = {"metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world, "steps": args.steps,
-           "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
-           "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded Philox normals, K channel bias N(0,4))",
-           "config": workload_config(w, world),
-           "roofline": roof, "gpu_launches": launches,
-           "clocks": clk.summary(),
-           "time_split_ms_per_step": {k: split[f"ms_{k}"]
-                                      for k in ("append", "reps", "prep", "select", "attend")}}
+    tokens_all = w.n_tokens * (1 if plan is not None else world)  # shards split one prompt; replicas run one each
+    fields = {"value": tokens_all / (ms_step / 1e3), "unit": "tok/s", "ms_per_step": ms_step,
+              "dtype": w.dtype, "config": workload_config(w, world, big, in_bytes),
+              "roofline": attn_roofline(w, st, flops, P, clk_att), "gpu_launches": launches * (1 if big else 1),
+              "clocks": clk.summary(),
+              "time_split_ms_per_step": {k: split[f"ms_{k}"] for k in ("append", "reps", "prep", "select", "attend")}}
+    del Q, K, V, OUT, flush
+    return fields, layer, (q_h, k_h, v_h)
 
-    if not args.no_e2e:
+
+def run_ours(args, rank, world):
+    import torch
+
+    _, _, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    w = synth.WORKLOADS[args.workload]
+    if args.tokens:
+        w = w.replace(n_tokens=min(args.tokens, w.n_tokens))
+    P = peaks()
+    stream = torch.cuda.current_stream(device)
+    plan = None
+    if args.parallel == "kv" and world > 1:
+        from block_memory_sparse_b200.sharding import ShardPlan
+        plan = ShardPlan(w.n_q_heads, w.n_kv_heads, world, rank)
+    fields, layer, (q_h, k_h, v_h) = time_prefill(args, w, torch, device, stream, local, world, P, plan)
+    if plan is not None:
+        fields["config"]["parallelism"] = f"KV heads split over {world} ranks ({plan.kv_per_rank} per rank)"
+    res = {"metric": METRIC, "value": fields["value"], "unit": "tok/s", "n_gpus": world, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": fields["ms_per_step"], "higher_is_better": True,
+           "scaling": "strong" if plan is not None else "weak", "vs_baseline": None, "dtype": w.dtype,
+           "data": "synthetic (seeded Philox normals, K channel bias N(0,4))", "config": fields["config"],
+           "roofline": fields["roofline"], "gpu_launches": fields["gpu_launches"], "clocks": fields["clocks"],
+           "time_split_ms_per_step": fields["time_split_ms_per_step"]}
+    if not args.no_e2e and plan is None:
         res["e2e"] = run_e2e(args, w, layer, q_h, k_h, v_h, torch, device, stream, world)
-    if not args.no_decode:
-        del Q, K, V, OUT
-        layer.close()
-        torch.cuda.empty_cache()
-        res["decode"] = run_decode(args, torch, device, stream, local)
-    else:
-        layer.close()
+    layer.close()
+    del q_h, k_h, v_h
+    torch.cuda.empty_cache()
     if rank == 0 and not args.no_cpu:
-        res["cpu_baseline"] = cpu_baseline(args.workload)
+        res["cpu_baseline"] = cpu_baseline(w.name)
+    # the other prefill workloads: same metric, their own roofline and oracle baseline
+    if not args.no_others:
+        others = {}
+        for name in ("llama3_128k", "needle_256k", "tiny_f32"):
+            if name == w.name:
+                continue
+            wo = synth.WORKLOADS[name]
+            f, lo, _ = time_prefill(args, wo, torch, device, stream, local, world, P)
+            lo.close()
+            torch.cuda.empty_cache()
+            if rank == 0 and not args.no_cpu:
+                f["cpu_baseline"] = cpu_baseline(name)
+            others[name] = f
+        res["other_workloads"] = others
+    if not args.no_decode:
+        res["decode"] = run_decode(args, torch, device, stream, local)
     return res
 
 
@@ -384,7 +458,7 @@ def run_decode(args, torch, device, stream, local):
     P = peaks()
     out = {}
     # memory of 1,052,800 tokens built once (untimed); both scoring pools are kept by the library
-    layer = InfLLMLayer.from_workload(w, max_tokens=w.n_tokens + 2 * steps + 32, max_chunk=w.build_chunk)
+    layer = InfLLMLayer.from_workload(w, max_tokens=w.n_tokens + 3 * steps + 48, max_chunk=w.build_chunk)
     t0 = time.time()
     for c0 in range(0, w.n_tokens, w.build_chunk):
         n = min(w.build_chunk, w.n_tokens - c0)
@@ -392,16 +466,19 @@ def run_decode(args, torch, device, stream, local):
         layer.append_chunk(to_dev(q, torch, device), to_dev(k, torch, device), to_dev(v, torch, device))
     torch.cuda.synchronize()
     build_s = time.time() - t0
-    qkv = [tuple(to_dev(a, torch, device) for a in synth.gen_chunk(w, w.n_tokens + s, 1)) for s in range(2 * steps)]
-    qkv_extra = [tuple(to_dev(a, torch, device) for a in synth.gen_chunk(w, w.n_tokens + 2 * steps + s, 1))
-                 for s in range(32)]
+    modes = ("reps", "repsum", "meankey")
+    nmodes = len(modes)
+    qkv = [tuple(to_dev(a, torch, device) for a in synth.gen_chunk(w, w.n_tokens + s, 1))
+           for s in range(nmodes * steps)]
+    qkv_extra = [tuple(to_dev(a, torch, device) for a in synth.gen_chunk(w, w.n_tokens + nmodes * steps + s, 1))
+                 for s in range(16 * nmodes)]
     o = torch.empty((1, w.n_q_heads, w.head_dim), dtype=torch.bfloat16, device=device)
     flush = torch.ones(256 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
     fsum = torch.empty((), dtype=torch.float32, device=device)
 
     def flush_l2():  # read 256 MB (> 126 MB L2): leaves clean lines, so no write-back lands in the step
         torch.sum(flush, dim=0, out=fsum)
-    for mi, mode in enumerate(("reps", "repsum")):
+    for mi, mode in enumerate(modes):
         layer.set_score_mode(mode)
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
         n_launch0 = layer.stats()["kernel_launches"]
@@ -450,16 +527,27 @@ def run_decode(args, torch, device, stream, local):
 
 
 def oracle_sample(workload):
-    """One steady chunk of the workload recomputed statelessly by the fp64 oracle: representatives
-    of every eligible unit, unit lookup, attention for the chunk's tokens."""
+    """A bounded sample of the workload through the fp64 oracle.  128K-token streams: one steady chunk
+    (chunk 64) recomputed statelessly -- representatives of every eligible unit, unit lookup, attention
+    for the chunk's tokens; the needle stream: its final chunk (the one that must find the needle); the
+    tiny fp32 stream: the whole stream, chunk by chunk (streaming oracle)."""
     from oracle import infllm_oracle as O
     from tests._source import Source
     w = synth.WORKLOADS[workload]
-    c0, n = synth.chunk_bounds(w)[64]
     src = Source(w)
+    chunks = synth.chunk_bounds(w)
+    if len(chunks) <= 64:
+        t = time.time()
+        layer = O.OracleLayer(w.as_config(), rep_method="linear")
+        for c0, n in chunks:
+            layer.append_chunk(src.q(c0, n), src.k(c0, n), src.v(c0, n))
+            layer.attend_chunk()
+        return w.n_tokens, time.time() - t, f"the whole {w.name} stream ({len(chunks)} chunks), streaming oracle"
+    ci = len(chunks) - 1 if w.needle else 64
+    c0, n = chunks[ci]
     t = time.time()
     O.chunk_stateless(src.q, src.k, src.v, c0, n, w.as_config())
-    return n, time.time() - t, f"chunk 64 (tokens [{c0}, {c0 + n})) of {w.name}, stateless recomputation"
+    return n, time.time() - t, f"chunk {ci} (tokens [{c0}, {c0 + n})) of {w.name}, stateless recomputation"
 
 
 def cpu_threads():
@@ -501,12 +589,17 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="mistral_128k", choices=["mistral_128k", "llama3_128k", "needle_256k"])
+    ap.add_argument("--workload", default="mistral_128k", choices=["mistral_128k", "llama3_128k", "needle_256k",
+                                                                    "tiny_f32"])
     ap.add_argument("--decode-steps", type=int, default=256)
     ap.add_argument("--decode-units", type=int, default=0, help="memory units of the decode workload (0: 8192)")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-others", action="store_true", help="skip the other prefill workloads")
+    ap.add_argument("--parallel", choices=["replicas", "kv"], default="replicas",
+                    help="N > 1: independent replicas (default, weak scaling) or one prompt's KV heads split over "
+                         "the ranks (strong scaling)")
     ap.add_argument("--tokens", type=int, default=0, help="truncate the prefill stream (small profiling cases)")
     ap.add_argument("--only", choices=["prefill", "decode"], default=None,
                     help="run only one part (profiling); the JSON line then carries that part alone")

@@ -22,7 +22,7 @@ library_path = os.path.join(_HERE, "libinfllm.so")
 
 STATUS = {0: "OK", 1: "EINVAL", 2: "ECAPACITY", 3: "ESTATE", 4: "ECUDA", 5: "EDEVICE"}
 DTYPES = {"f32": 0, "bf16": 1}
-SCORE_MODES = {"reps": 0, "repsum": 1}
+SCORE_MODES = {"reps": 0, "repsum": 1, "meankey": 2}
 
 
 class InfLLMError(RuntimeError):

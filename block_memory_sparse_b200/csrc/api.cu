@@ -58,6 +58,8 @@ struct infllm_ctx {
     // writes its selection to buffer L % 2 (so a lookup can run while the previous attention reads)
     int64_t nlook = 0;
     int last_sel = 0;   // selection buffer of the last attended chunk or token
+    unsigned long long dq_base = 0;  // the decode-step work counter's value at the next step's start
+    bool step_coop = true;           // decode steps in one cooperative launch (else three chained launches)
     int32_t* sel_base = nullptr;
     float* qbar_base = nullptr;
     // profiling
@@ -171,7 +173,8 @@ infllm_status validate(const infllm_config* g, char* msg, size_t n) {
     if (g->max_tokens < 1 || g->max_tokens > ((int64_t)1 << 31)) return bad("max_tokens must be in [1, 2^31]");
     if (!(g->rope_base > 1.0)) return bad("rope_base must be > 1");
     if (g->dtype != INFLLM_F32 && g->dtype != INFLLM_BF16) return bad("dtype must be INFLLM_F32 or INFLLM_BF16");
-    if (g->score_mode != INFLLM_SCORE_REPS && g->score_mode != INFLLM_SCORE_REPSUM) return bad("unknown score_mode");
+    if (g->score_mode != INFLLM_SCORE_REPS && g->score_mode != INFLLM_SCORE_REPSUM && g->score_mode != INFLLM_SCORE_MEANKEY)
+        return bad("unknown score_mode");
     const int64_t units = g->max_tokens / g->unit_size + 1;
     if (units > 16384) return bad("at most 16384 memory units (max_tokens / unit_size)");
     return INFLLM_OK;
@@ -338,69 +341,78 @@ infllm_status prefill_impl(infllm_ctx* c, const char* q, const char* k, const ch
 template <typename T>
 infllm_status decode_impl(infllm_ctx* c, const void* q, const void* k, const void* v, void* out) {
     infllm_status s;
-    bool new_reps = false;  // the lookup then needs the representatives just computed
-    if (sizeof(T) == 2 && c->use_tc && decode_tc_supported(c->D) && c->D.G <= 8) {
-        const Dev& D = c->D;
+    if (sizeof(T) == 2 && c->use_tc && decode_tc_supported(c->D)) {
+        // store + sink and window tiles (part 0) | lookup alongside | unit tiles + merge (part 1)
         const int64_t t = c->tokens;
-        const int64_t target = n_mem_at(t, D.S, D.W, D.U);
-        if (target > c->units_done) {
-            Prof p(c, K_REPS);
-            CK(launch_reps<T>(D, c->units_done, target, c->stream, pdl_ok(c)));
+        bool new_reps = false;  // the lookup then needs the representatives just computed
+        {
+            const Dev& D = c->D;
+            const int64_t target = n_mem_at(t, D.S, D.W, D.U);
+            if (target > c->units_done) {
+                Prof p(c, K_REPS);
+                CK(launch_reps<T>(D, c->units_done, target, c->stream, pdl_ok(c)));
+                c->chain = true;
+                p.done();
+                c->launches += 1;
+                c->units_done = target;
+                new_reps = true;
+            }
+        }
+        const int64_t L = c->nlook++;
+        const Dev D = lookup_dev(c, L);
+        const int nm = (int)n_mem_at(t, D.S, D.W, D.U);
+        const int kk = std::min(D.topk, nm);
+        const int64_t B = (int64_t)D.S + (int64_t)D.U * nm;
+        if (c->step_coop) {
+            // the whole step (store, sinks and window, lookup, units, merges) in one cooperative launch
+            Prof p(c, K_DECODE);
+            unsigned long long used = 0;
+            cudaError_t e = launch_decode_step(D, q, k, v, t, kk, B, nm, c->cfg.score_mode, (int)(L + 1), c->dq_base, out,
+                                               c->stream, c->tmaps, &used);
+            if (e != cudaSuccess) return fail(c, INFLLM_ECUDA, "decode step launch: %s", cudaGetErrorString(e));
+            c->dq_base += used;
             c->chain = true;
             p.done();
             c->launches += 1;
-            c->units_done = target;
-            new_reps = true;
+            c->tokens = t + 1;
+            c->pending = false;
+            record_attend(c, L, t, 1, nm, kk, B);
+            return INFLLM_OK;
         }
-        Prof p(c, K_APPEND);
-        CK(launch_decode_append(D, q, k, v, t, c->stream, pdl_ok(c)));
-        c->chain = true;
-        p.done();
-        c->launches += 1;
+        {   // three chained launches: part 0, the lookup alongside it, part 1
+            Prof p(c, K_DECODE);
+            cudaError_t e = launch_decode_tc(D, q, k, v, t, kk, B, 0, out, c->stream, c->tmaps, pdl_ok(c));
+            if (e != cudaSuccess) return fail(c, INFLLM_ECUDA, "decode launch (store, sinks, window): %s", cudaGetErrorString(e));
+            c->chain = true;
+            p.done();
+            c->launches += 1;
+        }
         c->tokens = t + 1;
-        c->pending = true;
-        c->pending_n = 1;
-        c->pending_c0 = t;
-    } else {
-        s = append_impl<T>(c, q, k, v, 1);
-        if (s != INFLLM_OK) return s;
+        c->pending = false;
+        if (kk > 0) {
+            s = stage_select<T>(c, L, nm, 1, q, new_reps);
+            if (s != INFLLM_OK) return s;
+            Prof p(c, K_DECODE);
+            cudaError_t e = launch_decode_tc(D, q, k, v, t, kk, B, 1, out, c->stream, c->tmaps, pdl_ok(c));
+            if (e != cudaSuccess) return fail(c, INFLLM_ECUDA, "decode launch (units): %s", cudaGetErrorString(e));
+            p.done();
+            c->launches += 1;
+        }
+        record_attend(c, L, t, 1, nm, kk, B);
+        return INFLLM_OK;
     }
+    s = append_impl<T>(c, q, k, v, 1);
+    if (s != INFLLM_OK) return s;
     const int64_t t = c->pending_c0;
-    c->pending = false;
     if (c->D.G > 8) {  // wide groups: the chunk kernels handle a single token as well
-        c->pending = true;
         return attend_impl<T>(c, q, 1, out, /*decoding=*/true);
     }
+    c->pending = false;
     const int64_t L = c->nlook++;
     const Dev D = lookup_dev(c, L);
     const int nm = (int)n_mem_at(t, D.S, D.W, D.U);
     const int kk = std::min(D.topk, nm);
     const int64_t B = (int64_t)D.S + (int64_t)D.U * nm;
-    if (sizeof(T) == 2 && c->use_tc && decode_tc_supported(D)) {
-        {   // sink and window tiles: independent of the lookup, so they run alongside it
-            Prof p(c, K_DECODE);
-            cudaError_t e = launch_decode_tc(D, q, t, kk, B, 0, c->stream, c->tmaps, pdl_ok(c));
-            if (e != cudaSuccess) return fail(c, INFLLM_ECUDA, "decode launch (sinks, window): %s", cudaGetErrorString(e));
-            c->chain = true;
-            p.done();
-            c->launches += 1;
-        }
-        if (kk > 0) {
-            s = stage_select<T>(c, L, nm, 1, q, new_reps);
-            if (s != INFLLM_OK) return s;
-        }
-        Prof p(c, K_DECODE);
-        if (kk > 0) {
-            cudaError_t e = launch_decode_tc(D, q, t, kk, B, 1, c->stream, c->tmaps, pdl_ok(c));
-            if (e != cudaSuccess) return fail(c, INFLLM_ECUDA, "decode launch (units): %s", cudaGetErrorString(e));
-            c->launches += 1;
-        }
-        CK(launch_decode_merge(D, t, kk, B, out, c->stream, pdl_ok(c)));
-        p.done();
-        c->launches += 1;
-        record_attend(c, L, t, 1, nm, kk, B);
-        return INFLLM_OK;
-    }
     if (kk > 0) {
         s = stage_select<T>(c, L, nm, 1, q, true);
         if (s != INFLLM_OK) return s;
@@ -417,7 +429,10 @@ infllm_status decode_impl(infllm_ctx* c, const void* q, const void* k, const voi
 
 infllm_status zero_state(infllm_ctx* c) {
     CK(cudaMemsetAsync(c->D.Y, 0, sizeof(float) * (size_t)((c->D.T_max / c->D.gblk) + 2) * c->D.Hkv * c->D.d, c->stream));
-    CK(cudaMemsetAsync(c->D.counters, 0, sizeof(unsigned) * 2 * c->D.Hkv, c->stream));
+    CK(cudaMemsetAsync(c->D.counters, 0, sizeof(unsigned) * 4 * c->D.Hkv, c->stream));
+    CK(cudaMemsetAsync(c->D.dflags, 0, sizeof(int) * 2 * c->D.Hkv, c->stream));
+    CK(cudaMemsetAsync(c->D.dq, 0, sizeof(unsigned long long), c->stream));
+    c->dq_base = 0;
     CK(cudaMemsetAsync(c->sel_base, 0xff, sizeof(int32_t) * 2 * (size_t)c->D.Hkv * std::max(1, c->D.topk), c->stream));
     c->tokens = 0;
     c->units_done = 0;
@@ -492,15 +507,20 @@ infllm_status create_impl(infllm_ctx* c) {
     AL(D.rep_ids, sizeof(int32_t) * (size_t)D.Hkv * D.units_max * D.r);
     AL(D.rep_keys, (size_t)D.Hkv * D.units_max * D.r * D.d * c->elt);
     AL(D.repsum, sizeof(float) * (size_t)D.Hkv * D.units_max * D.d);
+    AL(D.meankey, (size_t)D.Hkv * D.units_max * D.d * c->elt);
     AL(D.sel, sizeof(int32_t) * 2 * (size_t)D.Hkv * std::max(1, D.topk));  // two buffers
     AL(D.uscore, sizeof(float) * (size_t)D.Hkv * D.units_max);
     AL(D.qbar_part, sizeof(float) * 2 * (size_t)D.Hkv * D.qtiles_max * D.d);  // two buffers
     AL(D.cand, sizeof(uint64_t) * (size_t)D.Hkv * D.score_splits_max * 32);
-    AL(D.counters, sizeof(unsigned) * 2 * D.Hkv);
+    AL(D.counters, sizeof(unsigned) * 4 * D.Hkv);
+    AL(D.dflags, sizeof(int) * 2 * D.Hkv);
+    AL(D.dq, sizeof(unsigned long long));
     AL(D.Qm, (size_t)D.Hkv * 3 * D.qrows_max * D.d * c->elt);  // three slots
     AL(D.Qw, (size_t)D.Hkv * 3 * D.qrows_max * D.d * c->elt);
     AL(D.cs_chunk, sizeof(float2) * (size_t)g.max_chunk * D.half);
-    AL(D.dec_part, sizeof(float) * (size_t)D.Hkv * D.dec_splits_max * D.G * (D.d + 2));
+    AL(D.dec_part, sizeof(float) * (size_t)D.Hkv * D.dec_splits_max * D.G * (D.d + 4));
+
+
     double* invf = nullptr;
     float2* cs_rel = nullptr;
     float2* cs_w = nullptr;
@@ -540,6 +560,7 @@ infllm_status create_impl(infllm_ctx* c) {
     *c->err_host = 0;
     CK(cudaHostGetDevicePointer((void**)&D.err, c->err_host, 0));
     c->use_tc = false;
+    c->step_coop = getenv("INFLLM_DECODE_CHAIN") == nullptr;
     if (g.dtype == INFLLM_BF16 && attend_tc_supported(D) && getenv("INFLLM_FORCE_SIMT") == nullptr) {
         c->tmaps = malloc(tc_maps_size());
         c->use_tc = c->tmaps && make_tc_maps(D, c->tmaps);
@@ -723,7 +744,8 @@ infllm_status infllm_get_stats(infllm_ctx* c, infllm_stats* o) {
 
 infllm_status infllm_set_score_mode(infllm_ctx* c, int32_t mode) {
     if (!c) return INFLLM_EINVAL;
-    if (mode != INFLLM_SCORE_REPS && mode != INFLLM_SCORE_REPSUM) return fail(c, INFLLM_EINVAL, "unknown score_mode %d", mode);
+    if (mode != INFLLM_SCORE_REPS && mode != INFLLM_SCORE_REPSUM && mode != INFLLM_SCORE_MEANKEY)
+        return fail(c, INFLLM_EINVAL, "unknown score_mode %d", mode);
     c->cfg.score_mode = mode;
     return INFLLM_OK;
 }

@@ -29,12 +29,16 @@ struct Dev {
     int32_t* rep_ids;     // [Hkv][units_max][r] unit-local offsets, ascending
     void* rep_keys;       // [Hkv][units_max][r][d] raw keys (context dtype)
     float* repsum;        // [Hkv][units_max][d] fp32 sum of the r raw keys
+    void* meankey;        // [Hkv][units_max][d] mean of the unit's U raw keys (context dtype)
     // lookup
     int32_t* sel;         // [Hkv][topk] ascending ids, -1 padded (the current lookup's of two buffers)
     float* uscore;        // [Hkv][units_max] last chunk's unit scores
     float* qbar_part;     // [Hkv][qtiles_max][d] per-tile raw query sums (the current lookup's of two)
     uint64_t* cand;       // [Hkv][score_splits_max][32] top-k candidate lists
-    unsigned* counters;   // [2][Hkv] arrival counters (last CTA done): unit selection, CUDA-core decode merge
+    unsigned* counters;   // [4][Hkv] arrival counters (last CTA done): unit selection, CUDA-core decode merge,
+                          // tile decode part 0 and part 1
+    int* dflags;          // [2][Hkv] decode-step flags (step tags): selection final, sinks and window merged
+    unsigned long long* dq;  // decode-step work counter (monotonic; the host keeps each step's base)
     // rotated, packed queries of a chunk: [Hkv][3][qrows_max][d] (three slots, so later chunks'
     // queries can be packed while an earlier chunk's attention runs)
     void* Qm;             // R(W) q  (sink / memory frame)
@@ -50,7 +54,7 @@ struct Dev {
     // (cos, sin)(x 2^(11 L) theta_i) in fp64 for L < 3, x < 2048: exp(i t theta) for any
     // t < 2^33 is the product of three entries (t's 11-bit digits)
     const double2* cs_abs3;  // [3][2048][half]
-    // decode partials: [Hkv][dec_splits_max][G][d + 2]
+    // decode partials: [Hkv][dec_splits_max][G][d + 4] (the CUDA-core decode uses [G][d + 2] of a slot)
     float* dec_part;
     int dec_splits_max;
     int score_splits_max;
@@ -58,6 +62,10 @@ struct Dev {
     // error word (host-mapped)
     int* err;
 };
+
+// Unit-scoring operand (the score modes of the C ABI): the n_reps representative keys, their fp32
+// sum, or the mean of all of the unit's keys.
+enum ScoreOperand : int { OP_REPS = 0, OP_REPSUM = 1, OP_MEANKEY = 2 };
 
 // ---- programmatic dependent launch -------------------------------------------------------
 // Kernels of one stream are chained with programmatic dependent launch.  Two kinds:
@@ -83,6 +91,16 @@ enum ErrBits : int {
 
 __device__ __forceinline__ void set_err(const Dev& D, int bit) { atomicOr(D.err, bit); }
 
+// Release store / acquire load of a GPU-scope flag (kernels that hand a result to other CTAs).
+__device__ __forceinline__ void st_release(int* p, int v) {
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ int ld_acquire(const int* p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
 // ---- element conversions --------------------------------------------------------------
 template <typename T> __device__ __forceinline__ float to_f(T x);
 template <> __device__ __forceinline__ float to_f<float>(float x) { return x; }
@@ -90,6 +108,10 @@ template <> __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 x
 template <typename T> __device__ __forceinline__ T from_f(float x);
 template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
 template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
+// fp64 to the element type, one rounding (to nearest, ties to even)
+template <typename T> __device__ __forceinline__ T from_d(double x);
+template <> __device__ __forceinline__ float from_d<float>(double x) { return __double2float_rn(x); }
+template <> __device__ __forceinline__ __nv_bfloat16 from_d<__nv_bfloat16>(double x) { return __double2bfloat16(x); }
 
 // ---- ordered composite keys for deterministic top-k ------------------------------------
 // Larger key = better.  High word: order-preserving image of the float score (+0 == -0).

@@ -8,19 +8,23 @@
 // KV head rescales every partial by exp(m_s - M) and divides by the total sum.
 //
 // Launch sequence of one step (programmatic dependent launches after the first):
-//   k_decode_append           store the token (early kernel)
-//   k_decode_attn, part 0     sink and window tiles: need the store, not the selection
+//   k_decode_attn, part 0     the token's store (by the CTA whose tile holds it) and the sink and
+//                             window tiles, which need no selection; the last CTA of each KV head
+//                             merges their partials into one (early kernel)
 //   unit scoring + top-k      reads only the representative pool and the query, so it runs
 //                             alongside part 0 (it holds its completion until part 0 is done)
-//   k_decode_attn, part 1     the selected units' tiles (waits for the selection)
-//   k_decode_merge            log-sum-exp merge of every tile's partial
+//   k_decode_attn, part 1     the selected units' tiles (waits for the selection); the last CTA
+//                             of each KV head merges them with part 0's partial into the output
 #include <cuda.h>
 #include <math.h>
+
+#include <algorithm>
 
 #include "common.cuh"
 #include "kernels.h"
 #include "tc_maps.cuh"
 #include "tc_ptx.cuh"
+#include "topk.cuh"
 
 namespace infllm {
 namespace {
@@ -33,66 +37,19 @@ constexpr int DTHREADS = 128;
 constexpr int MAXG = 8;  // q heads per KV head on this path (rows of the padded MMA tile)
 constexpr int ERR_TIMEOUT = 16;
 // dynamic shared memory: K tile | V tile | this tile's rotated query [16 rows][d] bf16 (rows >= G
-// zero, padded row stride) | reductions.  The P V partials of the four warps reuse the K tile.
+// zero, padded row stride) | reductions | barrier and flags | (cos, sin)(t theta_i).  The P V
+// partials of the four warps reuse the K tile, and the final merges reuse both tiles.
 constexpr int QSTRIDE = DHD * 2 + 16;  // bytes per padded query row (conflict-free ldmatrix)
 constexpr int OFF_K = 0;
 constexpr int OFF_V = OFF_K + (int)DTILE;
 constexpr int OFF_Q = OFF_V + (int)DTILE;
 constexpr int OFF_RED = OFF_Q + 16 * QSTRIDE;
 constexpr int OFF_MISC = OFF_RED + 2 * 4 * 8 * 4;
-constexpr int DSMEM = OFF_MISC + 64 + 1024;  // + alignment slack
-
-// One CTA per KV head: K, R(t) K and V of token t into the stores, the query block sum of t,
-// and (cos, sin)(t theta_i) in fp64 for the attention kernel.
-__global__ void __launch_bounds__(DTHREADS) k_decode_append(Dev D, const __nv_bfloat16* __restrict__ q,
-                                                            const __nv_bfloat16* __restrict__ k,
-                                                            const __nv_bfloat16* __restrict__ v, int64_t t) {
-    __shared__ float2 cs[DHD / 2];
-    pdl_trigger();  // early kernel: the lookup may start now (it reads none of these stores)
-    const int hk = blockIdx.x;
-    for (int i = threadIdx.x; i < D.half; i += blockDim.x) {
-        cs[i] = cs_abs(D.cs_abs3, D.half, t, i);
-        if (hk == 0) D.cs_chunk[i] = cs[i];
-    }
-    __syncthreads();
-    __nv_bfloat16* Kraw = (__nv_bfloat16*)D.Kraw;
-    __nv_bfloat16* Krot = (__nv_bfloat16*)D.Krot;
-    __nv_bfloat16* V = (__nv_bfloat16*)D.V;
-    const int64_t dst = ((int64_t)hk * D.T_max + t) * D.d;
-    for (int i = threadIdx.x; i < D.half; i += blockDim.x) {
-        const __nv_bfloat16 a = k[hk * D.d + i], b = k[hk * D.d + i + D.half];
-        Kraw[dst + i] = a;
-        Kraw[dst + i + D.half] = b;
-        const float x1 = __bfloat162float(a), x2 = __bfloat162float(b);
-        Krot[dst + i] = __float2bfloat16_rn(x1 * cs[i].x - x2 * cs[i].y);
-        Krot[dst + i + D.half] = __float2bfloat16_rn(x2 * cs[i].x + x1 * cs[i].y);
-        V[dst + i] = v[hk * D.d + i];
-        V[dst + i + D.half] = v[hk * D.d + i + D.half];
-        if (t >= D.S) {  // query block sum (same arithmetic as the chunk kernel for one token)
-            const int64_t b = (t - D.S) / D.gblk, p = (t - D.S) % D.gblk;
-            float qx[MAXG], qy[MAXG];
-#pragma unroll
-            for (int h = 0; h < MAXG; ++h) {
-                qx[h] = qy[h] = 0.f;
-                if (h < D.G) {
-                    qx[h] = __bfloat162float(q[(hk * D.G + h) * D.d + i]);
-                    qy[h] = __bfloat162float(q[(hk * D.G + h) * D.d + i + D.half]);
-                }
-            }
-            float s1 = 0.f, s2 = 0.f;
-#pragma unroll
-            for (int h = 0; h < MAXG; ++h) {
-                s1 += qx[h];
-                s2 += qy[h];
-            }
-            const float2 c = D.cs_rel[p * D.half + i];
-            float* y = D.Y + (b * D.Hkv + hk) * D.d;
-            y[i] += s1 * c.x - s2 * c.y;
-            y[i + D.half] += s2 * c.x + s1 * c.y;
-        }
-    }
-    pdl_hold();
-}
+constexpr int OFF_CS = OFF_MISC + 64;
+constexpr int DSMEM = OFF_CS + (DHD / 2) * 8 + 1024;  // + alignment slack
+static_assert(MAXG * 64 * 4 + MAXG * 2 * 4 <= 16 * QSTRIDE, "merge weights do not fit the query rows' space");
+// A tile's partial softmax per q head: m (natural-log units), l, two pad floats, o[d] unnormalised.
+constexpr int PST = DHD + 4;
 
 struct DTile {
     int kind;  // 0 sink, 1 unit, 2 window
@@ -147,34 +104,162 @@ __device__ __forceinline__ uint32_t tile_chunk(uint32_t base, int j, int c) {
     return base + (uint32_t)(c >> 3) * DHALF + (uint32_t)j * 128 + ((uint32_t)((c & 7) ^ (j & 7)) << 4);
 }
 
-// Grid (tiles, Hkv), 128 threads = 4 warps, warp w owns keys [32w, 32w + 32) of the tile.
-// The group's G query heads (rows, padded to 16 with zeros) times the tile on the tensor cores
-// (mma.sync m16n8k16, bf16 in, fp32 accumulate): S = Q K^T, then O = P V with P kept in
-// registers; softmax statistics are combined across the four warps through shared memory.
-__global__ void __launch_bounds__(DTHREADS) k_decode_attn(const __grid_constant__ TcMaps maps, Dev D,
-                                                          const __nv_bfloat16* __restrict__ q, int64_t t, int kk,
-                                                          int64_t B, int part) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(ptx::smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
+// Combine the partial softmaxes of `ns` tiles of KV head hk (slot_of(i) gives the i-th tile's slot,
+// in a fixed order) into one: per q head, M = max m, L = sum exp(m - M) l, O = sum exp(m - M) o.
+// A batch of slots is copied into shared memory at once (16-byte asynchronous copies, every copy of
+// the batch in flight together); then one warp per q head computes M, the weights and L, and each
+// thread (one output dim) sums the weighted o.  Batches (when the slots exceed `cap` floats) are
+// combined by the same rule.  Writes the normalised output O / L (out != null) or the merged partial
+// into slot `dst_slot`.  Exact up to rounding: the log-sum-exp combination of disjoint key sets.
+template <typename SlotOf>
+__device__ void merge_partials(const Dev& D, int hk, int ns, SlotOf slot_of, float* sbuf, int cap,
+                               float (*wts)[64], float (*stat)[2], __nv_bfloat16* __restrict__ out, int dst_slot) {
+    // wts[MAXG][64]: weights of a batch's slots (at most 64 per batch); stat[MAXG][2]: a batch's (M, L)
+    const int G = D.G, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int sf = G * PST;  // floats per slot
+    const int per = min(64, cap / sf);
+    float* pbase = D.dec_part + (int64_t)hk * D.dec_splits_max * sf;
+    float M[MAXG], L[MAXG], O[MAXG];  // running totals (thread: output dim tid)
+#pragma unroll
+    for (int h = 0; h < MAXG; ++h) {
+        M[h] = -INFINITY;
+        L[h] = 0.f;
+        O[h] = 0.f;
+    }
+    for (int r0 = 0; r0 < ns; r0 += per) {
+        const int nr = min(per, ns - r0);
+        const int w4 = sf / 4;
+        for (int x = tid; x < nr * w4; x += DTHREADS) {
+            const int sl = x / w4, w = x % w4;
+            cp_async16(sbuf + (size_t)x * 4, pbase + (int64_t)slot_of(r0 + sl) * sf + 4 * w);
+        }
+        cp_async_wait_all();
+        __syncthreads();
+        for (int h = warp; h < G; h += DTHREADS / 32) {
+            float mx = -INFINITY;
+            for (int sl = lane; sl < nr; sl += 32) mx = fmaxf(mx, sbuf[sl * sf + h * PST]);
+            mx = warp_max(mx);
+            float l = 0.f;
+            for (int sl = lane; sl < nr; sl += 32) {
+                const float m = sbuf[sl * sf + h * PST];
+                const float wgt = m == -INFINITY ? 0.f : expf(m - mx);  // a tile with no attended key weighs 0
+                wts[h][sl] = wgt;
+                l = fmaf(wgt, sbuf[sl * sf + h * PST + 1], l);
+            }
+            l = warp_sum(l);
+            if (lane == 0) {
+                stat[h][0] = mx;
+                stat[h][1] = l;
+            }
+        }
+        __syncthreads();
+#pragma unroll
+        for (int h = 0; h < MAXG; ++h) {
+            if (h >= G) continue;
+            float o = 0.f;
+            for (int sl = 0; sl < nr; ++sl) o = fmaf(wts[h][sl], sbuf[sl * sf + h * PST + 4 + tid], o);
+            const float mb = stat[h][0], lb = stat[h][1];
+            if (mb == -INFINITY) continue;
+            if (mb > M[h]) {  // rescale the running totals to the larger max
+                const float f = M[h] == -INFINITY ? 0.f : expf(M[h] - mb);
+                L[h] = fmaf(L[h], f, lb);
+                O[h] = fmaf(O[h], f, o);
+                M[h] = mb;
+            } else {
+                const float f = expf(mb - M[h]);
+                L[h] = fmaf(f, lb, L[h]);
+                O[h] = fmaf(f, o, O[h]);
+            }
+        }
+        __syncthreads();  // the batch's buffers are reused
+    }
+#pragma unroll
+    for (int h = 0; h < MAXG; ++h) {
+        if (h >= G) continue;
+        if (out) {
+            out[(int64_t)(hk * G + h) * DHD + tid] = __float2bfloat16_rn(O[h] / L[h]);
+        } else {
+            float* p = pbase + (int64_t)dst_slot * sf + h * PST;
+            p[4 + tid] = O[h];
+            if (tid == 0) {
+                p[0] = M[h];
+                p[1] = L[h];
+            }
+        }
+    }
+}
+
+// One 128-key tile of the token's working context against the group's G query heads: the partial
+// softmax (m, l, o) of every q head into slot ti of KV head hk.  Block of 128 threads = 4 warps, warp
+// w owns keys [32w, 32w + 32) of the tile.  The group's G query heads (rows, padded to 16 with
+// zeros) times the tile on the tensor cores (mma.sync m16n8k16, bf16 in, fp32 accumulate): S = Q K^T,
+// then O = P V with P kept in registers; softmax statistics are combined across the four warps
+// through shared memory.  With store_here (the tile that holds token t) the token is stored first
+// (K, R(t) K and V of KV head hk, and its query block sum), so the step needs no store kernel.
+// `phase` is the parity of the CTA's tile barrier, flipped per tile.  Returns false on a timeout.
+__device__ bool tile_partial(const TcMaps& maps, const Dev& D, const __nv_bfloat16* __restrict__ q,
+                             const __nv_bfloat16* __restrict__ knew, const __nv_bfloat16* __restrict__ vnew, int64_t t,
+                             int hk, int ti, const DTile& T, bool store_here, uint8_t* sm, uint32_t& phase) {
     float* red = reinterpret_cast<float*>(sm + OFF_RED);  // [2][4 warps][8 rows]
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + OFF_MISC);
-    const int hk = blockIdx.y;
-    // tile index in the working context (sinks, units, window): part 0 takes sinks and window,
-    // part 1 the selected units
-    const int nst = ((D.S < t + 1 ? D.S : (int)(t + 1)) + DK - 1) / DK;
-    const int nut = kk * ((D.U + DK - 1) / DK);
-    const int ti = part == 1 ? nst + (int)blockIdx.x : ((int)blockIdx.x < nst ? (int)blockIdx.x : (int)blockIdx.x + nut);
+    const float2* cs_t = reinterpret_cast<const float2*>(sm + OFF_CS);  // (cos, sin)(t theta_i)
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, tg = lane & 3;
     const int G = D.G;
-    pdl_trigger();  // the next kernel reads nothing this one writes before the merge
-    if (tid == 0) {
-        ptx::mbar_init(bar, 1);
-        ptx::mbar_fence_init();
+    if (store_here) {
+        // this tile holds the new token: store it before the tile is loaded
+        __nv_bfloat16* Kraw = (__nv_bfloat16*)D.Kraw;
+        __nv_bfloat16* Krot = (__nv_bfloat16*)D.Krot;
+        __nv_bfloat16* Vs = (__nv_bfloat16*)D.V;
+        const int64_t dst = ((int64_t)hk * D.T_max + t) * DHD;
+        for (int i = tid; i < DHD / 2; i += DTHREADS) {
+            const __nv_bfloat16 a = knew[hk * DHD + i], b = knew[hk * DHD + i + DHD / 2];
+            Kraw[dst + i] = a;
+            Kraw[dst + i + DHD / 2] = b;
+            const float x1 = __bfloat162float(a), x2 = __bfloat162float(b);
+            const float2 c = cs_t[i];
+            Krot[dst + i] = __float2bfloat16_rn(x1 * c.x - x2 * c.y);
+            Krot[dst + i + DHD / 2] = __float2bfloat16_rn(x2 * c.x + x1 * c.y);
+            Vs[dst + i] = vnew[hk * DHD + i];
+            Vs[dst + i + DHD / 2] = vnew[hk * DHD + i + DHD / 2];
+            if (t >= D.S) {  // the token's query block sum (same arithmetic as the chunk kernel)
+                const int64_t blk = (t - D.S) / D.gblk, p = (t - D.S) % D.gblk;
+                float qx[MAXG], qy[MAXG];
+#pragma unroll
+                for (int h = 0; h < MAXG; ++h) {
+                    qx[h] = qy[h] = 0.f;
+                    if (h < G) {
+                        qx[h] = __bfloat162float(q[(hk * G + h) * DHD + i]);
+                        qy[h] = __bfloat162float(q[(hk * G + h) * DHD + i + DHD / 2]);
+                    }
+                }
+                float s1 = 0.f, s2 = 0.f;
+#pragma unroll
+                for (int h = 0; h < MAXG; ++h) {
+                    s1 += qx[h];
+                    s2 += qy[h];
+                }
+                const float2 cr = D.cs_rel[p * D.half + i];
+                float* y = D.Y + (blk * D.Hkv + hk) * DHD;
+                y[i] += s1 * cr.x - s2 * cr.y;
+                y[i + DHD / 2] += s2 * cr.x + s1 * cr.y;
+            }
+        }
+        // the rows just written are read next by this CTA's bulk tensor copy (async proxy)
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        __syncthreads();
     }
+    // shared memory written by the generic proxy (the previous tile's partial sums, a merge's copies)
+    // is about to be overwritten by a bulk tensor copy
+    ptx::fence_proxy_async_smem();
     __syncthreads();
-    pdl_wait();  // the token's store, its (cos, sin) and (part 1) the selection are ready past this point
-    const DTile T = decode_tile(D, hk, ti, t, kk, B);
     if (tid == 0) {
         const CUtensorMap* km = T.kind == 2 ? &maps.krot : &maps.kraw;
         ptx::mbar_expect_tx(bar, 2 * DTILE);
@@ -185,7 +270,7 @@ __global__ void __launch_bounds__(DTHREADS) k_decode_attn(const __grid_constant_
     }
     // this tile's query frame (R(W) q for sinks and memory, R(t) q for the window) as bf16 rows
     {
-        const float2* cs = T.kind == 2 ? D.cs_chunk : D.cs_W;
+        const float2* cs = T.kind == 2 ? cs_t : D.cs_W;
         for (int idx = tid; idx < 16 * (DHD / 2); idx += DTHREADS) {
             const int h = idx / (DHD / 2), i = idx % (DHD / 2);
             float r1 = 0.f, r2 = 0.f;
@@ -208,7 +293,8 @@ __global__ void __launch_bounds__(DTHREADS) k_decode_attn(const __grid_constant_
 #pragma unroll
         for (int ks = 0; ks < DHD / 16; ++ks) ldsm_x4(qbase + ks * 32, qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3]);
     }
-    bool ok = ptx::mbar_wait(bar, 0);
+    bool ok = ptx::mbar_wait(bar, phase);
+    phase ^= 1u;
     if (!ok) set_err(D, ERR_TIMEOUT);
     ok = __syncthreads_and(ok);
     // S for the warp's 32 keys: n-tiles nt -> keys 32w + 8nt + (0..7)
@@ -218,7 +304,7 @@ __global__ void __launch_bounds__(DTHREADS) k_decode_attn(const __grid_constant_
     for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
-    {
+    if (ok) {
         const int key_a = 32 * warp + (lane & 7);  // lanes 0-15: n-tile 2p, lanes 16-31: n-tile 2p + 1
 #pragma unroll
         for (int ks = 0; ks < DHD / 16; ++ks) {
@@ -271,16 +357,18 @@ __global__ void __launch_bounds__(DTHREADS) k_decode_attn(const __grid_constant_
     for (int nt = 0; nt < 16; ++nt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) oacc[nt][e] = 0.f;
+    if (ok) {
 #pragma unroll
-    for (int ks = 0; ks < 2; ++ks) {
-        const int key = 32 * warp + 16 * ks + (lane & 7) + (((lane >> 3) & 1) << 3);
+        for (int ks = 0; ks < 2; ++ks) {
+            const int key = 32 * warp + 16 * ks + (lane & 7) + (((lane >> 3) & 1) << 3);
 #pragma unroll
-        for (int np = 0; np < 8; ++np) {
-            const int c = 2 * np + (lane >> 4);
-            uint32_t b0, b1, b2, b3;
-            ldsm_x4_t(tile_chunk(vbase, key, c), b0, b1, b2, b3);
-            mma16816(oacc[2 * np], pa[ks], b0, b1);
-            mma16816(oacc[2 * np + 1], pa[ks], b2, b3);
+            for (int np = 0; np < 8; ++np) {
+                const int c = 2 * np + (lane >> 4);
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4_t(tile_chunk(vbase, key, c), b0, b1, b2, b3);
+                mma16816(oacc[2 * np], pa[ks], b0, b1);
+                mma16816(oacc[2 * np + 1], pa[ks], b2, b3);
+            }
         }
     }
     __syncthreads();  // every warp is done with the K tile: reuse it for the cross-warp sum of O
@@ -291,67 +379,304 @@ __global__ void __launch_bounds__(DTHREADS) k_decode_attn(const __grid_constant_
         obuf[(warp * 8 + g) * DHD + 8 * nt + 2 * tg + 1] = oacc[nt][1];
     }
     __syncthreads();
-    float* pout = D.dec_part + ((int64_t)hk * D.dec_splits_max + ti) * G * (DHD + 2);
+    float* pout = D.dec_part + ((int64_t)hk * D.dec_splits_max + ti) * G * PST;
     for (int h = 0; h < G; ++h) {
         const float o = obuf[(0 * 8 + h) * DHD + tid] + obuf[(1 * 8 + h) * DHD + tid] + obuf[(2 * 8 + h) * DHD + tid] +
                         obuf[(3 * 8 + h) * DHD + tid];
-        pout[h * (DHD + 2) + 2 + tid] = o;
+        pout[h * PST + 4 + tid] = o;
         if (tid == 0) {
             const float mh = fmaxf(fmaxf(red[h], red[8 + h]), fmaxf(red[16 + h], red[24 + h]));
-            pout[h * (DHD + 2) + 0] = mh == -INFINITY ? -INFINITY : mh * D.inv_sqrt_d;  // natural-log units
-            pout[h * (DHD + 2) + 1] = red[32 + h] + red[40 + h] + red[48 + h] + red[56 + h];
+            pout[h * PST + 0] = mh == -INFINITY ? -INFINITY : mh * D.inv_sqrt_d;  // natural-log units
+            pout[h * PST + 1] = red[32 + h] + red[40 + h] + red[48 + h] + red[56 + h];
         }
     }
+    return ok;
 }
 
-// Log-sum-exp merge of the NT tile partials of one (KV head, q head): grid (G, Hkv), 512 threads
-// = 4 slices of tiles x 128 output dims; every load of a slice issued in one batch.
-constexpr int MERGE_SLICES = 4;
-constexpr int MERGE_BATCH = 32;
+// The partials of KV head hk's tiles of one part are all written: merge them (part 0: sinks and
+// window into slot NT, or the output when no unit is selected; part 1: part 0's slot and the units
+// into the output).
+__device__ void merge_part(const Dev& D, int hk, int part, int nst, int nut, int nwt, int kk, uint8_t* sm,
+                           __nv_bfloat16* __restrict__ out) {
+    float* sbuf = reinterpret_cast<float*>(sm + OFF_K);  // K and V tiles: 64 KB
+    const int cap = (int)(2 * DTILE / 4);
+    auto wts = reinterpret_cast<float(*)[64]>(sm + OFF_Q);  // the query rows' space: 2 KB + 64 B
+    auto stat = reinterpret_cast<float(*)[2]>(sm + OFF_Q + MAXG * 64 * 4);
+    const int NT = nst + nut + nwt;
+    if (part == 0)
+        merge_partials(D, hk, nst + nwt, [=](int i) { return i < nst ? i : i + nut; }, sbuf, cap, wts, stat,
+                       kk == 0 ? out : nullptr, NT);
+    else
+        merge_partials(D, hk, 1 + nut, [=](int i) { return i == 0 ? NT : nst + i - 1; }, sbuf, cap, wts, stat, out, 0);
+}
 
-__global__ void __launch_bounds__(MERGE_SLICES * DHD) k_decode_merge(Dev D, __nv_bfloat16* __restrict__ out, int NT) {
-    __shared__ float ml[2][MERGE_SLICES * MERGE_BATCH];
-    __shared__ float red[2][MERGE_SLICES][DHD];
-    pdl_wait();     // the tile partials are complete past this point
-    pdl_trigger();  // every earlier kernel is complete: the next step's store kernels may start
-    const int h = blockIdx.x, hk = blockIdx.y, G = D.G, d = DHD;
-    const int dim = threadIdx.x % DHD, z = threadIdx.x / DHD;
-    const float* base = D.dec_part + (int64_t)hk * D.dec_splits_max * G * (d + 2) + (int64_t)h * (d + 2);
-    const int64_t stride = (int64_t)G * (d + 2);
-    for (int s = threadIdx.x; s < NT && s < MERGE_SLICES * MERGE_BATCH; s += blockDim.x) {
-        ml[0][s] = base[s * stride];
-        ml[1][s] = base[s * stride + 1];
+// Grid (tiles, Hkv), 128 threads: one tile per CTA.
+//   part 0: the sink and window tiles (an early kernel: it reads no result of its predecessor);
+//   part 1: the selected units' tiles, after the selection.
+// The head's last CTA of each part (arrival counter, no CTA waits for another) merges its partials.
+__global__ void __launch_bounds__(DTHREADS, 1) k_decode_attn(const __grid_constant__ TcMaps maps, Dev D,
+                                                          const __nv_bfloat16* __restrict__ q,
+                                                          const __nv_bfloat16* __restrict__ knew,
+                                                          const __nv_bfloat16* __restrict__ vnew, int64_t t, int kk,
+                                                          int64_t B, int part, __nv_bfloat16* __restrict__ out) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + OFF_MISC);
+    int* is_last = reinterpret_cast<int*>(sm + OFF_MISC + 8);
+    float2* cs_t = reinterpret_cast<float2*>(sm + OFF_CS);
+    const int hk = blockIdx.y, tid = threadIdx.x;
+    const int nst = ((D.S < t + 1 ? D.S : (int)(t + 1)) + DK - 1) / DK;
+    const int nut = kk * ((D.U + DK - 1) / DK);
+    const int nwt = (int)((t - B + 1 + DK - 1) / DK);
+    const int ti = part == 1 ? nst + (int)blockIdx.x : ((int)blockIdx.x < nst ? (int)blockIdx.x : (int)blockIdx.x + nut);
+    if (part == 0) pdl_trigger();  // early: the lookup runs alongside
+    if (tid == 0) {
+        ptx::mbar_init(bar, 1);
+        ptx::mbar_fence_init();
+    }
+    for (int i = tid; i < DHD / 2; i += DTHREADS) cs_t[i] = cs_abs(D.cs_abs3, D.half, t, i);
+    __syncthreads();
+    if (part == 1) {
+        pdl_wait();  // the selection (and everything before it) is complete past this point
+        pdl_trigger();
+    }
+    const DTile T = decode_tile(D, hk, ti, t, kk, B);
+    uint32_t phase = 0;
+    tile_partial(maps, D, q, knew, vnew, t, hk, ti, T, part == 0 && t >= T.y0 && t < T.y0 + T.nv, sm, phase);
+    __threadfence();
+    __syncthreads();
+    unsigned* ctr = D.counters + (2 + part) * D.Hkv + hk;
+    const int nblocks = part == 0 ? nst + nwt : nut;
+    if (tid == 0) *is_last = atomicAdd(ctr, 1u) == (unsigned)(nblocks - 1);
+    __syncthreads();
+    if (*is_last) {
+        __threadfence();
+        merge_part(D, hk, part, nst, nut, nwt, kk, sm, out);
+        if (tid == 0) *ctr = 0u;  // re-armed for the next step
+    }
+    if (part == 0) pdl_hold();
+}
+
+// ---- one decode step in one cooperative launch ------------------------------------------------
+
+// Per-step arguments of k_decode_step.
+struct StepArgs {
+    const __nv_bfloat16* q;
+    const __nv_bfloat16* k;
+    const __nv_bfloat16* v;
+    __nv_bfloat16* out;
+    int64_t t, B;
+    unsigned long long qbase;  // value of the context's work counter when this step's items start
+    int kk, nm, nst, nwt, nut;  // selected units, eligible units, sink / window / unit tiles per head
+    int upi, n_split;           // units per scoring item, scoring items per head
+    int mode, tag;              // scoring operand; this step's flag value (> every earlier step's)
+};
+
+// Bounded wait (one thread) for a flag another CTA of this grid sets to `tag` with a release store.
+__device__ __forceinline__ bool wait_flag(const Dev& D, const int* flag, int tag) {
+    if (ld_acquire(flag) == tag) return true;
+    const long long t0 = clock64();
+    while (ld_acquire(flag) != tag) {
+        if (clock64() - t0 > (1ll << 32)) {  // ~2 s: something is broken; give up cleanly
+            set_err(D, ERR_TIMEOUT);
+            return false;
+        }
+        __nanosleep(100);
+    }
+    return true;
+}
+
+// Unit scores of units [split * upi, ...) of KV head hk (rows of ROWB bytes of E elements) by the
+// CTA's four warps: the same arithmetic and lane mapping as the streaming scoring kernel of the
+// lookup (a warp takes 4 units per step for 512- and 1024-byte rows, 8 units for 256-byte rows;
+// consecutive lanes load consecutive 16 bytes), then the CTA's top-32 list, and the head's selection
+// by its last scoring item, published on the head's selection flag.
+template <typename E, int ROWB>
+__device__ void score_item(const Dev& D, const StepArgs& A, int hk, int split, uint8_t* sm) {
+    float* qb = reinterpret_cast<float*>(sm + OFF_Q);                               // [128]
+    auto lists = reinterpret_cast<uint64_t(*)[32]>(sm + OFF_Q + 512);            // [4][32]
+    constexpr int V = 16 / sizeof(E);
+    constexpr int HALFROW = ROWB == 256;
+    constexpr int CPL = HALFROW ? 1 : ROWB / 512;
+    constexpr int UB = HALFROW ? 8 : 4;  // units per warp step
+    constexpr int GRP = 32 / (HALFROW ? 8 : 4);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int u_begin = split * A.upi, u_end = min(A.nm, u_begin + A.upi);
+    const uint4* base = A.mode == OP_REPS
+        ? reinterpret_cast<const uint4*>((const __nv_bfloat16*)D.rep_keys + (int64_t)hk * D.units_max * D.r * D.d)
+        : A.mode == OP_REPSUM ? reinterpret_cast<const uint4*>(D.repsum + (int64_t)hk * D.units_max * D.d)
+                              : reinterpret_cast<const uint4*>((const __nv_bfloat16*)D.meankey + (int64_t)hk * D.units_max * D.d);
+    const int half = lane >> 4, piece = lane & 15;
+    uint4 raw[4][CPL];
+    auto load = [&](int u0) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) {
+                const int u = HALFROW ? u0 + 2 * i + half : u0 + i;
+                raw[i][c] = u < u_end ? __ldg(HALFROW ? base + (int64_t)u * 16 + piece : base + (int64_t)u * 32 * CPL + c * 32 + lane)
+                                      : make_uint4(0, 0, 0, 0);
+            }
+    };
+    load(u_begin + warp * UB);  // requested before the query sum, which it does not need
+    __syncthreads();            // the previous item's use of qb and lists is over
+    if (tid < DHD / 2) {        // R(W) (sum of the group's q heads)
+        float a = 0.f, b = 0.f;
+        for (int h = 0; h < D.G; ++h) {
+            a += __bfloat162float(A.q[(hk * D.G + h) * DHD + tid]);
+            b += __bfloat162float(A.q[(hk * D.G + h) * DHD + tid + DHD / 2]);
+        }
+        const float2 cw = D.cs_W[tid];
+        qb[tid] = a * cw.x - b * cw.y;
+        qb[tid + DHD / 2] = b * cw.x + a * cw.y;
     }
     __syncthreads();
-    float M = -INFINITY;
-    for (int s = 0; s < NT; ++s) M = fmaxf(M, ml[0][s]);
-    float L = 0.f, O = 0.f;
-    float acc[MERGE_BATCH];
+    float qr[V];
+    {
+        const int i0 = ((HALFROW ? piece : lane) * V) % DHD;
 #pragma unroll
-    for (int u = 0; u < MERGE_BATCH; ++u) {
-        const int s = z + MERGE_SLICES * u;
-        acc[u] = s < NT ? base[s * stride + 2 + dim] : 0.f;
+        for (int x = 0; x < V; ++x) qr[x] = qb[i0 + x];
     }
+    uint64_t list = 0, cand = 0;
+    int it = 0;
+    for (int u0 = u_begin + warp * UB; u0 < u_end; u0 += 4 * UB, ++it) {  // warp-uniform
+        if (it > 0) load(u0);
+        float acc[4];
 #pragma unroll
-    for (int u = 0; u < MERGE_BATCH; ++u) {
-        const int s = z + MERGE_SLICES * u;
-        if (s < NT) {
-            const float m = ml[0][s];
-            const float w = m == -INFINITY ? 0.f : expf(m - M);
-            L += w * ml[1][s];
-            O += w * acc[u];
+        for (int i = 0; i < 4; ++i) {
+            float a = 0.f;
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) {
+                if (sizeof(E) == 2) {
+                    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw[i][c]);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 f = __bfloat1622float2(h2[e]);
+                        a += f.x * qr[2 * e] + f.y * qr[2 * e + 1];
+                    }
+                } else {
+                    const float* f = reinterpret_cast<const float*>(&raw[i][c]);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) a += f[e] * qr[e];
+                }
+            }
+            acc[i] = a;
+        }
+        // halving steps then a butterfly: full rows -- masks 16, 8 then 4, 2, 1 (lane l: unit l / 8);
+        // half rows -- masks 8, 4 then 2, 1 inside each half (lane l: unit 2 ((l / 4) % 4) + l / 16)
+#pragma unroll
+        for (int m = HALFROW ? 8 : 16, nv = 4; nv > 1; m >>= 1, nv >>= 1) {
+            const bool upper = (lane & m) != 0;
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                if (i < nv / 2) {
+                    const float send = upper ? acc[i] : acc[i + nv / 2];
+                    const float keep = upper ? acc[i + nv / 2] : acc[i];
+                    acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+                }
+            }
+        }
+#pragma unroll
+        for (int m = HALFROW ? 2 : 4; m >= 1; m >>= 1) acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], m);
+        const int j = HALFROW ? u0 + 2 * ((lane >> 2) & 3) + half : u0 + lane / 8;
+        const int sub = HALFROW ? (lane & 3) : (lane & 7);
+        const float sc = acc[0] * D.inv_sqrt_d;
+        if (j < u_end) {
+            if (sub == 0) D.uscore[(int64_t)hk * D.units_max + j] = sc;
+            if (sub == it % GRP) cand = make_key(sc, (uint32_t)j);
+        }
+        if (it % GRP == GRP - 1) {
+            list = warp_topk_insert(list, cand);
+            cand = 0;
         }
     }
-    red[0][z][dim] = L;
-    red[1][z][dim] = O;
+    if (__any_sync(0xffffffffu, cand != 0)) list = warp_topk_insert(list, cand);
+    lists[warp][lane] = list;
+    for (int stride = 1; stride < 4; stride *= 2) {
+        __syncthreads();
+        if ((warp % (2 * stride)) == 0 && warp + stride < 4)
+            lists[warp][lane] = warp_merge_desc(lists[warp][lane], lists[warp + stride][lane]);
+    }
     __syncthreads();
-    if (z == 0) {
-        float Lt = 0.f, Ot = 0.f;
-        for (int q = 0; q < MERGE_SLICES; ++q) {
-            Lt += red[0][q][dim];
-            Ot += red[1][q][dim];
+    publish_and_select(D, hk, split, A.nm, A.n_split, lists, 4, D.dflags + hk, A.tag);
+}
+
+// A whole decode step in one cooperative launch: every CTA is resident at once, and takes work items
+// from the context's counter until none is left.  The items, in order:
+//   the sink and window tiles of every KV head (the tile holding token t stores it first); the
+//     head's last one merges them and publishes the merge on the head's window flag;
+//   the scoring items (upi units of one head each); the head's last one selects its top-k and
+//     publishes the selection on the head's selection flag;
+//   the selected units' tiles; each waits (bounded) for its head's selection; the head's last one
+//     waits (bounded) for the window flag and merges everything into the output.
+// Only items after every non-waiting item wait, and every CTA is resident, so every wait ends.
+template <typename E, int ROWB>
+__global__ void __launch_bounds__(DTHREADS) k_decode_step(const __grid_constant__ TcMaps maps, Dev D, StepArgs A) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + OFF_MISC);
+    float2* cs_t = reinterpret_cast<float2*>(sm + OFF_CS);
+    __shared__ int item_s, flag_s;
+    const int tid = threadIdx.x;
+    if (tid == 0) {
+        ptx::mbar_init(bar, 1);
+        ptx::mbar_fence_init();
+    }
+    for (int i = tid; i < DHD / 2; i += DTHREADS) cs_t[i] = cs_abs(D.cs_abs3, D.half, A.t, i);
+    __syncthreads();
+    const int per_w = A.nst + A.nwt;
+    const int NW = per_w * D.Hkv, NS = A.n_split * D.Hkv * (A.kk > 0), NU = A.nut * D.Hkv;
+    const int total = NW + NS + NU;
+    uint32_t phase = 0;
+    for (;;) {
+        if (tid == 0) item_s = (int)(atomicAdd(D.dq, 1ull) - A.qbase);
+        __syncthreads();
+        const int item = item_s;
+        __syncthreads();
+        if (item >= total) break;
+        if (item < NS + NW && item >= NW) {  // scoring
+            const int it = item - NW;
+            score_item<E, ROWB>(D, A, it / A.n_split, it % A.n_split, sm);
+            continue;
         }
-        out[(int64_t)(hk * G + h) * d + dim] = __float2bfloat16_rn(Ot / Lt);
+        int hk, ti, part;
+        if (item < NW) {
+            hk = item / per_w;
+            const int wi = item % per_w;
+            ti = wi < A.nst ? wi : wi + A.nut;
+            part = 0;
+        } else {
+            const int it = item - NW - NS;
+            hk = it / A.nut;
+            ti = A.nst + it % A.nut;
+            part = 1;
+            if (tid == 0) flag_s = wait_flag(D, D.dflags + hk, A.tag);  // the head's selection
+            __syncthreads();
+        }
+        const bool ok_sel = part == 0 || flag_s;
+        const DTile T = ok_sel ? decode_tile(D, hk, ti, A.t, A.kk, A.B) : DTile{1, 0, 0};
+        tile_partial(maps, D, A.q, A.k, A.v, A.t, hk, ti, T, part == 0 && A.t >= T.y0 && A.t < T.y0 + T.nv, sm,
+                     phase);
+        __threadfence();
+        __syncthreads();
+        unsigned* ctr = D.counters + (2 + part) * D.Hkv + hk;
+        const int nblocks = part == 0 ? per_w : A.nut;
+        if (tid == 0) item_s = atomicAdd(ctr, 1u) == (unsigned)(nblocks - 1);
+        __syncthreads();
+        if (!item_s) continue;
+        __threadfence();
+        if (part == 1) {  // part 0's merged slot must be complete
+            if (tid == 0) flag_s = wait_flag(D, D.dflags + D.Hkv + hk, A.tag);
+            __syncthreads();
+        }
+        merge_part(D, hk, part, A.nst, A.nut, A.nwt, A.kk, sm, A.out);
+        if (part == 0 && A.kk > 0) {  // publish the merged sinks and window
+            __threadfence();
+            __syncthreads();
+            if (tid == 0) st_release(D.dflags + D.Hkv + hk, A.tag);
+        }
+        if (tid == 0) *ctr = 0u;  // re-armed for the next step
+        __syncthreads();
     }
 }
 
@@ -359,31 +684,96 @@ __global__ void __launch_bounds__(MERGE_SLICES * DHD) k_decode_merge(Dev D, __nv
 
 bool decode_tc_supported(const Dev& D) { return D.d == DHD && D.G <= MAXG && D.topk <= 32; }
 
-cudaError_t launch_decode_append(const Dev& D, const void* q, const void* k, const void* v, int64_t t,
-                                 cudaStream_t st, bool pdl) {
-    return launch_k(k_decode_append, dim3(D.Hkv), dim3(DTHREADS), 0, st, pdl, D, (const __nv_bfloat16*)q,
-                    (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, t);
-}
-
-cudaError_t launch_decode_tc(const Dev& D, const void* q, int64_t t, int kk, int64_t B, int part, cudaStream_t st,
-                             const void* tmaps, bool pdl) {
+cudaError_t launch_decode_tc(const Dev& D, const void* q, const void* k, const void* v, int64_t t, int kk, int64_t B,
+                             int part, void* out, cudaStream_t st, const void* tmaps, bool pdl) {
     const int S_eff = (int)(D.S < t + 1 ? D.S : t + 1);
     const int64_t win = t - B + 1;
     const int nst = (S_eff + DK - 1) / DK, nut = kk * ((D.U + DK - 1) / DK), nwt = (int)((win + DK - 1) / DK);
-    if (nst + nut + nwt > D.dec_splits_max || nst + nut + nwt > MERGE_SLICES * MERGE_BATCH) return cudaErrorInvalidValue;
+    if (nst + nut + nwt + 1 > D.dec_splits_max) return cudaErrorInvalidValue;  // + the merged slot
     const int tiles = part == 1 ? nut : nst + nwt;
     if (tiles == 0) return cudaSuccess;
     static std::atomic<unsigned long long> attr_done{0};
     cudaError_t e = smem_limit_once(k_decode_attn, DSMEM, attr_done);
     if (e != cudaSuccess) return e;
     return launch_k(k_decode_attn, dim3(tiles, D.Hkv), dim3(DTHREADS), DSMEM, st, pdl,
-                    *reinterpret_cast<const TcMaps*>(tmaps), D, (const __nv_bfloat16*)q, t, kk, B, part);
+                    *reinterpret_cast<const TcMaps*>(tmaps), D, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
+                    (const __nv_bfloat16*)v, t, kk, B, part, (__nv_bfloat16*)out);
 }
 
-cudaError_t launch_decode_merge(const Dev& D, int64_t t, int kk, int64_t B, void* out, cudaStream_t st, bool pdl) {
-    const int S_eff = (int)(D.S < t + 1 ? D.S : t + 1);
-    const int NT = (S_eff + DK - 1) / DK + kk * ((D.U + DK - 1) / DK) + (int)((t - B + 1 + DK - 1) / DK);
-    return launch_k(k_decode_merge, dim3(D.G, D.Hkv), dim3(MERGE_SLICES * DHD), 0, st, pdl, D, (__nv_bfloat16*)out, NT);
+template <typename E, int ROWB>
+static cudaError_t launch_step(const Dev& D, const StepArgs& A, int grid, cudaStream_t st, const void* tmaps) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(DTHREADS);
+    cfg.dynamicSmemBytes = DSMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k_decode_step<E, ROWB>, *reinterpret_cast<const TcMaps*>(tmaps), D, A);
+}
+
+// Resident CTAs of k_decode_step<E, ROWB> on the current device (the cooperative grid size).
+template <typename E, int ROWB>
+static int step_grid(cudaError_t* err) {
+    static std::atomic<unsigned long long> attr_done{0};
+    *err = smem_limit_once(k_decode_step<E, ROWB>, DSMEM, attr_done);
+    if (*err != cudaSuccess) return 0;
+    int dev = 0, sms = 0, per_sm = 0;
+    if ((*err = cudaGetDevice(&dev)) != cudaSuccess) return 0;
+    if ((*err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return 0;
+    if ((*err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_decode_step<E, ROWB>, DTHREADS, DSMEM)) !=
+        cudaSuccess)
+        return 0;
+    return per_sm * sms;
+}
+
+cudaError_t launch_decode_step(const Dev& D, const void* q, const void* k, const void* v, int64_t t, int kk, int64_t B,
+                               int nm, int score_mode, int tag, unsigned long long qbase, void* out, cudaStream_t st,
+                               const void* tmaps, unsigned long long* consumed) {
+    StepArgs A;
+    A.q = (const __nv_bfloat16*)q;
+    A.k = (const __nv_bfloat16*)k;
+    A.v = (const __nv_bfloat16*)v;
+    A.out = (__nv_bfloat16*)out;
+    A.t = t;
+    A.B = B;
+    A.qbase = qbase;
+    A.kk = kk;
+    A.nm = nm;
+    A.nst = (int)((std::min<int64_t>(D.S, t + 1) + DK - 1) / DK);
+    A.nwt = (int)((t - B + 1 + DK - 1) / DK);
+    A.nut = kk * ((D.U + DK - 1) / DK);
+    A.mode = score_mode;
+    A.tag = tag;
+    if (A.nst + A.nut + A.nwt + 1 > D.dec_splits_max) return cudaErrorInvalidValue;  // + the merged slot
+    const int row_bytes = score_mode == OP_REPS ? D.r * D.d * 2 : score_mode == OP_REPSUM ? D.d * 4 : D.d * 2;
+    cudaError_t err = cudaSuccess;
+    int grid = 0;
+    switch (row_bytes) {
+        case 1024: grid = step_grid<__nv_bfloat16, 1024>(&err); break;
+        case 512: grid = score_mode == OP_REPSUM ? step_grid<float, 512>(&err) : step_grid<__nv_bfloat16, 512>(&err); break;
+        case 256: grid = step_grid<__nv_bfloat16, 256>(&err); break;
+        default: return cudaErrorInvalidValue;
+    }
+    if (err != cudaSuccess) return err;
+    if (grid <= 0) return cudaErrorInvalidConfiguration;
+    // about two scoring items per resident CTA; a multiple of what the four warps take per step
+    const int step_units = row_bytes == 256 ? 32 : 16;
+    const int64_t want = ((int64_t)nm * D.Hkv + 2 * grid - 1) / (2 * grid);
+    A.upi = (int)std::max<int64_t>(step_units, (want + step_units - 1) / step_units * step_units);
+    A.n_split = kk > 0 ? (nm + A.upi - 1) / A.upi : 0;
+    if (A.n_split > D.score_splits_max) return cudaErrorInvalidValue;
+    const int total = (A.nst + A.nwt) * D.Hkv + A.n_split * D.Hkv + A.nut * D.Hkv;
+    *consumed = (unsigned long long)total + (unsigned long long)grid;  // every CTA's last take overshoots once
+    switch (row_bytes) {
+        case 1024: return launch_step<__nv_bfloat16, 1024>(D, A, grid, st, tmaps);
+        case 512: return score_mode == OP_REPSUM ? launch_step<float, 512>(D, A, grid, st, tmaps)
+                                                 : launch_step<__nv_bfloat16, 512>(D, A, grid, st, tmaps);
+        default: return launch_step<__nv_bfloat16, 256>(D, A, grid, st, tmaps);
+    }
 }
 
 }  // namespace infllm

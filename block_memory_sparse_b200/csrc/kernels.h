@@ -46,15 +46,17 @@ cudaError_t launch_decode(const Dev& D, const void* q, int64_t t, int kk, int64_
 
 int decode_split_keys(int elt_bytes);
 
-// Decode on the TMA path (bf16, head dim 128, G <= 8): store the token, split-KV attention over
-// 128-key tiles (sinks and window alongside the lookup, the selected units after it), then a
-// log-sum-exp merge.
+// Decode on the TMA path (bf16, head dim 128, G <= 8): split-KV attention over 128-key tiles.
+// part 0: the sink and window tiles; stores the token (k, v, its query block sum) and merges the
+//         tiles' partials (into the output when kk == 0); runs alongside the lookup.
+// part 1: the selected units' tiles, then the merge with part 0's partial into `out`.
 bool decode_tc_supported(const Dev& D);
-cudaError_t launch_decode_append(const Dev& D, const void* q, const void* k, const void* v, int64_t t, cudaStream_t st,
-                                 bool pdl);
-// part 0: sink and window tiles (no selection needed); part 1: the selected units' tiles.
-cudaError_t launch_decode_tc(const Dev& D, const void* q, int64_t t, int kk, int64_t B, int part, cudaStream_t st,
-                             const void* tmaps, bool pdl);
-cudaError_t launch_decode_merge(const Dev& D, int64_t t, int kk, int64_t B, void* out, cudaStream_t st, bool pdl);
+cudaError_t launch_decode_tc(const Dev& D, const void* q, const void* k, const void* v, int64_t t, int kk, int64_t B,
+                             int part, void* out, cudaStream_t st, const void* tmaps, bool pdl);
+// The whole decode step in one cooperative launch (k_decode_step); *consumed receives how far the
+// step advances the context's work counter.
+cudaError_t launch_decode_step(const Dev& D, const void* q, const void* k, const void* v, int64_t t, int kk, int64_t B,
+                               int nm, int score_mode, int tag, unsigned long long qbase, void* out, cudaStream_t st,
+                               const void* tmaps, unsigned long long* consumed);
 
 }  // namespace infllm

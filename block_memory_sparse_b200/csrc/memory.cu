@@ -125,7 +125,9 @@ __global__ void __launch_bounds__(1024) k_ysum(Dev D, const T* __restrict__ q, i
     pdl_hold();
 }
 
-// Representatives of units [j0, j0 + gridDim.x) for kv head blockIdx.y, 256 threads.
+// Representatives of units [j0, j0 + gridDim.x) for kv head blockIdx.y, 256 threads.  Also the
+// unit's mean key (the mean-of-keys representation of "InfLLM: Training-Free Long-Context
+// Extrapolation ..." (research-map summary), "Measured effects", ablation row on mean key vectors).
 //   Qt = sum_{i=e}^{e+W-1} sum_h R(i - e) q_{i,h}  (from the block sums, e = unit end)
 //   rho_m = <R(e - m) Qt, k_m> / sqrt(d)  ==  sum_i sum_h <R(i) q_{i,h}, R(m) k_m> / sqrt(d)
 // then the top r by (rho desc, m asc), stored ascending, plus the raw rep keys and their sum.
@@ -262,6 +264,20 @@ __global__ void __launch_bounds__(256) k_reps(Dev D, int64_t j0) {
                 }
         }
         rs[i] = s;
+    }
+    // the unit's mean key: the sum of its U keys in fp64 (exact for bf16 keys), divided by U, rounded
+    // once to the context dtype
+    T* mk = (T*)D.meankey + ((int64_t)hk * D.units_max + j) * D.d;
+    for (int i = threadIdx.x; i < D.d; i += blockDim.x) {
+        double s = 0.0;
+        for (int m0b = 0; m0b < D.U; m0b += 8) {
+            T x[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) x[u] = m0b + u < D.U ? K[(int64_t)(m0b + u) * D.d + i] : from_f<T>(0.f);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) s += (double)to_f(x[u]);
+        }
+        mk[i] = from_d<T>(s / (double)D.U);
     }
     pdl_hold();
 }

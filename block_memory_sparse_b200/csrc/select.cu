@@ -9,9 +9,12 @@
 //   sigma_j = <R(W) sum_t sum_h q_{t,h}, sum_m k_{j,m}> / sqrt(d)
 // which is linear, so the queries are summed first (prep kernel) and each unit costs one
 // read of its representative keys (REPS mode) or of their fp32 sum (REPSUM mode).
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "tc_maps.cuh"
+#include "topk.cuh"
 
 namespace infllm {
 
@@ -128,68 +131,6 @@ template <> struct Vec16<float> {
     }
 };
 
-// Top-k of one KV head from the scoring CTAs' top-32 lists (composite keys, descending), run by
-// the last scoring CTA of that head: warp w merges lists w, w + nw, ... (loads of a batch issued
-// together), then the warp lists are merged pairwise in shared memory; the k ids are written in
-// ascending order.  Ties go to the lower unit index.  Valid for k <= 32.
-__device__ void merge_select(const Dev& D, int hk, int n_mem, int n_split, uint64_t (*lists)[32], int nw) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const uint64_t* cb = D.cand + (int64_t)hk * D.score_splits_max * 32 + lane;
-    uint64_t m = 0;
-    for (int s0 = warp; s0 < n_split; s0 += nw * 4) {
-        uint64_t b[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int sp = s0 + nw * u;
-            b[u] = sp < n_split ? __ldcg(cb + (int64_t)sp * 32) : 0ull;
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-            if (s0 + nw * u < n_split) m = warp_merge_desc(m, b[u]);
-    }
-    __syncthreads();  // the caller's use of lists[] is over
-    lists[warp][lane] = m;
-    for (int stride = 1; stride < nw; stride *= 2) {
-        __syncthreads();
-        if ((warp % (2 * stride)) == 0 && warp + stride < nw)
-            lists[warp][lane] = warp_merge_desc(lists[warp][lane], lists[warp + stride][lane]);
-    }
-    __syncthreads();
-    if (warp == 0) {
-        const int kk = min(D.topk, n_mem);
-        uint64_t sk = (lane < kk) ? (uint64_t)(0xffffffffu - key_index(lists[0][lane])) : 0ull;
-        sk = warp_sort_desc(sk);  // ascending ids
-        if (lane < D.topk) {
-            int o = -1;
-            if (lane < kk) {
-                o = (int)(0xffffffffu - (uint32_t)sk);
-                if (o < 0 || o >= n_mem) {
-                    set_err(D, ERR_SEL_RANGE);
-                    o = 0;
-                }
-            }
-            D.sel[hk * D.topk + lane] = o;
-        }
-    }
-}
-
-// This CTA's top-32 list of KV head hk goes to D.cand; the last CTA of the head to finish (device
-// counter, threadfence pattern: no CTA waits for another) merges all lists into the selection and
-// re-arms the counter for the next launch.
-__device__ void publish_and_select(const Dev& D, int hk, int split, int n_mem, int n_split, uint64_t (*lists)[32],
-                                   int nw) {
-    __shared__ int is_last;
-    if (threadIdx.x < 32) D.cand[((int64_t)hk * D.score_splits_max + split) * 32 + threadIdx.x] = lists[0][threadIdx.x];
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) is_last = atomicAdd(&D.counters[hk], 1u) == (unsigned)(n_split - 1);
-    __syncthreads();
-    if (!is_last) return;
-    __threadfence();
-    merge_select(D, hk, n_mem, n_split, lists, nw);
-    if (threadIdx.x == 0) D.counters[hk] = 0u;
-}
-
 // Grid (n_split, Hkv), 512 threads.  Each unit is scored by a group of LPU lanes that split
 // its operand (16-byte loads issued in batches of 8), reduced inside the group; PER = 512 / LPU
 // units per CTA.  Writes the unit scores and, with do_select, the top-k (last CTA per head).
@@ -254,26 +195,27 @@ __global__ void __launch_bounds__(SC_THREADS, 2) k_score_topk(Dev D, int n_mem, 
     float acc = 0.f;
     if (j < n_mem) {
         // 16-byte vectors kept raw in registers (8 per batch), converted at use
-        const T* p = MODE == 0 ? (const T*)D.rep_keys + ((int64_t)hk * D.units_max + j) * D.r * D.d
-                               : nullptr;
-        const float* pf = MODE == 0 ? nullptr : D.repsum + ((int64_t)hk * D.units_max + j) * D.d;
-        constexpr int N = MODE == 0 ? Vec16<T>::N : 4;  // elements per vector
-        const int total = MODE == 0 ? D.r * D.d : D.d;
+        const T* p = MODE == OP_REPS ? (const T*)D.rep_keys + ((int64_t)hk * D.units_max + j) * D.r * D.d
+                   : MODE == OP_MEANKEY ? (const T*)D.meankey + ((int64_t)hk * D.units_max + j) * D.d
+                                        : nullptr;
+        const float* pf = MODE == OP_REPSUM ? D.repsum + ((int64_t)hk * D.units_max + j) * D.d : nullptr;
+        constexpr int N = MODE != OP_REPSUM ? Vec16<T>::N : 4;  // elements per vector
+        const int total = MODE == OP_REPS ? D.r * D.d : D.d;
         for (int e0 = sub * N; e0 < total; e0 += 8 * LPU * N) {
             uint4 raw[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 const int e = e0 + u * LPU * N;
                 if (e < total)
-                    raw[u] = MODE == 0 ? __ldg(reinterpret_cast<const uint4*>(p + e))
-                                       : __ldg(reinterpret_cast<const uint4*>(pf + e));
+                    raw[u] = MODE != OP_REPSUM ? __ldg(reinterpret_cast<const uint4*>(p + e))
+                                               : __ldg(reinterpret_cast<const uint4*>(pf + e));
             }
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 const int e = e0 + u * LPU * N;
                 if (e < total) {
                     const int i0 = e % D.d;
-                    if (MODE == 0 && sizeof(T) == 2) {
+                    if (MODE != OP_REPSUM && sizeof(T) == 2) {
                         const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw[u]);
 #pragma unroll
                         for (int c = 0; c < 4; ++c) {
@@ -349,6 +291,33 @@ __device__ __forceinline__ void rotated_query_sum(const Dev& D, int hk, int n_qt
     }
 }
 
+// Dot products of one 16-byte piece of an operand row (E = bf16 or fp32 elements) with V query values.
+template <typename E>
+__device__ __forceinline__ float dot16(const uint4& raw, const float* qr) {
+    float a = 0.f;
+    if (sizeof(E) == 2) {
+        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(h2[e]);
+            a += f.x * qr[2 * e] + f.y * qr[2 * e + 1];
+        }
+    } else {
+        const float* f = reinterpret_cast<const float*>(&raw);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) a += f[e] * qr[e];
+    }
+    return a;
+}
+
+// The scoring operand of KV head hk: representative keys, their fp32 sum, or the mean key.
+template <typename T>
+__device__ __forceinline__ const uint4* score_operand(const Dev& D, int mode, int hk) {
+    if (mode == OP_REPS) return reinterpret_cast<const uint4*>((const T*)D.rep_keys + (int64_t)hk * D.units_max * D.r * D.d);
+    if (mode == OP_REPSUM) return reinterpret_cast<const uint4*>(D.repsum + (int64_t)hk * D.units_max * D.d);
+    return reinterpret_cast<const uint4*>((const T*)D.meankey + (int64_t)hk * D.units_max * D.d);
+}
+
 // One stage of the scoring pipeline: UB units' operand rows (C 16-byte chunks per lane each).
 template <int UB, int C>
 __device__ __forceinline__ void load_units(uint4 (&r)[UB][C], const uint4* base, int ub, int valid, int lane) {
@@ -365,7 +334,7 @@ __device__ __forceinline__ void dot_units(const uint4 (&r)[UB][C], const float (
         float a = 0.f;
 #pragma unroll
         for (int k = 0; k < C; ++k) {
-            if (MODE == 0 && sizeof(T) == 2) {
+            if (MODE != OP_REPSUM && sizeof(T) == 2) {
                 const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&r[u][k]);
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
@@ -397,12 +366,10 @@ __global__ void __launch_bounds__(256, 2) k_score_wpu(Dev D, int n_mem, int n_sp
     if (wait_first) pdl_wait();  // as in k_score_topk
     pdl_trigger();
     const int split = blockIdx.x, hk = blockIdx.y;
-    constexpr int V = MODE == 0 ? (int)(16 / sizeof(T)) : 4;  // elements per 16-byte chunk
+    constexpr int V = MODE != OP_REPSUM ? (int)(16 / sizeof(T)) : 4;  // elements per 16-byte chunk
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
     const int u0 = (split * nw + warp) * 32;
-    const uint4* base = MODE == 0
-        ? reinterpret_cast<const uint4*>((const T*)D.rep_keys + ((int64_t)hk * D.units_max + u0) * D.r * D.d)
-        : reinterpret_cast<const uint4*>(D.repsum + ((int64_t)hk * D.units_max + u0) * D.d);
+    const uint4* base = score_operand<T>(D, MODE, hk) + (int64_t)u0 * 32 * C;
     // two register stages of UB units: the loads of one stage are in flight while the other is
     // multiplied; the first stage is issued before the query sum, which it does not need
     constexpr int UB = C >= 4 ? 2 : 4;
@@ -456,6 +423,184 @@ __global__ void __launch_bounds__(256, 2) k_score_wpu(Dev D, int n_mem, int n_sp
         publish_and_select(D, hk, split, n_mem, n_split, lists, nw);
     }
     if (!wait_first) pdl_hold();  // this grid must not complete before its predecessor (see k_score_topk)
+}
+
+// The CTA's top-32 candidate list from its warps' lists, then the head's selection (last CTA).
+__device__ __forceinline__ void cta_lists_and_select(const Dev& D, int hk, int split, int n_mem, int n_split,
+                                                     uint64_t (*lists)[32], uint64_t list) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    lists[warp][lane] = list;
+    for (int stride = 1; stride < nw; stride *= 2) {
+        __syncthreads();
+        if ((warp % (2 * stride)) == 0 && warp + stride < nw)
+            lists[warp][lane] = warp_merge_desc(lists[warp][lane], lists[warp + stride][lane]);
+    }
+    __syncthreads();
+    publish_and_select(D, hk, split, n_mem, n_split, lists, nw);
+}
+
+// Streaming scoring for one query token (decode), the bandwidth-bound read of the whole scoring
+// pool.  Grid (n_split, Hkv), 256 threads; CTA s scores units [s * upc, s * upc + upc) of KV head
+// hk; every unit's operand row is 32 * CPL 16-byte pieces of E elements.  Each warp takes UB
+// consecutive units per step: lane l loads the pieces l, l + 32, ... (CPL per unit) of every
+// unit's row -- consecutive lanes on consecutive 16 bytes, so each load instruction reads 512
+// contiguous bytes -- and multiplies them with its slice of the rotated query sum, held in
+// registers (every piece of a lane covers the same dims, since 32 pieces span a whole number of
+// d-element rows).  The UB partial sums are transposed across the warp (log2(UB) halving steps)
+// and then summed over the 32/UB lanes that share a unit, which leaves the unit's score in each of
+// those lanes.  The warp keeps a running top-32 list (one candidate per lane every 32/UB steps);
+// the CTA's list and the head's selection follow as in k_score_wpu.
+template <typename T, typename E, int CPL, int UB>
+__global__ void __launch_bounds__(256) k_score_dec(Dev D, int mode, int n_mem, int upc, int n_split, const T* qraw,
+                                                   int wait_first) {
+    __shared__ float qb[128];
+    __shared__ uint64_t lists[8][32];
+    if (wait_first) pdl_wait();  // new representatives come from the kernels before
+    pdl_trigger();
+    constexpr int V = 16 / sizeof(E);  // elements per 16-byte piece
+    constexpr int GRP = 32 / UB;       // lanes that end with one unit's score
+    const int split = blockIdx.x, hk = blockIdx.y;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    const int u_begin = split * upc, u_end = min(n_mem, u_begin + upc);
+    const uint4* base = score_operand<T>(D, mode, hk);
+    // the first step's rows are requested before the query sum, which they do not need
+    uint4 raw[UB][CPL];
+    auto load = [&](int u0) {
+#pragma unroll
+        for (int u = 0; u < UB; ++u)
+#pragma unroll
+            for (int c = 0; c < CPL; ++c)
+                raw[u][c] = u0 + u < u_end ? __ldg(base + (int64_t)(u0 + u) * 32 * CPL + c * 32 + lane)
+                                           : make_uint4(0, 0, 0, 0);
+    };
+    load(u_begin + warp * UB);
+    rotated_query_sum<T>(D, hk, 1, qraw, qb);
+    __syncthreads();
+    float qr[V];
+    {
+        const int i0 = (lane * V) % D.d;
+#pragma unroll
+        for (int v = 0; v < V; ++v) qr[v] = qb[i0 + v];
+    }
+    uint64_t list = 0, cand = 0;
+    int it = 0;
+    for (int u0 = u_begin + warp * UB; u0 < u_end; u0 += nw * UB, ++it) {  // warp-uniform
+        if (it > 0) load(u0);
+        float acc[UB];
+#pragma unroll
+        for (int u = 0; u < UB; ++u) {
+            float a = 0.f;
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) a += dot16<E>(raw[u][c], qr);
+            acc[u] = a;
+        }
+        // transpose: after the halving steps (masks 16 .. GRP) lane l holds unit l / GRP's partial,
+        // then the butterfly over the GRP lanes of a unit completes it in each of them
+#pragma unroll
+        for (int m = 16, nv = UB; m >= 1; m >>= 1) {
+            if (nv > 1) {
+                const bool upper = (lane & m) != 0;
+#pragma unroll
+                for (int i = 0; i < UB / 2; ++i) {
+                    if (i < nv / 2) {
+                        const float send = upper ? acc[i] : acc[i + nv / 2];
+                        const float keep = upper ? acc[i + nv / 2] : acc[i];
+                        acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+                    }
+                }
+                nv >>= 1;
+            } else {
+                acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], m);
+            }
+        }
+        const int j = u0 + lane / GRP;
+        const float sc = acc[0] * D.inv_sqrt_d;
+        if (j < u_end) {
+            if ((lane % GRP) == 0) D.uscore[(int64_t)hk * D.units_max + j] = sc;
+            if ((lane % GRP) == (it % GRP)) cand = make_key(sc, (uint32_t)j);
+        }
+        if ((it % GRP) == GRP - 1) {
+            list = warp_topk_insert(list, cand);
+            cand = 0;
+        }
+    }
+    if (__any_sync(0xffffffffu, cand != 0)) list = warp_topk_insert(list, cand);
+    cta_lists_and_select(D, hk, split, n_mem, n_split, lists, list);
+    if (!wait_first) pdl_hold();  // this grid must not complete before its predecessor (see k_score_topk)
+}
+
+// The same for operand rows of 256 bytes (16 pieces: one bf16 mean key of d = 128, or an fp32 row of
+// d = 64): each load instruction covers two units (lane l: unit l / 16, piece l % 16), four
+// instructions per step, so a warp scores 8 units per step.  The four partials of a lane are
+// transposed within its half-warp (masks 8 and 4) and summed over the 4 lanes left per unit
+// (masks 2 and 1): lanes l with the same l / 4 then hold the score of unit u0 + 2 ((l / 4) % 4) + l / 16.
+template <typename T, typename E>
+__global__ void __launch_bounds__(256) k_score_dec_half(Dev D, int mode, int n_mem, int upc, int n_split,
+                                                        const T* qraw, int wait_first) {
+    __shared__ float qb[128];
+    __shared__ uint64_t lists[8][32];
+    if (wait_first) pdl_wait();
+    pdl_trigger();
+    constexpr int V = 16 / sizeof(E);
+    const int split = blockIdx.x, hk = blockIdx.y;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    const int u_begin = split * upc, u_end = min(n_mem, u_begin + upc);
+    const uint4* base = score_operand<T>(D, mode, hk);
+    const int half = lane >> 4, piece = lane & 15;
+    const int slot = (lane >> 2) & 3;
+    // the first step's rows are requested before the query sum, which they do not need
+    uint4 raw[4];
+    auto load = [&](int u0) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int u = u0 + 2 * i + half;
+            raw[i] = u < u_end ? __ldg(base + (int64_t)u * 16 + piece) : make_uint4(0, 0, 0, 0);
+        }
+    };
+    load(u_begin + warp * 8);
+    rotated_query_sum<T>(D, hk, 1, qraw, qb);
+    __syncthreads();
+    float qr[V];
+    {
+        const int i0 = ((lane & 15) * V) % D.d;
+#pragma unroll
+        for (int v = 0; v < V; ++v) qr[v] = qb[i0 + v];
+    }
+    uint64_t list = 0, cand = 0;
+    int it = 0;
+    for (int u0 = u_begin + warp * 8; u0 < u_end; u0 += nw * 8, ++it) {  // warp-uniform
+        if (it > 0) load(u0);
+        float acc[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[i] = dot16<E>(raw[i], qr);
+#pragma unroll
+        for (int m = 8, nv = 4; m >= 4; m >>= 1, nv >>= 1) {
+            const bool upper = (lane & m) != 0;
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                if (i < nv / 2) {
+                    const float send = upper ? acc[i] : acc[i + nv / 2];
+                    const float keep = upper ? acc[i + nv / 2] : acc[i];
+                    acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+                }
+            }
+        }
+        acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], 2);
+        acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], 1);
+        const int j = u0 + 2 * slot + half;
+        const float sc = acc[0] * D.inv_sqrt_d;
+        if (j < u_end) {
+            if ((lane & 3) == 0) D.uscore[(int64_t)hk * D.units_max + j] = sc;
+            if ((lane & 3) == (it & 3)) cand = make_key(sc, (uint32_t)j);
+        }
+        if ((it & 3) == 3) {
+            list = warp_topk_insert(list, cand);
+            cand = 0;
+        }
+    }
+    if (__any_sync(0xffffffffu, cand != 0)) list = warp_topk_insert(list, cand);
+    cta_lists_and_select(D, hk, split, n_mem, n_split, lists, list);
+    if (!wait_first) pdl_hold();
 }
 
 // Selection for top_k > 32: one CTA per kv head sorts every unit's composite key in shared
@@ -565,18 +710,33 @@ static cudaError_t launch_wpu1(const Dev& D, dim3 grid, int threads, int n_mem, 
                     do_select, wait_first);
 }
 
+template <typename T, int MODE>
+static cudaError_t launch_wpu_c(const Dev& D, int C, dim3 grid, int threads, int n_mem, int n_split, int n_qtiles,
+                                const T* qraw, int do_select, cudaStream_t st, bool pdl, int wf) {
+    if (C == 1) return launch_wpu1<T, MODE, 1>(D, grid, threads, n_mem, n_split, n_qtiles, qraw, do_select, st, pdl, wf);
+    if (C == 2) return launch_wpu1<T, MODE, 2>(D, grid, threads, n_mem, n_split, n_qtiles, qraw, do_select, st, pdl, wf);
+    return launch_wpu1<T, MODE, 4>(D, grid, threads, n_mem, n_split, n_qtiles, qraw, do_select, st, pdl, wf);
+}
+
 template <typename T>
 static cudaError_t launch_wpu(const Dev& D, int mode, int C, dim3 grid, int threads, int n_mem, int n_split,
                               int n_qtiles, const T* qraw, int do_select, cudaStream_t st, bool pdl,
                               int wf) {
-    if (mode == 0) {
-        if (C == 1) return launch_wpu1<T, 0, 1>(D, grid, threads, n_mem, n_split, n_qtiles, qraw, do_select, st, pdl, wf);
-        if (C == 2) return launch_wpu1<T, 0, 2>(D, grid, threads, n_mem, n_split, n_qtiles, qraw, do_select, st, pdl, wf);
-        return launch_wpu1<T, 0, 4>(D, grid, threads, n_mem, n_split, n_qtiles, qraw, do_select, st, pdl, wf);
-    }
-    if (C == 1) return launch_wpu1<T, 1, 1>(D, grid, threads, n_mem, n_split, n_qtiles, qraw, do_select, st, pdl, wf);
-    if (C == 2) return launch_wpu1<T, 1, 2>(D, grid, threads, n_mem, n_split, n_qtiles, qraw, do_select, st, pdl, wf);
-    return launch_wpu1<T, 1, 4>(D, grid, threads, n_mem, n_split, n_qtiles, qraw, do_select, st, pdl, wf);
+    if (mode == OP_REPS) return launch_wpu_c<T, OP_REPS>(D, C, grid, threads, n_mem, n_split, n_qtiles, qraw, do_select, st, pdl, wf);
+    if (mode == OP_REPSUM)
+        return launch_wpu_c<T, OP_REPSUM>(D, C, grid, threads, n_mem, n_split, n_qtiles, qraw, do_select, st, pdl, wf);
+    return launch_wpu_c<T, OP_MEANKEY>(D, C, grid, threads, n_mem, n_split, n_qtiles, qraw, do_select, st, pdl, wf);
+}
+
+// Decode scoring kernels by operand row size: 256 bytes (half-warp rows) or 512 / 1024 bytes.
+template <typename T, typename E>
+static cudaError_t launch_dec(const Dev& D, int mode, int row_bytes, dim3 grid, int n_mem, int upc, int n_split,
+                              const T* qraw, cudaStream_t st, bool pdl, int wf) {
+    if (row_bytes == 256)
+        return launch_k(k_score_dec_half<T, E>, grid, dim3(256), 0, st, pdl, D, mode, n_mem, upc, n_split, qraw, wf);
+    if (row_bytes == 512)
+        return launch_k(k_score_dec<T, E, 1, 4>, grid, dim3(256), 0, st, pdl, D, mode, n_mem, upc, n_split, qraw, wf);
+    return launch_k(k_score_dec<T, E, 2, 4>, grid, dim3(256), 0, st, pdl, D, mode, n_mem, upc, n_split, qraw, wf);
 }
 
 template <typename T>
@@ -587,11 +747,23 @@ cudaError_t launch_select(const Dev& D, int score_mode, int n_mem, int n_qtiles,
     if (n_mem <= 0 || D.topk <= 0) return cudaSuccess;
     const int fast = D.topk <= 32;
     // warp-per-32-units scoring when a unit's operand is a whole number of 512-byte rows
-    const int unit_bytes = score_mode == 0 ? D.r * D.d * (int)sizeof(T) : D.d * 4;
+    const int unit_bytes = score_mode == OP_REPS ? D.r * D.d * (int)sizeof(T)
+                         : score_mode == OP_REPSUM ? D.d * 4 : D.d * (int)sizeof(T);
     const int C = unit_bytes % 512 == 0 ? unit_bytes / 512 : 0;
     int n_split;
     cudaError_t err;
-    if (C == 1 || C == 2 || C == 4) {
+    if (qraw != nullptr && fast && (unit_bytes == 256 || unit_bytes == 512 || unit_bytes == 1024)) {
+        // one query token: stream the pool with at most two CTAs of 256 threads per SM, so that the whole
+        // grid is resident beside the decode step's sink and window tiles (they share the SMs)
+        const int64_t want = ((int64_t)n_mem * D.Hkv + 2 * 148 - 1) / (2 * 148);
+        int upc = (int)std::max<int64_t>(32, (want + 31) / 32 * 32);
+        n_split = (n_mem + upc - 1) / upc;
+        if (n_split > D.score_splits_max) return cudaErrorInvalidValue;
+        const dim3 grid(n_split, D.Hkv);
+        err = score_mode == OP_REPSUM
+                  ? launch_dec<T, float>(D, score_mode, unit_bytes, grid, n_mem, upc, n_split, (const T*)qraw, st, pdl, wf)
+                  : launch_dec<T, T>(D, score_mode, unit_bytes, grid, n_mem, upc, n_split, (const T*)qraw, st, pdl, wf);
+    } else if (C == 1 || C == 2 || C == 4) {
         // warps per CTA (4..8, each warp scores 32 units): the one whose CTA count fills the
         // waves of 2 CTAs per SM on 148 SMs best, the larger on ties (fewer lists to merge); not
         // fewer than 4 warps, as the last CTA of a head merges the lists of the others
@@ -616,9 +788,11 @@ cudaError_t launch_select(const Dev& D, int score_mode, int n_mem, int n_qtiles,
         n_split = (n_mem + per - 1) / per;
         if (n_split > D.score_splits_max) return cudaErrorInvalidValue;
         dim3 grid(n_split, D.Hkv);
-        err = score_mode == 0
-                  ? launch_score<T, 0>(D, lpu, grid, n_mem, n_split, n_qtiles, (const T*)qraw, fast, st, pdl, wf)
-                  : launch_score<T, 1>(D, lpu, grid, n_mem, n_split, n_qtiles, (const T*)qraw, fast, st, pdl, wf);
+        err = score_mode == OP_REPS
+                  ? launch_score<T, OP_REPS>(D, lpu, grid, n_mem, n_split, n_qtiles, (const T*)qraw, fast, st, pdl, wf)
+              : score_mode == OP_REPSUM
+                  ? launch_score<T, OP_REPSUM>(D, lpu, grid, n_mem, n_split, n_qtiles, (const T*)qraw, fast, st, pdl, wf)
+                  : launch_score<T, OP_MEANKEY>(D, lpu, grid, n_mem, n_split, n_qtiles, (const T*)qraw, fast, st, pdl, wf);
     }
     ++*launches;
     if (err != cudaSuccess) return err;

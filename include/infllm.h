@@ -61,10 +61,15 @@ typedef enum {
 
 typedef enum { INFLLM_F32 = 0, INFLLM_BF16 = 1 } infllm_dtype;
 
-/* How a unit is scored against the chunk's queries.  Both are the same number in exact
- * arithmetic (the dot product is linear in the key): REPS reads the n_reps representative
- * keys of every unit; REPSUM reads one fp32 sum of them per unit (half the bytes). */
-typedef enum { INFLLM_SCORE_REPS = 0, INFLLM_SCORE_REPSUM = 1 } infllm_score_mode;
+/* How a unit is scored against the chunk's queries.  REPS and REPSUM are the same number in exact
+ * arithmetic (the dot product is linear in the key): REPS reads the n_reps representative keys of
+ * every unit; REPSUM reads one fp32 sum of them per unit (half the bytes).  MEANKEY scores a unit by
+ * the mean of all of its keys (one vector per unit in the context dtype, the sum taken in fp64 and
+ * rounded once), the alternative representation that "InfLLM: Training-Free Long-Context
+ * Extrapolation for LLMs with an Efficient Context Memory" (research-map summary, "Measured effects",
+ * row "Use selected representative tokens instead of mean key-vector representations") compares
+ * against; it selects different units than REPS. */
+typedef enum { INFLLM_SCORE_REPS = 0, INFLLM_SCORE_REPSUM = 1, INFLLM_SCORE_MEANKEY = 2 } infllm_score_mode;
 
 typedef struct {
     int32_t n_q_heads;   /* Hq; Hq % Hkv == 0; q head h uses kv head h / (Hq/Hkv) */
@@ -187,7 +192,7 @@ infllm_status infllm_get_reps(infllm_ctx* ctx, int32_t unit_begin, int32_t n_uni
 
 infllm_status infllm_get_stats(infllm_ctx* ctx, infllm_stats* out);
 
-/* Switch the unit-scoring operand (infllm_score_mode) for later calls; both pools are always
+/* Switch the unit-scoring operand (infllm_score_mode) for later calls; every operand pool is always
  * maintained, so this is valid at any point of a stream. */
 infllm_status infllm_set_score_mode(infllm_ctx* ctx, int32_t score_mode);
 

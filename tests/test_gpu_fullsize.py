@@ -33,8 +33,11 @@ def _check_chunk(w, src, cfg, oreps, rep_keys, c0, n, g_out, g_sel, g_scores, g_
     tol = TOL[w.dtype]
     n_dec, bad = compare_selection(g_sel, info["sigma"], w.top_k)
     # unit scores: where the GPU chose the same representatives, the scores must agree
-    same = np.array([[sorted(oreps[j][h]) == sorted(int(x) for x in g_reps[h, j]) for j in range(nm)]
-                     for h in range(w.n_kv_heads)])
+    if cfg.get("unit_repr") == "meankey":  # mean keys do not depend on the representatives
+        same = np.ones((w.n_kv_heads, nm), dtype=bool)
+    else:
+        same = np.array([[sorted(oreps[j][h]) == sorted(int(x) for x in g_reps[h, j]) for j in range(nm)]
+                         for h in range(w.n_kv_heads)])
     for h in range(w.n_kv_heads):
         scale = max(1e-6, float(np.max(np.abs(info["sigma"][h]))))
         diff = np.abs(g_scores[h][:nm] - info["sigma"][h])[same[h]]
@@ -126,7 +129,7 @@ def test_decode_1m_fullsize(cuda_ok):
     import torch
     w = synth.WORKLOADS["decode_1m"]
     cfg, src = w.as_config(), Source(w)
-    layer = make_layer(w)
+    layer = make_layer(w, max_tokens=w.total_tokens + 2)
     for c0 in range(0, w.n_tokens, w.build_chunk):
         n = min(w.build_chunk, w.n_tokens - c0)
         q, k, v = synth.gen_chunk(w, c0, n)
@@ -153,4 +156,16 @@ def test_decode_1m_fullsize(cuda_ok):
         nm = O.n_mem(t, w.n_sink, w.window, w.unit_size)
         _check_chunk(w, src, cfg, oreps, rep_keys[:, :nm], t, 1, rec[s]["out"], rec[s]["sel"], rec[s]["scores"],
                      g_reps)
+    # two more steps scoring units by their mean keys, against the oracle's mean-key table
+    layer.set_score_mode("meankey")
+    mcfg = dict(cfg, unit_repr="meankey")
+    nu2 = O.n_mem(w.n_tokens + w.decode_steps + 1, w.n_sink, w.window, w.unit_size)  # a unit is evicted at step 256
+    means = O.mean_key_table(src.k, nu2, mcfg)[:, :, None, :]
+    for s in range(w.decode_steps, w.decode_steps + 2):
+        t = w.n_tokens + s
+        q, k, v = synth.gen_chunk(w, t, 1)
+        out = layer.decode_step(to_torch(q), to_torch(k), to_torch(v))
+        torch.cuda.synchronize()
+        _check_chunk(w, src, mcfg, oreps, means, t, 1, to_np64(out), layer.selection().copy(),
+                     layer.unit_scores().copy(), g_reps)
     layer.close()

@@ -22,24 +22,33 @@ SMALL_PREFILL = ["small_gqa", "small_g4", "small_d64", "small_u256", "small_nosi
                  "small_g2"]
 
 
-def _stream_oracle(w):
+def _stream_oracle(w, score_mode="reps"):
     src = Source(w)
     T = w.n_tokens
-    layer = O.OracleLayer(w.as_config(), rep_method="linear")
+    layer = O.OracleLayer(_oracle_cfg(w, score_mode), rep_method="linear")
     q, k, v = src.q(0, T), src.k(0, T), src.v(0, T)
     return layer, q, k, v
 
 
-# every shape with the representative keys; the fp32 sum of them (REPSUM) on four shapes
-PREFILL_CASES = [(n, "reps") for n in SMALL_PREFILL] + [(n, "repsum") for n in
-                                                       ("small_gqa", "small_g4", "small_f32", "small_g8")]
+# every shape with the representative keys; the fp32 sum of them (REPSUM) and the units' mean keys
+# (MEANKEY) on four shapes each
+PREFILL_CASES = ([(n, "reps") for n in SMALL_PREFILL] +
+                 [(n, "repsum") for n in ("small_gqa", "small_g4", "small_f32", "small_g8")] +
+                 [(n, "meankey") for n in ("small_gqa", "small_g4", "small_f32", "small_d64")])
+
+
+def _oracle_cfg(w, score_mode):
+    cfg = w.as_config()
+    if score_mode == "meankey":
+        cfg["unit_repr"] = "meankey"
+    return cfg
 
 
 @pytest.mark.parametrize("name,score_mode", PREFILL_CASES)
 def test_prefill_stream_matches_oracle(cuda_ok, name, score_mode):
     w = synth.SMALL[name]
     glayer, res = run_prefill(w, score_mode=score_mode)
-    olayer, q, k, v = _stream_oracle(w)
+    olayer, q, k, v = _stream_oracle(w, score_mode)
     tol = TOL[w.dtype]
     worst = 0.0
     n_dec = n_sel = 0
@@ -100,13 +109,14 @@ def test_chunked_equals_stateless_on_gpu_reps(cuda_ok):
     glayer.close()
 
 
-@pytest.mark.parametrize("name", ["small_decode", "small_decode_g8"])
-def test_decode_matches_oracle(cuda_ok, name):
+@pytest.mark.parametrize("name,score_mode", [("small_decode", "reps"), ("small_decode_g8", "reps"),
+                                             ("small_decode", "meankey"), ("small_decode", "repsum")])
+def test_decode_matches_oracle(cuda_ok, name, score_mode):
     import torch
     w = synth.SMALL[name]
-    glayer = make_layer(w)
+    glayer = make_layer(w, score_mode=score_mode)
     src = Source(w)
-    olayer = O.OracleLayer(w.as_config(), rep_method="linear")
+    olayer = O.OracleLayer(_oracle_cfg(w, score_mode), rep_method="linear")
     T0 = w.n_tokens
     for c0 in range(0, T0, w.build_chunk):
         n = min(w.build_chunk, T0 - c0)

@@ -5,7 +5,6 @@ finished. Each kernel has one of three codes (the griddepcontrol instructions it
 - early: trigger at entry, and one thread waits at exit. Its body may run beside the kernels
   before it; it completes only after its predecessor has.
 - late: wait at entry, then trigger. Past the wait, every earlier kernel is complete.
-- late, trigger first (the decode tile kernel): trigger at entry, then wait before the body.
 Plainly launched kernels (the first of each call, every launch with chaining off, and the
 kernels launched without the attribute) start only once their predecessor is complete.
 
@@ -26,7 +25,7 @@ import math
 
 import pytest
 
-EARLY, LATE, LTF, NOPDL = "early", "late", "late_trigger_first", "no_pdl"
+EARLY, LATE, NOPDL = "early", "late", "no_pdl"
 PLAIN = "plain"
 
 
@@ -168,15 +167,26 @@ class Schedule:
         self.chain = False
         t = self.tokens
         if self.tc_decode and self.G <= 8:
-            new_reps = self.reps_to(self.n_mem(t))
-            self.launch("decode_append", EARLY, {("in", tag)},
-                        self.keys(t, t + 1) | {("cs_chunk",)} | self.yblocks(t, t + 1))
+            # representatives of a newly evicted unit, then the whole step in one cooperative launch
+            # (launched without the chaining attribute: it starts once everything before has finished)
+            self.reps_to(self.n_mem(t))
+            L = self.nlook
+            self.nlook += 1
+            nm = self.n_mem(t)
+            B = self.S + self.U * nm
+            reads = {("in", tag), self.selbuf(L)} | self.keys(0, t + 1) | {("rep", j) for j in range(nm)} | \
+                self.yblocks(t, t + 1)
+            writes = self.keys(t, t + 1) | self.yblocks(t, t + 1) | {("dpart", 0), ("dpart", 1), ("out", tag),
+                                                                    self.selbuf(L), ("uscore",), ("cand",)}
+            if self.plant == "decode_step_chained":
+                self.launch("decode_step", EARLY, reads, writes)
+            else:
+                self.launch("decode_step", NOPDL, reads, writes, attr=False)
             self.chain = True
             self.tokens = t + 1
-        else:
-            self.pending_c0 = t
-            self.stage_store(1, tag)
-            new_reps = True
+            return
+        self.pending_c0 = t
+        self.stage_store(1, tag)
         if self.G > 8:
             self.attend_chunk(1, tag, decoding=True)
             return
@@ -184,18 +194,6 @@ class Schedule:
         self.nlook += 1
         nm = self.n_mem(t)
         kk = min(self.topk, nm)
-        B = self.S + self.U * nm
-        if self.tc_decode:
-            self.launch("decode_tiles0", LTF, {("in", tag), ("cs_chunk",)} | self.keys(0, min(self.S, t + 1)) |
-                        self.keys(B, t + 1), {("dpart", 0)})
-            self.chain = True
-            if kk > 0:
-                wait_first = new_reps and self.plant != "decode_score_never_waits"
-                self.stage_select(L, nm, tag, wait_first)
-                self.launch("decode_tiles1", LTF, {("in", tag), self.selbuf(L)} |
-                            self.keys(self.S, self.S + nm * self.U), {("dpart", 1)})
-            self.launch("decode_merge", LATE, {("dpart", 0), ("dpart", 1)}, {("out", tag)})
-            return
         if kk > 0:
             self.stage_select(L, nm, tag, True)
         self.launch("decode", NOPDL, {("in", tag), ("cs_chunk",), self.selbuf(L)} | self.keys(0, t + 1),
@@ -205,7 +203,7 @@ class Schedule:
 def overlapping_conflicts(launches):
     """Pairs (a, b), a < b, that launch chaining may run at the same time and that touch one
     buffer with at least one write."""
-    body_waits = {PLAIN, LATE, LTF}      # the body starts only after the predecessor completed
+    body_waits = {PLAIN, LATE}           # the body starts only after the predecessor completed
     trigger_waits = {PLAIN, LATE}        # the trigger comes only after the predecessor completed
     found = []
     for b, (nb, mb, rb, wb) in enumerate(launches):
@@ -318,7 +316,7 @@ PLANTS = {
     "one_selection_buffer": ("attend", "score", "sel"),          # lookup c over the selection attend c-1 reads
     "attention_early": ("score", "attend", "sel"),               # attention before its selection is final
     "chunk1_chained_without_lookup": ("ysum", "reps", "Y"),      # chunk 1's representatives beside chunk 0's sums
-    "decode_score_never_waits": ("reps", "score", "rep"),        # scoring units whose representatives are in flight
+    "decode_step_chained": ("reps", "decode_step", "rep"),       # a decode step beside its new representatives
 }
 
 
