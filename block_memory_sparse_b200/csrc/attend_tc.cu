@@ -15,9 +15,7 @@
 //                             online softmax over its columns of every tile -- its own running
 //                             max, sum and accumulator O_h -- so the two never wait for each
 //                             other inside the loop; O_h is rescaled lazily (only when the half's
-//                             max grows by > 2^8), and a tile's exponentials are taken against the
-//                             running reference while its max is found, so they are redone only on
-//                             a rescale.  P_i goes as bf16 into the TMEM columns of S_i.
+//                             max grows by > 2^8).  P_i goes as bf16 into the TMEM columns of S_i.
 //                             After the last tile the halves exchange (max, sum) once through
 //                             shared memory and each thread stores 64 outputs of the merged row.
 // Splitting a row's keys in two and merging the partial softmaxes at the end is exact (up to
@@ -208,21 +206,6 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
-// Exponentials of 64 logits (log2 units after fma(s, sc, nref)) as 32 packed bf16 pairs, and their
-// sums in 4 independent partials.
-__device__ __forceinline__ void exp_pack(const float* s, float sc, float nref, uint32_t* w, float* rs) {
-#pragma unroll
-    for (int e = 0; e < 4; ++e) rs[e] = 0.f;
-#pragma unroll
-    for (int e = 0; e < 32; ++e) {
-        const float p0 = ex2(fmaf(s[2 * e], sc, nref)), p1 = ex2(fmaf(s[2 * e + 1], sc, nref));
-        rs[(2 * e) & 3] += p0;
-        rs[(2 * e + 1) & 3] += p1;
-        __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
-        w[e] = *reinterpret_cast<uint32_t*>(&h);
-    }
-}
-
 // PV completions are consumed strictly in order, and never more than one phase late: a parity
 // wait on an mbarrier that has completed two phases past the awaited one would wait for a third.
 // Tile i consumes PV(i - 1) before it releases P_i; PV(i) cannot have been issued by then.
@@ -273,51 +256,57 @@ __device__ void softmax_role(const Plan& P, const Dev& D, Bars* bars, float* lsu
             lim = c < (int64_t)lim ? (int)(c < 0 ? 0 : c) : lim;
         }
         const int own = lim - half * 64;  // valid columns of this half
-        if (!__all_sync(0xffffffffu, own >= 64)) {
+        float mq[8];                       // independent partial maxima (short dependency chains)
 #pragma unroll
-            for (int c = 0; c < 64; ++c) s[c] = c < own ? s[c] : -INFINITY;
+        for (int e = 0; e < 8; ++e) mq[e] = -INFINITY;
+        if (__all_sync(0xffffffffu, own >= 64)) {
+#pragma unroll
+            for (int c = 0; c < 64; ++c) mq[c & 7] = fmaxf(mq[c & 7], s[c]);
+        } else {
+#pragma unroll
+            for (int c = 0; c < 64; ++c) {
+                s[c] = c < own ? s[c] : -INFINITY;
+                mq[c & 7] = fmaxf(mq[c & 7], s[c]);
+            }
         }
-        // The exponentials are taken against the running reference max together with this tile's max
-        // (the two do not depend on each other); only when the max grows past the lazy threshold, or a
-        // row has no reference yet, are they taken again against the new reference.
-        float rs[4];
-        uint32_t w[32];  // this half's 64 keys as 32 columns of packed bf16 pairs
-        const bool spec = !__any_sync(0xffffffffu, m_used == -INFINITY);
-        if (spec) exp_pack(s, sc, -m_used, w, rs);
-        float mq[4];  // independent partial maxima (short dependency chains)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) mq[e] = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < 64; ++c) mq[c & 3] = fmaxf(mq[c & 3], s[c]);
-        const float mx = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
+        const float mx = fmaxf(fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])), fmaxf(fmaxf(mq[4], mq[5]), fmaxf(mq[6], mq[7])));
         const float mt = mx * sc;
         const bool need = mt > m_used + RESCALE_LOG2;
         const float m_new = need ? mt : m_used;
-        const bool any_need = __any_sync(0xffffffffu, need);
-        if (!spec || any_need) {  // rare after the first tiles: the speculative exponentials are dropped
-            if (i >= 1 && any_need) {  // O_half must hold every earlier product first
-                if (!pv.upto(i - 1, bars, D)) {
-                    ok = false;
-                    break;
-                }
-                ptx::tc_fence_after();
-                const float f = need ? ex2(m_used - m_new) : 1.f;
-                l *= f;
-#pragma unroll
-                for (int c4 = 0; c4 < HD / 32; ++c4) {
-                    float o[32];
-                    ptx::tmem_ld32(o_addr + c4 * 32, o);
-                    ptx::tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) o[e] *= f;
-                    ptx::tmem_st32(o_addr + c4 * 32, o);
-                }
+        if (i >= 1 && __any_sync(0xffffffffu, need)) {  // O_half must hold every earlier product first
+            if (!pv.upto(i - 1, bars, D)) {
+                ok = false;
+                break;
             }
-            m_used = m_new;
-            exp_pack(s, sc, m_used == -INFINITY ? 0.f : -m_used, w, rs);
+            ptx::tc_fence_after();
+            const float f = need ? ex2(m_used - m_new) : 1.f;
+            l *= f;
+#pragma unroll
+            for (int c4 = 0; c4 < HD / 32; ++c4) {
+                float o[32];
+                ptx::tmem_ld32(o_addr + c4 * 32, o);
+                ptx::tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) o[e] *= f;
+                ptx::tmem_st32(o_addr + c4 * 32, o);
+            }
+        }
+        m_used = m_new;
+        const float nref = m_used == -INFINITY ? 0.f : -m_used;
+        float rs[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) rs[e] = 0.f;
+        uint32_t w[32];  // this half's 64 keys as 32 columns of packed bf16 pairs
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+            const float p0 = ex2(fmaf(s[2 * e], sc, nref)), p1 = ex2(fmaf(s[2 * e + 1], sc, nref));
+            rs[(2 * e) & 7] += p0;
+            rs[(2 * e + 1) & 7] += p1;
+            __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
+            w[e] = *reinterpret_cast<uint32_t*>(&h);
         }
         ptx::tmem_st32(sbase + half * 64, reinterpret_cast<const float*>(w));  // over this half's own S columns
-        l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
+        l += ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
         ptx::tmem_wait_st();
         // PV(i - 1) ran during this tile's exponentials; consume its completion before P_i is
         // released (PV(i) is issued only after the arrival below)
