@@ -257,9 +257,9 @@ infllm_status stage_attend(infllm_ctx* c, int64_t L, int64_t c0, int32_t n, void
     const int kk = lookup ? std::min(D.topk, nm) : 0;  // without lookup: sinks and window only
     const int64_t B = (int64_t)D.S + (int64_t)D.U * nm;
     Prof p(c, K_ATTEND);
-    if (c->use_tc && sizeof(T) == 2) {
+    if constexpr (sizeof(T) == 2) {  // bf16: always the tensor cores (create refuses shapes they cannot take)
         CK(launch_attend_tc(D, c0, n, kk, B, (int)(L % 3), out, c->stream, c->tmaps, pdl_ok(c)));
-    } else {
+    } else {  // fp32 operands: CUDA cores
         CK(launch_attend_simt<T>(D, c0, n, kk, B, (int)(L % 3), out, c->stream, pdl_ok(c)));
     }
     c->chain = true;
@@ -561,9 +561,13 @@ infllm_status create_impl(infllm_ctx* c) {
     CK(cudaHostGetDevicePointer((void**)&D.err, c->err_host, 0));
     c->use_tc = false;
     c->step_coop = getenv("INFLLM_DECODE_CHAIN") == nullptr;
-    if (g.dtype == INFLLM_BF16 && attend_tc_supported(D) && getenv("INFLLM_FORCE_SIMT") == nullptr) {
+    if (g.dtype == INFLLM_BF16) {
+        if (!attend_tc_supported(D))
+            return fail(c, INFLLM_EINVAL, "bf16 needs the tensor-core attention: head_dim 64 or 128, "
+                        "q heads per KV head dividing 128, top_k <= 4096, an sm_100 device");
         c->tmaps = malloc(tc_maps_size());
         c->use_tc = c->tmaps && make_tc_maps(D, c->tmaps);
+        if (!c->use_tc) return fail(c, INFLLM_ECUDA, "tensor map encoding failed");
     }
     infllm_status zs = zero_state(c);
     if (zs != INFLLM_OK) return zs;

@@ -1,7 +1,6 @@
 // Exact attention of a chunk over sinks U selected units U local window, on the CUDA cores
-// with fp32 arithmetic.  This is the path for fp32 layers (fp32 inputs need fp32 products;
-// TF32 tensor cores are not accurate enough) and for shapes the tensor-core kernel does not
-// cover.
+// with fp32 arithmetic.  This is the path of fp32 layers: fp32 inputs need fp32 products, and
+// TF32 tensor cores are not accurate enough.  bf16 layers always run on the tensor cores.
 //
 // Method: "InfLLM Guide: Training-Free Long-Context Memory Units", "Core Innovation 2",
 // item 3 "Exact Attention Evaluation": one softmax over the working context
@@ -137,7 +136,5 @@ cudaError_t launch_attend_simt(const Dev& D, int64_t c0, int n, int kk, int64_t 
 }
 
 template cudaError_t launch_attend_simt<float>(const Dev&, int64_t, int, int, int64_t, int, void*, cudaStream_t, bool);
-template cudaError_t launch_attend_simt<__nv_bfloat16>(const Dev&, int64_t, int, int, int64_t, int, void*, cudaStream_t,
-                                                       bool);
 
 }  // namespace infllm

@@ -39,24 +39,31 @@ namespace {
 
 constexpr int BM = 128;  // packed query rows per CTA
 constexpr int BN = 128;  // keys per tile
-constexpr int HD = 128;  // head dim handled here
 constexpr int NTHREADS = 320;  // producer warp, MMA warp, 8 softmax warps
 constexpr int NSOFT = 256;     // softmax threads
-constexpr uint32_t TILE = BN * HD * 2;  // bytes of one bf16 128 x 128 tile
-constexpr uint32_t HALF = TILE / 2;     // one 64-column swizzle block (128 rows x 128 B)
-constexpr int NSTAGE = 2;                      // K and V ring depth
-constexpr int OFF_QM = 0;                      // R(W) q tile (sinks and memory units)
-constexpr int OFF_QW = OFF_QM + (int)TILE;     // R(t) q tile (window)
-constexpr int OFF_K = OFF_QW + (int)TILE;
-constexpr int OFF_V = OFF_K + NSTAGE * (int)TILE;
-constexpr int OFF_BAR = OFF_V + NSTAGE * (int)TILE;
-constexpr int OFF_LSUM = OFF_BAR + 256;            // [2 halves][128] row sums
-constexpr int OFF_MREF = OFF_LSUM + 2 * 128 * 4;   // [2 halves][128] reference maxima (log2 units)
-constexpr int OFF_SEL = OFF_MREF + 2 * 128 * 4;    // selected unit ids of this KV head
-constexpr int MAX_SEL = 256;
-constexpr int SMEM_BYTES = OFF_SEL + MAX_SEL * 4 + 1024;  // + alignment slack
-constexpr uint32_t TMEM_COLS = 512;  // S0 / P0 [0,128), S1 / P1 [128,256), O_0 [256,384), O_1 [384,512)
-constexpr uint32_t TM_O = 256;       // O_h: the products with the keys of column half h of every tile
+constexpr uint32_t SWB = BN * 128;  // one 64-column swizzle block of a tile (128 rows x 128 B)
+constexpr int NSTAGE = 2;           // K and V ring depth
+constexpr int MAX_SEL = 4096;       // selected unit ids of this KV head kept in shared memory
+
+// Shared-memory layout for head dim HD (64 or 128): a tile is HD / 64 swizzle blocks.
+template <int HD>
+struct Lay {
+    static constexpr uint32_t TILE = BN * HD * 2;  // bytes of one bf16 128 x HD tile
+    static constexpr int OFF_QM = 0;               // R(W) q tile (sinks and memory units)
+    static constexpr int OFF_QW = OFF_QM + (int)TILE;  // R(t) q tile (window)
+    static constexpr int OFF_K = OFF_QW + (int)TILE;
+    static constexpr int OFF_V = OFF_K + NSTAGE * (int)TILE;
+    static constexpr int OFF_BAR = OFF_V + NSTAGE * (int)TILE;
+    static constexpr int OFF_LSUM = OFF_BAR + 256;           // [2 halves][128] row sums
+    static constexpr int OFF_MREF = OFF_LSUM + 2 * 128 * 4;  // [2 halves][128] reference maxima (log2 units)
+    static constexpr int OFF_SEL = OFF_MREF + 2 * 128 * 4;   // selected unit ids of this KV head
+    static constexpr int SMEM_BYTES = OFF_SEL + MAX_SEL * 4 + 1024;  // + alignment slack
+};
+static_assert(Lay<128>::SMEM_BYTES <= 227 * 1024, "shared-memory layout exceeds the per-CTA limit");
+
+// TMEM columns: S0 / P0 [0,128), S1 / P1 [128,256), O_0 [256, 256 + HD), O_1 [256 + HD, 256 + 2 HD)
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t TM_O = 256;  // O_h: the products with the keys of column half h of every tile
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float RESCALE_LOG2 = 8.0f;
 constexpr int ERR_TIMEOUT = 16;
@@ -109,7 +116,16 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Bars* b
     return true;
 }
 
+// One tile row of HD bf16 is HD / 64 swizzle blocks, each its own 64-column TMA box.
+template <int HD>
+__device__ __forceinline__ void load_tile(uint8_t* dst, const CUtensorMap* m, uint64_t* bar, int y, int hk) {
+#pragma unroll
+    for (int b = 0; b < HD / 64; ++b) ptx::tma_load_3d(dst + b * SWB, m, bar, 64 * b, y, hk);
+}
+
+template <int HD>
 __device__ void producer(const TcMaps& maps, const Plan& P, const Dev& D, uint8_t* sm, Bars* bars) {
+    using Y = Lay<HD>;
     ptx::prefetch_tmap(&maps.qm);
     ptx::prefetch_tmap(&maps.qw);
     ptx::prefetch_tmap(&maps.kraw);
@@ -117,11 +133,9 @@ __device__ void producer(const TcMaps& maps, const Plan& P, const Dev& D, uint8_
     ptx::prefetch_tmap(&maps.v);
     {   // both rotated query tiles of this CTA's 128 packed rows (slot par of the query buffers)
         const int y = P.par * (int)D.qrows_max + P.a * BM;
-        ptx::mbar_expect_tx(&bars->q, 2 * TILE);
-        ptx::tma_load_3d(sm + OFF_QM, &maps.qm, &bars->q, 0, y, P.hk);
-        ptx::tma_load_3d(sm + OFF_QM + HALF, &maps.qm, &bars->q, 64, y, P.hk);
-        ptx::tma_load_3d(sm + OFF_QW, &maps.qw, &bars->q, 0, y, P.hk);
-        ptx::tma_load_3d(sm + OFF_QW + HALF, &maps.qw, &bars->q, 64, y, P.hk);
+        ptx::mbar_expect_tx(&bars->q, 2 * Y::TILE);
+        load_tile<HD>(sm + Y::OFF_QM, &maps.qm, &bars->q, y, P.hk);
+        load_tile<HD>(sm + Y::OFF_QW, &maps.qw, &bars->q, y, P.hk);
     }
     int issued = 0;
     for (int i = 0; i < P.NT; ++i) {
@@ -130,16 +144,14 @@ __device__ void producer(const TcMaps& maps, const Plan& P, const Dev& D, uint8_
         if (i >= NSTAGE && !wait_bar(&bars->kempty[s], (use - 1) & 1, bars, D)) break;
         const TileInfo T = P.tile(D, i);
         const CUtensorMap* km = T.kind == 2 ? &maps.krot : &maps.kraw;
-        ptx::mbar_expect_tx(&bars->kfull[s], TILE);
-        ptx::tma_load_3d(sm + OFF_K + s * TILE, km, &bars->kfull[s], 0, (int)T.y0, P.hk);
-        ptx::tma_load_3d(sm + OFF_K + s * TILE + HALF, km, &bars->kfull[s], 64, (int)T.y0, P.hk);
+        ptx::mbar_expect_tx(&bars->kfull[s], Y::TILE);
+        load_tile<HD>(sm + Y::OFF_K + s * Y::TILE, km, &bars->kfull[s], (int)T.y0, P.hk);
         if (i >= NSTAGE && !wait_bar(&bars->vempty[s], (use - 1) & 1, bars, D)) {
             issued = i + 1;
             break;
         }
-        ptx::mbar_expect_tx(&bars->vfull[s], TILE);
-        ptx::tma_load_3d(sm + OFF_V + s * TILE, &maps.v, &bars->vfull[s], 0, (int)T.y0, P.hk);
-        ptx::tma_load_3d(sm + OFF_V + s * TILE + HALF, &maps.v, &bars->vfull[s], 64, (int)T.y0, P.hk);
+        ptx::mbar_expect_tx(&bars->vfull[s], Y::TILE);
+        load_tile<HD>(sm + Y::OFF_V + s * Y::TILE, &maps.v, &bars->vfull[s], (int)T.y0, P.hk);
         issued = i + 1;
     }
     if (*(volatile int*)&bars->abort) {
@@ -152,13 +164,15 @@ __device__ void producer(const TcMaps& maps, const Plan& P, const Dev& D, uint8_
     }
 }
 
+template <int HD>
 __device__ void mma_issuer(const Plan& P, const Dev& D, uint8_t* sm, Bars* bars, uint32_t tmem) {
+    using Y = Lay<HD>;
     constexpr uint32_t IDESC_QK = ptx::idesc_bf16_f32(BM, BN, false, false);
     constexpr uint32_t IDESC_PV = ptx::idesc_bf16_f32(BM, HD, false, true);
     if (!wait_bar(&bars->q, 0, bars, D)) return;  // the query tiles have landed
     ptx::tc_fence_after();
-    const uint32_t qm = ptx::smem_u32(sm + OFF_QM), qw = ptx::smem_u32(sm + OFF_QW);
-    const uint32_t kb = ptx::smem_u32(sm + OFF_K), vb = ptx::smem_u32(sm + OFF_V);
+    const uint32_t qm = ptx::smem_u32(sm + Y::OFF_QM), qw = ptx::smem_u32(sm + Y::OFF_QW);
+    const uint32_t kb = ptx::smem_u32(sm + Y::OFF_K), vb = ptx::smem_u32(sm + Y::OFF_V);
     for (int i = 0; i <= P.NT; ++i) {
         if (i < P.NT) {
             // S_i into buffer i & 1, which held P_{i-2}: PV(i - 2) was issued in the previous
@@ -167,10 +181,10 @@ __device__ void mma_issuer(const Plan& P, const Dev& D, uint8_t* sm, Bars* bars,
             if (!wait_bar(&bars->kfull[s], (uint32_t)(i / NSTAGE) & 1, bars, D)) return;
             ptx::tc_fence_after();
             const uint32_t qa = P.tile(D, i).kind == 2 ? qw : qm;
-            const uint32_t ka = kb + s * TILE;
+            const uint32_t ka = kb + s * Y::TILE;
 #pragma unroll
-            for (int ks = 0; ks < HD / 16; ++ks) {
-                const uint32_t off = (uint32_t)(ks >> 2) * HALF + (uint32_t)(ks & 3) * 32;
+            for (int ks = 0; ks < HD / 16; ++ks) {  // 16 of the head dim: swizzle block ks / 4, 32 B each
+                const uint32_t off = (uint32_t)(ks >> 2) * SWB + (uint32_t)(ks & 3) * 32;
                 ptx::mma_bf16(tmem + b * BN, ptx::sdesc_sw128(qa + off, 16, 1024), ptx::sdesc_sw128(ka + off, 16, 1024),
                               IDESC_QK, ks > 0 ? 1u : 0u);
             }
@@ -182,12 +196,12 @@ __device__ void mma_issuer(const Plan& P, const Dev& D, uint8_t* sm, Bars* bars,
             if (!wait_bar(&bars->pfull, (uint32_t)j & 1, bars, D)) return;
             if (!wait_bar(&bars->vfull[sj], (uint32_t)(j / NSTAGE) & 1, bars, D)) return;
             ptx::tc_fence_after();
-            const uint32_t va = vb + sj * TILE;
+            const uint32_t va = vb + sj * Y::TILE;
 #pragma unroll
             for (int ks = 0; ks < BN / 16; ++ks)  // keys 16 ks ..: half h = ks / 4 of P_j into O_h
                 ptx::mma_bf16_ts(tmem + TM_O + (uint32_t)(ks >> 2) * HD,
                                  tmem + bj * BN + (uint32_t)(ks >> 2) * 64 + (uint32_t)(ks & 3) * 8,
-                                 ptx::sdesc_sw128(va + (uint32_t)ks * 2048, HALF, 1024), IDESC_PV,
+                                 ptx::sdesc_sw128(va + (uint32_t)ks * 2048, SWB, 1024), IDESC_PV,
                                  (j > 0 || (ks & 3) > 0) ? 1u : 0u);
             ptx::mma_commit(&bars->pvdone);
             ptx::mma_commit(&bars->vempty[sj]);
@@ -220,6 +234,7 @@ struct PvTrack {
     }
 };
 
+template <int HD>
 __device__ void softmax_role(const Plan& P, const Dev& D, Bars* bars, float* lsum, float* mref, uint32_t tmem,
                              int64_t c0, int n, __nv_bfloat16* __restrict__ out, int warp, int lane) {
     const int quarter = warp & 3;        // TMEM lanes this warp may access
@@ -319,8 +334,8 @@ __device__ void softmax_role(const Plan& P, const Dev& D, Bars* bars, float* lsu
     }
     ok = ok && pv.upto(P.NT - 1, bars, D);
     // the two halves of the row meet: O = (2^(m_0 - M) O_0 + 2^(m_1 - M) O_1) / (same weights on
-    // l_0, l_1), M = max(m_0, m_1).  Every softmax thread reaches this barrier: all waits above
-    // are bounded.
+    // l_0, l_1), M = max(m_0, m_1); each of the pair stores HD / 2 outputs of the row.  Every
+    // softmax thread reaches this barrier: all waits above are bounded.
     lsum[half * 128 + row] = l;
     mref[half * 128 + row] = m_used;
     asm volatile("bar.sync 1, %0;" ::"n"(NSOFT) : "memory");
@@ -331,12 +346,13 @@ __device__ void softmax_role(const Plan& P, const Dev& D, Bars* bars, float* lsu
     const float f0 = m0 == -INFINITY ? 0.f : ex2(m0 - M), f1 = m1 == -INFINITY ? 0.f : ex2(m1 - M);
     const float inv = 1.f / (lsum[row] * f0 + lsum[128 + row] * f1);
     const float g0 = f0 * inv, g1 = f1 * inv;
-    __nv_bfloat16* orow = out + ((int64_t)tl * D.Hq + P.hk * D.G + hg) * HD + half * 64;
+    constexpr int OWN = HD / 2;
+    __nv_bfloat16* orow = out + ((int64_t)tl * D.Hq + P.hk * D.G + hg) * HD + half * OWN;
 #pragma unroll 1
-    for (int c4 = 0; c4 < 2; ++c4) {
+    for (int c4 = 0; c4 < OWN / 32; ++c4) {
         float o0[32], o1[32];
-        ptx::tmem_ld32(tl_addr + TM_O + half * 64 + c4 * 32, o0);
-        ptx::tmem_ld32(tl_addr + TM_O + HD + half * 64 + c4 * 32, o1);
+        ptx::tmem_ld32(tl_addr + TM_O + half * OWN + c4 * 32, o0);
+        ptx::tmem_ld32(tl_addr + TM_O + HD + half * OWN + c4 * 32, o1);
         ptx::tmem_wait_ld();
         if (valid) {
 #pragma unroll
@@ -355,12 +371,14 @@ __device__ void softmax_role(const Plan& P, const Dev& D, Bars* bars, float* lsu
     }
 }
 
+template <int HD>
 __global__ void __launch_bounds__(NTHREADS, 1)
     k_attn_tc(const __grid_constant__ TcMaps maps, Dev D, int64_t c0, int n, int kk, int64_t B, int par,
               __nv_bfloat16* __restrict__ out) {
+    using Y = Lay<HD>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    Bars* bars = reinterpret_cast<Bars*>(sm + OFF_BAR);
+    Bars* bars = reinterpret_cast<Bars*>(sm + Y::OFF_BAR);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     Plan P;
@@ -381,7 +399,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     P.nwt = P.win_len > 0 ? (int)((P.win_len + BN - 1) / BN) : 0;
     P.NT = P.nst + P.nut + P.nwt;
 
-    int* sel_s = reinterpret_cast<int*>(sm + OFF_SEL);
+    int* sel_s = reinterpret_cast<int*>(sm + Y::OFF_SEL);
     P.sel = sel_s;
     if (threadIdx.x == 0) {
         ptx::mbar_init(&bars->q, 1);
@@ -420,12 +438,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
     if (P.NT > 0) {
         if (warp == 0) {
-            if (lane == 0) producer(maps, P, D, sm, bars);
+            if (lane == 0) producer<HD>(maps, P, D, sm, bars);
         } else if (warp == 1) {
-            if (lane == 0) mma_issuer(P, D, sm, bars, tmem);
+            if (lane == 0) mma_issuer<HD>(P, D, sm, bars, tmem);
         } else {
-            softmax_role(P, D, bars, reinterpret_cast<float*>(sm + OFF_LSUM), reinterpret_cast<float*>(sm + OFF_MREF),
-                         tmem, c0, n, out, warp, lane);
+            softmax_role<HD>(P, D, bars, reinterpret_cast<float*>(sm + Y::OFF_LSUM),
+                             reinterpret_cast<float*>(sm + Y::OFF_MREF), tmem, c0, n, out, warp, lane);
         }
     }
     ptx::tc_fence_before();
@@ -450,12 +468,12 @@ EncodeTiledFn get_encode() {
     return fn;
 }
 
-// 3-D bf16 map over [dim2][dim1][HD] with box [1][128][64], 128-byte swizzle.
-bool encode_3d(CUtensorMap* m, void* base, uint64_t dim1, uint64_t dim2) {
+// 3-D bf16 map over [dim2][dim1][hd] with box [1][128][64], 128-byte swizzle.
+bool encode_3d(CUtensorMap* m, void* base, uint64_t hd, uint64_t dim1, uint64_t dim2) {
     EncodeTiledFn enc = get_encode();
     if (!enc) return false;
-    cuuint64_t gdim[3] = {(cuuint64_t)HD, (cuuint64_t)dim1, (cuuint64_t)dim2};
-    cuuint64_t gstride[2] = {(cuuint64_t)HD * 2, (cuuint64_t)HD * 2 * dim1};
+    cuuint64_t gdim[3] = {(cuuint64_t)hd, (cuuint64_t)dim1, (cuuint64_t)dim2};
+    cuuint64_t gstride[2] = {(cuuint64_t)hd * 2, (cuuint64_t)hd * 2 * dim1};
     cuuint32_t box[3] = {64, (cuuint32_t)BN, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, gdim, gstride, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -466,7 +484,7 @@ bool encode_3d(CUtensorMap* m, void* base, uint64_t dim1, uint64_t dim2) {
 }  // namespace
 
 bool attend_tc_supported(const Dev& D) {
-    if (D.d != HD || D.G > BM || BM % D.G != 0 || D.qt * D.G != BM || D.topk > MAX_SEL) return false;
+    if ((D.d != 64 && D.d != 128) || D.G > BM || BM % D.G != 0 || D.qt * D.G != BM || D.topk > MAX_SEL) return false;
     int dev = 0, major = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return false;
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return false;
@@ -477,22 +495,31 @@ size_t tc_maps_size() { return sizeof(TcMaps); }
 
 bool make_tc_maps(const Dev& D, void* out) {
     TcMaps* m = reinterpret_cast<TcMaps*>(out);
-    return encode_3d(&m->kraw, D.Kraw, (uint64_t)D.T_max, (uint64_t)D.Hkv) &&
-           encode_3d(&m->krot, D.Krot, (uint64_t)D.T_max, (uint64_t)D.Hkv) &&
-           encode_3d(&m->v, D.V, (uint64_t)D.T_max, (uint64_t)D.Hkv) &&
-           encode_3d(&m->qm, D.Qm, 3 * (uint64_t)D.qrows_max, (uint64_t)D.Hkv) &&
-           encode_3d(&m->qw, D.Qw, 3 * (uint64_t)D.qrows_max, (uint64_t)D.Hkv);
+    const uint64_t hd = (uint64_t)D.d;
+    return encode_3d(&m->kraw, D.Kraw, hd, (uint64_t)D.T_max, (uint64_t)D.Hkv) &&
+           encode_3d(&m->krot, D.Krot, hd, (uint64_t)D.T_max, (uint64_t)D.Hkv) &&
+           encode_3d(&m->v, D.V, hd, (uint64_t)D.T_max, (uint64_t)D.Hkv) &&
+           encode_3d(&m->qm, D.Qm, hd, 3 * (uint64_t)D.qrows_max, (uint64_t)D.Hkv) &&
+           encode_3d(&m->qw, D.Qw, hd, 3 * (uint64_t)D.qrows_max, (uint64_t)D.Hkv);
 }
 
 cudaError_t launch_attend_tc(const Dev& D, int64_t c0, int n, int kk, int64_t B, int par, void* out, cudaStream_t st,
                              const void* tmaps, bool pdl) {
     if (n <= 0) return cudaSuccess;
-    static std::atomic<unsigned long long> attr_done{0};
-    cudaError_t e = smem_limit_once(k_attn_tc, SMEM_BYTES, attr_done);
-    if (e != cudaSuccess) return e;
     const int tiles = (n + D.qt - 1) / D.qt;
-    return launch_k(k_attn_tc, dim3(tiles, D.Hkv), dim3(NTHREADS), SMEM_BYTES, st, pdl,
-                    *reinterpret_cast<const TcMaps*>(tmaps), D, c0, n, kk, B, par, (__nv_bfloat16*)out);
+    const TcMaps& maps = *reinterpret_cast<const TcMaps*>(tmaps);
+    if (D.d == 64) {
+        static std::atomic<unsigned long long> attr_done{0};
+        cudaError_t e = smem_limit_once(k_attn_tc<64>, Lay<64>::SMEM_BYTES, attr_done);
+        if (e != cudaSuccess) return e;
+        return launch_k(k_attn_tc<64>, dim3(tiles, D.Hkv), dim3(NTHREADS), Lay<64>::SMEM_BYTES, st, pdl, maps, D, c0, n,
+                        kk, B, par, (__nv_bfloat16*)out);
+    }
+    static std::atomic<unsigned long long> attr_done{0};
+    cudaError_t e = smem_limit_once(k_attn_tc<128>, Lay<128>::SMEM_BYTES, attr_done);
+    if (e != cudaSuccess) return e;
+    return launch_k(k_attn_tc<128>, dim3(tiles, D.Hkv), dim3(NTHREADS), Lay<128>::SMEM_BYTES, st, pdl, maps, D, c0, n,
+                    kk, B, par, (__nv_bfloat16*)out);
 }
 
 }  // namespace infllm

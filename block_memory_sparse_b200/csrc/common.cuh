@@ -169,6 +169,16 @@ __device__ __forceinline__ uint64_t warp_topk_insert(uint64_t list, uint64_t can
     return warp_merge_desc(list, warp_sort_desc(cand));
 }
 
+// 16-byte asynchronous copy global -> shared, cached in L2 only (data other CTAs wrote this launch).
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)), "l"(src)
+                 : "memory");
+}
+// Wait for every asynchronous copy this thread issued.
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
 __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll
     for (int m = 16; m > 0; m >>= 1) x += __shfl_xor_sync(0xffffffffu, x, m);

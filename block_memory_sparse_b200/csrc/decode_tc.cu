@@ -104,12 +104,6 @@ __device__ __forceinline__ uint32_t tile_chunk(uint32_t base, int j, int c) {
     return base + (uint32_t)(c >> 3) * DHALF + (uint32_t)j * 128 + ((uint32_t)((c & 7) ^ (j & 7)) << 4);
 }
 
-__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(ptx::smem_u32(dst)), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() {
-    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
-}
 
 // Combine the partial softmaxes of `ns` tiles of KV head hk (slot_of(i) gives the i-th tile's slot,
 // in a fixed order) into one: per q head, M = max m, L = sum exp(m - M) l, O = sum exp(m - M) o.
@@ -486,41 +480,54 @@ __device__ __forceinline__ bool wait_flag(const Dev& D, const int* flag, int tag
     return true;
 }
 
-// Unit scores of units [split * upi, ...) of KV head hk (rows of ROWB bytes of E elements) by the
-// CTA's four warps: the same arithmetic and lane mapping as the streaming scoring kernel of the
-// lookup (a warp takes 4 units per step for 512- and 1024-byte rows, 8 units for 256-byte rows;
-// consecutive lanes load consecutive 16 bytes), then the CTA's top-32 list, and the head's selection
-// by its last scoring item, published on the head's selection flag.
+// Scoring rows stream through a ring of SSTAGES bulk copies of SBYTES each, in the K and V tiles'
+// shared memory; each stage has its own mbarrier after the tile barrier.
+constexpr int SSTAGES = 4;
+constexpr uint32_t SBYTES = 16384;
+static_assert(SSTAGES * SBYTES <= 2 * DTILE, "scoring ring does not fit the tile buffers");
+constexpr int OFF_SBAR = OFF_MISC + 16;
+static_assert(16 + SSTAGES * 8 <= 64, "stage barriers overflow their slot");
+
+// Unit scores of units [split * upi, ...) of KV head hk (rows of ROWB bytes of E elements).  Thread 0
+// keeps up to SSTAGES bulk copies of the item's rows in flight (one contiguous range of the pool, so
+// the whole ring is in flight while the first stage is scored); the CTA's four warps score each
+// stage from shared memory: a warp takes 4 units per step for 512- and 1024-byte rows, 8 units for
+// 256-byte rows (consecutive lanes read consecutive 16 bytes), reduces each unit's dot product with a
+// transpose-reduce and keeps a top-32 list; then the CTA's list, and the head's selection by its last
+// scoring item, published on the head's selection flag.  `sph` holds the stage barriers' parities.
+// Returns false (error word set, the copies in flight waited for) if a stage never arrived.
 template <typename E, int ROWB>
-__device__ void score_item(const Dev& D, const StepArgs& A, int hk, int split, uint8_t* sm) {
-    float* qb = reinterpret_cast<float*>(sm + OFF_Q);                               // [128]
-    auto lists = reinterpret_cast<uint64_t(*)[32]>(sm + OFF_Q + 512);            // [4][32]
+__device__ bool score_item(const Dev& D, const StepArgs& A, int hk, int split, uint8_t* sm, uint32_t& sph) {
+    float* qb = reinterpret_cast<float*>(sm + OFF_Q);                     // [128]
+    auto lists = reinterpret_cast<uint64_t(*)[32]>(sm + OFF_Q + 512);  // [4][32]
+    uint64_t* sbar = reinterpret_cast<uint64_t*>(sm + OFF_SBAR);
+    uint8_t* ring = sm + OFF_K;
     constexpr int V = 16 / sizeof(E);
     constexpr int HALFROW = ROWB == 256;
     constexpr int CPL = HALFROW ? 1 : ROWB / 512;
     constexpr int UB = HALFROW ? 8 : 4;  // units per warp step
     constexpr int GRP = 32 / (HALFROW ? 8 : 4);
+    constexpr int UPS = (int)SBYTES / ROWB;  // units per stage
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int u_begin = split * A.upi, u_end = min(A.nm, u_begin + A.upi);
-    const uint4* base = A.mode == OP_REPS
-        ? reinterpret_cast<const uint4*>((const __nv_bfloat16*)D.rep_keys + (int64_t)hk * D.units_max * D.r * D.d)
-        : A.mode == OP_REPSUM ? reinterpret_cast<const uint4*>(D.repsum + (int64_t)hk * D.units_max * D.d)
-                              : reinterpret_cast<const uint4*>((const __nv_bfloat16*)D.meankey + (int64_t)hk * D.units_max * D.d);
-    const int half = lane >> 4, piece = lane & 15;
-    uint4 raw[4][CPL];
-    auto load = [&](int u0) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int c = 0; c < CPL; ++c) {
-                const int u = HALFROW ? u0 + 2 * i + half : u0 + i;
-                raw[i][c] = u < u_end ? __ldg(HALFROW ? base + (int64_t)u * 16 + piece : base + (int64_t)u * 32 * CPL + c * 32 + lane)
-                                      : make_uint4(0, 0, 0, 0);
-            }
+    const int nch = (u_end - u_begin + UPS - 1) / UPS;
+    const uint8_t* src = (A.mode == OP_REPS ? (const uint8_t*)D.rep_keys
+                          : A.mode == OP_REPSUM ? (const uint8_t*)D.repsum
+                                                : (const uint8_t*)D.meankey) +
+                         ((int64_t)hk * D.units_max + u_begin) * ROWB;
+    auto issue = [&](int c) {  // stage c % SSTAGES <- rows of units [u_begin + c UPS, ...)
+        const uint32_t bytes = (uint32_t)(min(UPS, u_end - u_begin - c * UPS) * ROWB);
+        uint64_t* bar = &sbar[c % SSTAGES];
+        ptx::mbar_expect_tx(bar, bytes);
+        ptx::bulk_load(ring + (c % SSTAGES) * SBYTES, src + (int64_t)c * SBYTES, bytes, bar);
     };
-    load(u_begin + warp * UB);  // requested before the query sum, which it does not need
-    __syncthreads();            // the previous item's use of qb and lists is over
-    if (tid < DHD / 2) {        // R(W) (sum of the group's q heads)
+    // the ring overwrites shared memory that the generic proxy wrote (a tile's partial sums, a merge's
+    // copies); the previous item's use of qb and lists is over past the barrier
+    ptx::fence_proxy_async_smem();
+    __syncthreads();
+    if (tid == 0)
+        for (int c = 0; c < min(SSTAGES, nch); ++c) issue(c);
+    if (tid < DHD / 2) {  // R(W) (sum of the group's q heads)
         float a = 0.f, b = 0.f;
         for (int h = 0; h < D.G; ++h) {
             a += __bfloat162float(A.q[(hk * D.G + h) * DHD + tid]);
@@ -533,62 +540,90 @@ __device__ void score_item(const Dev& D, const StepArgs& A, int hk, int split, u
     __syncthreads();
     float qr[V];
     {
-        const int i0 = ((HALFROW ? piece : lane) * V) % DHD;
+        const int i0 = ((HALFROW ? lane & 15 : lane) * V) % DHD;
 #pragma unroll
         for (int x = 0; x < V; ++x) qr[x] = qb[i0 + x];
     }
+    const int half = lane >> 4, piece = lane & 15;
     uint64_t list = 0, cand = 0;
     int it = 0;
-    for (int u0 = u_begin + warp * UB; u0 < u_end; u0 += 4 * UB, ++it) {  // warp-uniform
-        if (it > 0) load(u0);
-        float acc[4];
+    for (int c = 0; c < nch; ++c) {
+        const int st = c % SSTAGES;
+        const bool ok = __syncthreads_and(ptx::mbar_wait(&sbar[st], (sph >> st) & 1u));
+        if (!ok) {  // the stage never landed: wait (bounded) for the copies in flight, then give up
+            if (tid == 0) {
+                set_err(D, ERR_TIMEOUT);
+                for (int cc = c + 1; cc < min(nch, c + SSTAGES); ++cc)
+                    ptx::mbar_wait(&sbar[cc % SSTAGES], (sph >> (cc % SSTAGES)) & 1u, 1ll << 28);
+            }
+            __syncthreads();
+            return false;
+        }
+        sph ^= 1u << st;
+        const uint4* base = reinterpret_cast<const uint4*>(ring + st * SBYTES);
+        const int u0c = u_begin + c * UPS, nu = min(UPS, u_end - u0c);
+        for (int g = warp; g * UB < nu; g += 4, ++it) {  // warp-uniform
+            uint4 raw[4][CPL];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            float a = 0.f;
+            for (int i = 0; i < 4; ++i)
 #pragma unroll
-            for (int c = 0; c < CPL; ++c) {
-                if (sizeof(E) == 2) {
-                    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw[i][c]);
+                for (int cc = 0; cc < CPL; ++cc) {
+                    const int u = HALFROW ? g * UB + 2 * i + half : g * UB + i;
+                    raw[i][cc] = u < nu ? (HALFROW ? base[u * 16 + piece] : base[u * 32 * CPL + cc * 32 + lane])
+                                        : make_uint4(0, 0, 0, 0);
+                }
+            float acc[4];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 f = __bfloat1622float2(h2[e]);
-                        a += f.x * qr[2 * e] + f.y * qr[2 * e + 1];
+            for (int i = 0; i < 4; ++i) {
+                float a = 0.f;
+#pragma unroll
+                for (int cc = 0; cc < CPL; ++cc) {
+                    if (sizeof(E) == 2) {
+                        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw[i][cc]);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 f = __bfloat1622float2(h2[e]);
+                            a += f.x * qr[2 * e] + f.y * qr[2 * e + 1];
+                        }
+                    } else {
+                        const float* f = reinterpret_cast<const float*>(&raw[i][cc]);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) a += f[e] * qr[e];
                     }
-                } else {
-                    const float* f = reinterpret_cast<const float*>(&raw[i][c]);
+                }
+                acc[i] = a;
+            }
+            // halving steps then a butterfly: full rows -- masks 16, 8 then 4, 2, 1 (lane l: unit l / 8);
+            // half rows -- masks 8, 4 then 2, 1 inside each half (lane l: unit 2 ((l / 4) % 4) + l / 16)
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) a += f[e] * qr[e];
+            for (int m = HALFROW ? 8 : 16, nv = 4; nv > 1; m >>= 1, nv >>= 1) {
+                const bool upper = (lane & m) != 0;
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    if (i < nv / 2) {
+                        const float send = upper ? acc[i] : acc[i + nv / 2];
+                        const float keep = upper ? acc[i + nv / 2] : acc[i];
+                        acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+                    }
                 }
             }
-            acc[i] = a;
-        }
-        // halving steps then a butterfly: full rows -- masks 16, 8 then 4, 2, 1 (lane l: unit l / 8);
-        // half rows -- masks 8, 4 then 2, 1 inside each half (lane l: unit 2 ((l / 4) % 4) + l / 16)
 #pragma unroll
-        for (int m = HALFROW ? 8 : 16, nv = 4; nv > 1; m >>= 1, nv >>= 1) {
-            const bool upper = (lane & m) != 0;
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                if (i < nv / 2) {
-                    const float send = upper ? acc[i] : acc[i + nv / 2];
-                    const float keep = upper ? acc[i + nv / 2] : acc[i];
-                    acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
-                }
+            for (int m = HALFROW ? 2 : 4; m >= 1; m >>= 1) acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], m);
+            const int jl = HALFROW ? g * UB + 2 * ((lane >> 2) & 3) + half : g * UB + lane / 8;
+            const int sub = HALFROW ? (lane & 3) : (lane & 7);
+            const float sc = acc[0] * D.inv_sqrt_d;
+            if (jl < nu) {
+                const int j = u0c + jl;
+                if (sub == 0) D.uscore[(int64_t)hk * D.units_max + j] = sc;
+                if (sub == it % GRP) cand = make_key(sc, (uint32_t)j);
+            }
+            if (it % GRP == GRP - 1) {
+                list = warp_topk_insert(list, cand);
+                cand = 0;
             }
         }
-#pragma unroll
-        for (int m = HALFROW ? 2 : 4; m >= 1; m >>= 1) acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], m);
-        const int j = HALFROW ? u0 + 2 * ((lane >> 2) & 3) + half : u0 + lane / 8;
-        const int sub = HALFROW ? (lane & 3) : (lane & 7);
-        const float sc = acc[0] * D.inv_sqrt_d;
-        if (j < u_end) {
-            if (sub == 0) D.uscore[(int64_t)hk * D.units_max + j] = sc;
-            if (sub == it % GRP) cand = make_key(sc, (uint32_t)j);
-        }
-        if (it % GRP == GRP - 1) {
-            list = warp_topk_insert(list, cand);
-            cand = 0;
-        }
+        __syncthreads();  // every warp is done with stage st
+        if (tid == 0 && c + SSTAGES < nch) issue(c + SSTAGES);
     }
     if (__any_sync(0xffffffffu, cand != 0)) list = warp_topk_insert(list, cand);
     lists[warp][lane] = list;
@@ -598,7 +633,9 @@ __device__ void score_item(const Dev& D, const StepArgs& A, int hk, int split, u
             lists[warp][lane] = warp_merge_desc(lists[warp][lane], lists[warp + stride][lane]);
     }
     __syncthreads();
-    publish_and_select(D, hk, split, A.nm, A.n_split, lists, 4, D.dflags + hk, A.tag);
+    publish_and_select(D, hk, split, A.nm, A.n_split, lists, 4, D.dflags + hk, A.tag,
+                       reinterpret_cast<uint64_t*>(ring), (int)(SSTAGES * SBYTES / 256));
+    return true;
 }
 
 // A whole decode step in one cooperative launch: every CTA is resident at once, and takes work items
@@ -620,6 +657,7 @@ __global__ void __launch_bounds__(DTHREADS) k_decode_step(const __grid_constant_
     const int tid = threadIdx.x;
     if (tid == 0) {
         ptx::mbar_init(bar, 1);
+        for (int s = 0; s < SSTAGES; ++s) ptx::mbar_init(reinterpret_cast<uint64_t*>(sm + OFF_SBAR) + s, 1);
         ptx::mbar_fence_init();
     }
     for (int i = tid; i < DHD / 2; i += DTHREADS) cs_t[i] = cs_abs(D.cs_abs3, D.half, A.t, i);
@@ -627,7 +665,7 @@ __global__ void __launch_bounds__(DTHREADS) k_decode_step(const __grid_constant_
     const int per_w = A.nst + A.nwt;
     const int NW = per_w * D.Hkv, NS = A.n_split * D.Hkv * (A.kk > 0), NU = A.nut * D.Hkv;
     const int total = NW + NS + NU;
-    uint32_t phase = 0;
+    uint32_t phase = 0, sph = 0;
     for (;;) {
         if (tid == 0) item_s = (int)(atomicAdd(D.dq, 1ull) - A.qbase);
         __syncthreads();
@@ -636,7 +674,7 @@ __global__ void __launch_bounds__(DTHREADS) k_decode_step(const __grid_constant_
         if (item >= total) break;
         if (item < NS + NW && item >= NW) {  // scoring
             const int it = item - NW;
-            score_item<E, ROWB>(D, A, it / A.n_split, it % A.n_split, sm);
+            if (!score_item<E, ROWB>(D, A, it / A.n_split, it % A.n_split, sm, sph)) break;
             continue;
         }
         int hk, ti, part;

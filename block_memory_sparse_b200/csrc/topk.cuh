@@ -9,6 +9,8 @@ namespace infllm {
 // the last scoring CTA of that head: warp w merges lists w, w + nw, ... (loads of a batch issued
 // together), then the warp lists are merged pairwise in shared memory; the k ids are written in
 // ascending order.  Ties go to the lower unit index.  Valid for k <= 32.
+static __device__ void finish_select(const Dev& D, int hk, int n_mem, uint64_t (*lists)[32], int nw, uint64_t m);
+
 static __device__ void merge_select(const Dev& D, int hk, int n_mem, int n_split, uint64_t (*lists)[32], int nw) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint64_t* cb = D.cand + (int64_t)hk * D.score_splits_max * 32 + lane;
@@ -24,6 +26,37 @@ static __device__ void merge_select(const Dev& D, int hk, int n_mem, int n_split
         for (int u = 0; u < 4; ++u)
             if (s0 + nw * u < n_split) m = warp_merge_desc(m, b[u]);
     }
+    finish_select(D, hk, n_mem, lists, nw, m);
+}
+
+// As merge_select, for a CTA that can lend `stage` (n_split x 32 keys of shared memory): every list
+// is first copied there in one batch of 16-byte asynchronous copies, so the lists cost one round trip
+// to L2, and each warp then merges its lists (w, w + nw, ...) in four independent chains, so that
+// consecutive merges do not wait for each other.
+static __device__ void merge_select_staged(const Dev& D, int hk, int n_mem, int n_split, uint64_t (*lists)[32], int nw,
+                                           uint64_t* stage) {
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint64_t* cb = D.cand + (int64_t)hk * D.score_splits_max * 32;
+    for (int x = tid; x < n_split * 16; x += nw * 32) cp_async16(stage + 2 * x, cb + 2 * x);
+    cp_async_wait_all();
+    __syncthreads();
+    uint64_t m0 = 0, m1 = 0, m2 = 0, m3 = 0;
+    int sp = warp;
+    for (; sp + 3 * nw < n_split; sp += 4 * nw) {  // four independent merges per pass
+        const uint64_t b0 = stage[sp * 32 + lane], b1 = stage[(sp + nw) * 32 + lane];
+        const uint64_t b2 = stage[(sp + 2 * nw) * 32 + lane], b3 = stage[(sp + 3 * nw) * 32 + lane];
+        m0 = warp_merge_desc(m0, b0);
+        m1 = warp_merge_desc(m1, b1);
+        m2 = warp_merge_desc(m2, b2);
+        m3 = warp_merge_desc(m3, b3);
+    }
+    for (; sp < n_split; sp += nw) m0 = warp_merge_desc(m0, stage[sp * 32 + lane]);
+    finish_select(D, hk, n_mem, lists, nw, warp_merge_desc(warp_merge_desc(m0, m1), warp_merge_desc(m2, m3)));
+}
+
+// The warps' merged lists -> the head's selection (k ids, ascending) in D.sel.
+static __device__ void finish_select(const Dev& D, int hk, int n_mem, uint64_t (*lists)[32], int nw, uint64_t m) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     __syncthreads();  // the caller's use of lists[] is over
     lists[warp][lane] = m;
     for (int stride = 1; stride < nw; stride *= 2) {
@@ -53,9 +86,11 @@ static __device__ void merge_select(const Dev& D, int hk, int n_mem, int n_split
 // This CTA's top-32 list of KV head hk goes to D.cand; the last CTA of the head to finish (device
 // counter, threadfence pattern: no CTA waits for another) merges all lists into the selection and
 // re-arms the counter for the next launch.  With `done_flag`, the merging CTA then publishes `tag`
-// there (release): a reader that acquires the tag sees the whole selection.
+// there (release): a reader that acquires the tag sees the whole selection.  With `stage` (room for
+// `stage_lists` lists in shared memory), the merge stages the lists there first.
 static __device__ void publish_and_select(const Dev& D, int hk, int split, int n_mem, int n_split,
-                                          uint64_t (*lists)[32], int nw, int* done_flag = nullptr, int tag = 0) {
+                                          uint64_t (*lists)[32], int nw, int* done_flag = nullptr, int tag = 0,
+                                          uint64_t* stage = nullptr, int stage_lists = 0) {
     __shared__ int is_last;
     if (threadIdx.x < 32) D.cand[((int64_t)hk * D.score_splits_max + split) * 32 + threadIdx.x] = lists[0][threadIdx.x];
     __threadfence();
@@ -64,7 +99,10 @@ static __device__ void publish_and_select(const Dev& D, int hk, int split, int n
     __syncthreads();
     if (!is_last) return;
     __threadfence();
-    merge_select(D, hk, n_mem, n_split, lists, nw);
+    if (stage && n_split <= stage_lists)
+        merge_select_staged(D, hk, n_mem, n_split, lists, nw, stage);
+    else
+        merge_select(D, hk, n_mem, n_split, lists, nw);
     if (done_flag) {
         __threadfence();  // each writer of the selection, before the CTA barrier
         __syncthreads();

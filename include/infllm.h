@@ -83,7 +83,9 @@ typedef struct {
     int32_t max_chunk;   /* largest n accepted by append/attend */
     int64_t max_tokens;  /* capacity of the token stream; max_tokens / unit_size + 1 <= 16384 units */
     double rope_base;    /* RoPE base (> 1) */
-    int32_t dtype;       /* infllm_dtype of q/k/v/out */
+    int32_t dtype;       /* infllm_dtype of q/k/v/out.  bf16 attention runs on the tcgen05 tensor
+                          * cores, which take Hq / Hkv dividing 128 and top_k <= 4096: other bf16
+                          * shapes are refused (EINVAL).  fp32 runs on the CUDA cores. */
     int32_t score_mode;  /* infllm_score_mode */
 } infllm_config;
 
@@ -95,7 +97,7 @@ typedef struct {
     int64_t window_base;     /* first window token of the last attended chunk */
     int64_t active_tokens;   /* keys attended by the last query of the last attended chunk */
     int64_t kernel_launches; /* kernels enqueued since create (or the last stats reset) */
-    int32_t attend_path;     /* chunk attention kernel in use: 0 = CUDA-core fp32, 1 = tcgen05 tensor cores */
+    int32_t attend_path;     /* chunk attention kernel: 0 = CUDA cores (fp32), 1 = tcgen05 tensor cores (bf16) */
     int32_t score_mode;      /* infllm_score_mode in use */
     /* filled when profiling is on (infllm_set_profiling), device times from CUDA events: */
     double ms_append, ms_reps, ms_prep, ms_select, ms_attend, ms_decode;
@@ -110,7 +112,8 @@ typedef struct infllm_ctx infllm_ctx; /* opaque */
  * later work.  The pools hold the three parts of the context that "InfLLM Guide: Training-Free
  * Long-Context Memory Units", "Core Innovation 1: Structured Context Partitioning", names:
  * initial (sink) tokens, memory units of unit_size tokens, and the local window.
- * Errors: EINVAL (cfg out of range, message on stderr), ECUDA (allocation failed).  On failure
+ * Errors: EINVAL (cfg out of range, or a bf16 shape the tensor-core kernel does not take; message
+ * on stderr), ECUDA (allocation failed).  On failure
  * *out is NULL and nothing stays allocated.  The caller owns the context until infllm_destroy. */
 infllm_status infllm_create(const infllm_config* cfg, void* cuda_stream, infllm_ctx** out);
 

@@ -57,8 +57,8 @@ def test_prefill_stream_matches_oracle(cuda_ok, name, score_mode):
         g = res[ci]
         nm = O.n_mem(c0, w.n_sink, w.window, w.unit_size)
         assert g["stats"]["n_mem"] == nm
-        # bf16 with d = 128 runs on the tcgen05 kernel; fp32 and d = 64 on the CUDA-core kernel
-        assert g["stats"]["attend_path"] == (1 if (w.dtype == "bf16" and w.head_dim == 128) else 0)
+        # bf16 runs on the tcgen05 kernel (d = 64 and 128); fp32 on the CUDA-core kernel
+        assert g["stats"]["attend_path"] == (1 if w.dtype == "bf16" else 0)
         # unit scores: oracle on the GPU's representatives
         if nm > 0 and w.top_k > 0:
             greps = glayer.reps(0, nm) if nm else None
@@ -241,15 +241,20 @@ def test_state_errors(cuda_ok):
     layer.close()
 
 
-def test_tensor_core_path_matches_cuda_core_path(cuda_ok, monkeypatch):
-    """Same stream through the tcgen05 kernel and the fp32 CUDA-core kernel (forced at create)."""
-    w = synth.SMALL["small_g4"].replace(chunk=512, n_tokens=4096)
-    tc_layer, tc = run_prefill(w)
-    monkeypatch.setenv("INFLLM_FORCE_SIMT", "1")
-    simt_layer, simt = run_prefill(w)
-    assert tc[0]["stats"]["attend_path"] == 1 and simt[0]["stats"]["attend_path"] == 0
-    for ci in tc:
-        assert tc[ci]["sel"].tolist() == simt[ci]["sel"].tolist()
-        assert np.max(np.abs(tc[ci]["out"] - simt[ci]["out"])) <= 2e-2
-    tc_layer.close()
-    simt_layer.close()
+def test_bf16_runs_on_the_tensor_cores_or_is_refused(cuda_ok):
+    """bf16 attention has one path, the tcgen05 kernel (head dim 64 or 128); a bf16 shape that it cannot
+    take is refused at create with EINVAL rather than run elsewhere.  fp32 runs on the CUDA cores."""
+    from block_memory_sparse_b200 import InfLLMError, InfLLMLayer
+    for name in ("small_d64", "small_g4"):
+        layer = make_layer(synth.SMALL[name], max_tokens=64)
+        assert layer.stats()["attend_path"] == 1, name
+        layer.close()
+    base = dict(n_q_heads=12, n_kv_heads=4, head_dim=64, n_sink=4, window=64, unit_size=16, n_reps=2, top_k=2,
+                max_chunk=64, max_tokens=256, rope_base=1e4)
+    for bad in (dict(), dict(n_q_heads=8, top_k=5000)):  # 3 q heads per KV head; too many selected units
+        with pytest.raises(InfLLMError) as e:
+            InfLLMLayer(**dict(base, **bad), dtype="bf16")
+        assert e.value.status == 1  # EINVAL
+    layer = InfLLMLayer(**base, dtype="f32")
+    assert layer.stats()["attend_path"] == 0
+    layer.close()
