@@ -431,6 +431,7 @@ infllm_status zero_state(infllm_ctx* c) {
     CK(cudaMemsetAsync(c->D.Y, 0, sizeof(float) * (size_t)((c->D.T_max / c->D.gblk) + 2) * c->D.Hkv * c->D.d, c->stream));
     CK(cudaMemsetAsync(c->D.counters, 0, sizeof(unsigned) * 4 * c->D.Hkv, c->stream));
     CK(cudaMemsetAsync(c->D.dflags, 0, sizeof(int) * 2 * c->D.Hkv, c->stream));
+    CK(cudaMemsetAsync(c->D.uflags, 0, sizeof(unsigned long long) * c->D.Hkv * std::max(1, c->D.topk), c->stream));
     CK(cudaMemsetAsync(c->D.dq, 0, sizeof(unsigned long long), c->stream));
     c->dq_base = 0;
     CK(cudaMemsetAsync(c->sel_base, 0xff, sizeof(int32_t) * 2 * (size_t)c->D.Hkv * std::max(1, c->D.topk), c->stream));
@@ -514,6 +515,7 @@ infllm_status create_impl(infllm_ctx* c) {
     AL(D.cand, sizeof(uint64_t) * (size_t)D.Hkv * D.score_splits_max * 32);
     AL(D.counters, sizeof(unsigned) * 4 * D.Hkv);
     AL(D.dflags, sizeof(int) * 2 * D.Hkv);
+    AL(D.uflags, sizeof(unsigned long long) * D.Hkv * std::max(1, D.topk));
     AL(D.dq, sizeof(unsigned long long));
     AL(D.Qm, (size_t)D.Hkv * 3 * D.qrows_max * D.d * c->elt);  // three slots
     AL(D.Qw, (size_t)D.Hkv * 3 * D.qrows_max * D.d * c->elt);

@@ -69,7 +69,9 @@ constexpr float RESCALE_LOG2 = 8.0f;
 constexpr int ERR_TIMEOUT = 16;
 
 struct Bars {
-    uint64_t q, kfull[NSTAGE], kempty[NSTAGE], vfull[NSTAGE], vempty[NSTAGE], sfull[2], pfull, pvdone;
+    // pfull and pvdone alternate by tile parity: P(i) is released on pfull[i & 1] and PV(i) completes on
+    // pvdone[i & 1], so that neither consumer can fall two phases behind one barrier (parity aliasing)
+    uint64_t q, kfull[NSTAGE], kempty[NSTAGE], vfull[NSTAGE], vempty[NSTAGE], sfull[2], pfull[2], pvdone[2];
     uint32_t tmem;
     int abort;
 };
@@ -193,7 +195,7 @@ __device__ void mma_issuer(const Plan& P, const Dev& D, uint8_t* sm, Bars* bars,
         }
         if (i >= 1) {
             const int j = i - 1, sj = j % NSTAGE, bj = j & 1;
-            if (!wait_bar(&bars->pfull, (uint32_t)j & 1, bars, D)) return;
+            if (!wait_bar(&bars->pfull[j & 1], (uint32_t)(j >> 1) & 1, bars, D)) return;
             if (!wait_bar(&bars->vfull[sj], (uint32_t)(j / NSTAGE) & 1, bars, D)) return;
             ptx::tc_fence_after();
             const uint32_t va = vb + sj * Y::TILE;
@@ -203,7 +205,7 @@ __device__ void mma_issuer(const Plan& P, const Dev& D, uint8_t* sm, Bars* bars,
                                  tmem + bj * BN + (uint32_t)(ks >> 2) * 64 + (uint32_t)(ks & 3) * 8,
                                  ptx::sdesc_sw128(va + (uint32_t)ks * 2048, SWB, 1024), IDESC_PV,
                                  (j > 0 || (ks & 3) > 0) ? 1u : 0u);
-            ptx::mma_commit(&bars->pvdone);
+            ptx::mma_commit(&bars->pvdone[j & 1]);
             ptx::mma_commit(&bars->vempty[sj]);
         }
     }
@@ -220,14 +222,15 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
-// PV completions are consumed strictly in order, and never more than one phase late: a parity
-// wait on an mbarrier that has completed two phases past the awaited one would wait for a third.
-// Tile i consumes PV(i - 1) before it releases P_i; PV(i) cannot have been issued by then.
+// PV completions are consumed strictly in order, PV(x) as phase x >> 1 of pvdone[x & 1], and never
+// two phases late on one barrier: a parity wait on an mbarrier that has completed two phases past
+// the awaited one would wait for a third.  Tile i consumes PV(i - 2) before it releases P_i, and
+// PV(i) is issued only after that release, so at most PV(i - 1) can be complete past it.
 struct PvTrack {
     int seen = 0;  // PV products known complete: tiles [0, seen)
     __device__ __forceinline__ bool upto(int j, Bars* bars, const Dev& D) {
         while (seen <= j) {
-            if (!warp_wait(&bars->pvdone, (uint32_t)seen & 1, bars, D)) return false;
+            if (!warp_wait(&bars->pvdone[seen & 1], (uint32_t)(seen >> 1) & 1, bars, D)) return false;
             ++seen;
         }
         return true;
@@ -323,14 +326,14 @@ __device__ void softmax_role(const Plan& P, const Dev& D, Bars* bars, float* lsu
         ptx::tmem_st32(sbase + half * 64, reinterpret_cast<const float*>(w));  // over this half's own S columns
         l += ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
         ptx::tmem_wait_st();
-        // PV(i - 1) ran during this tile's exponentials; consume its completion before P_i is
-        // released (PV(i) is issued only after the arrival below)
-        if (i >= 1 && !pv.upto(i - 1, bars, D)) {
+        // consume PV(i - 2) before P_i is released (PV(i) is issued only after the arrival below);
+        // PV(i - 1) may still run while this row goes on to tile i + 1
+        if (i >= 2 && !pv.upto(i - 2, bars, D)) {
             ok = false;
             break;
         }
         ptx::tc_fence_before();
-        ptx::mbar_arrive(&bars->pfull);
+        ptx::mbar_arrive(&bars->pfull[i & 1]);
     }
     ok = ok && pv.upto(P.NT - 1, bars, D);
     // the two halves of the row meet: O = (2^(m_0 - M) O_0 + 2^(m_1 - M) O_1) / (same weights on
@@ -409,9 +412,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             ptx::mbar_init(&bars->vfull[s], 1);
             ptx::mbar_init(&bars->vempty[s], 1);
         }
-        for (int b = 0; b < 2; ++b) ptx::mbar_init(&bars->sfull[b], 1);
-        ptx::mbar_init(&bars->pfull, NSOFT);
-        ptx::mbar_init(&bars->pvdone, 1);
+        for (int b = 0; b < 2; ++b) {
+            ptx::mbar_init(&bars->sfull[b], 1);
+            ptx::mbar_init(&bars->pfull[b], NSOFT);
+            ptx::mbar_init(&bars->pvdone[b], 1);
+        }
         bars->abort = 0;
         ptx::mbar_fence_init();
     }

@@ -38,6 +38,7 @@ struct Dev {
     unsigned* counters;   // [4][Hkv] arrival counters (last CTA done): unit selection, CUDA-core decode merge,
                           // tile decode part 0 and part 1
     int* dflags;          // [2][Hkv] decode-step flags (step tags): selection final, sinks and window merged
+    unsigned long long* uflags;  // [Hkv][topk] decode-step slot flags: (step tag << 32) | selected unit id
     unsigned long long* dq;  // decode-step work counter (monotonic; the host keeps each step's base)
     // rotated, packed queries of a chunk: [Hkv][3][qrows_max][d] (three slots, so later chunks'
     // queries can be packed while an earlier chunk's attention runs)
@@ -98,6 +99,14 @@ __device__ __forceinline__ void st_release(int* p, int v) {
 __device__ __forceinline__ int ld_acquire(const int* p) {
     int v;
     asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release64(unsigned long long* p, unsigned long long v) {
+    asm volatile("st.release.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ unsigned long long ld_acquire64(const unsigned long long* p) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
     return v;
 }
 

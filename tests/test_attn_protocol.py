@@ -10,7 +10,9 @@ interleaves at random, with exact mbarrier parity semantics.
 - TMA engine: lands copies in any order.
 - Two softmax threads: the two column halves of a row, each with its own online softmax. A
   half may rescale its accumulator O_h (only after PV(i - 1) is complete) and writes its half
-  of P(i) over its half of S(i).
+  of P(i) over its half of S(i); it releases P(i) once PV(i - 2) is complete, so PV(i - 1) can
+  run while it works on the next tile.  P releases and PV completions alternate between two
+  barriers each (by tile parity), which keeps every consumer within one phase of its barrier.
 
 Every data hand-off is asserted where it happens:
 - a ring slot is refilled only after the MMA that read it has executed;
@@ -56,7 +58,7 @@ class Bar:
 
 def run(NT, seed, plant=None):
     rnd = random.Random(seed)
-    bars = {"q": Bar("q", 1), "pfull": Bar("pfull", 2), "pvdone": Bar("pvdone", 1),
+    bars = {"q": Bar("q", 1), "pfull0": Bar("pfull0", 2), "pfull1": Bar("pfull1", 2), "pvdone0": Bar("pvdone0", 1), "pvdone1": Bar("pvdone1", 1),
             "sfull0": Bar("sfull0", 1), "sfull1": Bar("sfull1", 1)}
     for s in range(NSTAGE):
         for x in ("kfull", "kempty", "vfull", "vempty"):
@@ -118,10 +120,10 @@ def run(NT, seed, plant=None):
                 yield
             if i >= 1:
                 j = i - 1
-                yield from wait("pfull", j)
+                yield from wait(f"pfull{j & 1}", j >> 1)
                 if plant != "pv_skips_v_wait":
                     yield from wait(f"vfull{j % NSTAGE}", j // NSTAGE)
-                pipe.extend([("pv", j), ("commit", "pvdone"), ("commit", f"vempty{j % NSTAGE}")])
+                pipe.extend([("pv", j), ("commit", f"pvdone{j & 1}"), ("commit", f"vempty{j % NSTAGE}")])
                 yield
 
     def tensor_pipe():
@@ -152,9 +154,9 @@ def run(NT, seed, plant=None):
     def softmax(h):
         seen = [0]  # PV completions consumed: tiles [0, seen)
 
-        def upto(j):
+        def upto(j):  # PV(x) completes phase x >> 1 of pvdone[x & 1]
             while seen[0] <= j:
-                yield from wait("pvdone", seen[0])
+                yield from wait(f"pvdone{seen[0] & 1}", seen[0] >> 1)
                 seen[0] += 1
 
         for i in range(NT):
@@ -169,9 +171,12 @@ def run(NT, seed, plant=None):
             S[b][1].add(h)
             P[b][h] = i  # over this half's own S columns (it has read them; the partner never does)
             yield
-            if i >= 1 and plant != "release_without_pv_wait":
-                yield from upto(i - 1)
-            bars["pfull"].arrive()
+            # PV(i - 2) is consumed before P(i) is released: PV(i) is issued only after the release, so
+            # the barrier is then at most one phase ahead of this consumer (no parity aliasing), and
+            # PV(i - 1) may still run while this half works on tile i + 1
+            if i >= 2 and plant != "release_without_pv_wait":
+                yield from upto(i - 2)
+            bars[f"pfull{i & 1}"].arrive()
             yield
         yield from upto(NT - 1)
         assert pv_done == list(range(NT)), f"half {h} read O with PVs done {pv_done}"
@@ -218,7 +223,7 @@ def test_model_matches_kernel_source():
     for each of the tensor-pipe barriers."""
     src = open(KERNEL).read()
     assert int(re.search(r"constexpr int NSTAGE = (\d+);", src).group(1)) == NSTAGE
-    for init in ("mbar_init(&bars->q, 1)", "mbar_init(&bars->pfull, NSOFT)", "mbar_init(&bars->pvdone, 1)",
+    for init in ("mbar_init(&bars->q, 1)", "mbar_init(&bars->pfull[b], NSOFT)", "mbar_init(&bars->pvdone[b], 1)",
                  "mbar_init(&bars->sfull[b], 1)", "mbar_init(&bars->kfull[s], 1)", "mbar_init(&bars->vempty[s], 1)"):
         assert init in src, init
     # the two halves of a row never wait for each other inside the tile loop (no exchange barrier)
