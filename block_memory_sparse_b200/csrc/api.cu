@@ -58,8 +58,6 @@ struct infllm_ctx {
     // writes its selection to buffer L % 2 (so a lookup can run while the previous attention reads)
     int64_t nlook = 0;
     int last_sel = 0;   // selection buffer of the last attended chunk or token
-    unsigned long long dq_base = 0;  // the decode-step work counter's value at the next step's start
-    bool step_coop = true;           // decode steps in one cooperative launch (else three chained launches)
     int32_t* sel_base = nullptr;
     float* qbar_base = nullptr;
     // profiling
@@ -363,23 +361,7 @@ infllm_status decode_impl(infllm_ctx* c, const void* q, const void* k, const voi
         const int nm = (int)n_mem_at(t, D.S, D.W, D.U);
         const int kk = std::min(D.topk, nm);
         const int64_t B = (int64_t)D.S + (int64_t)D.U * nm;
-        if (c->step_coop) {
-            // the whole step (store, sinks and window, lookup, units, merges) in one cooperative launch
-            Prof p(c, K_DECODE);
-            unsigned long long used = 0;
-            cudaError_t e = launch_decode_step(D, q, k, v, t, kk, B, nm, c->cfg.score_mode, (int)(L + 1), c->dq_base, out,
-                                               c->stream, c->tmaps, &used);
-            if (e != cudaSuccess) return fail(c, INFLLM_ECUDA, "decode step launch: %s", cudaGetErrorString(e));
-            c->dq_base += used;
-            c->chain = true;
-            p.done();
-            c->launches += 1;
-            c->tokens = t + 1;
-            c->pending = false;
-            record_attend(c, L, t, 1, nm, kk, B);
-            return INFLLM_OK;
-        }
-        {   // three chained launches: part 0, the lookup alongside it, part 1
+        {
             Prof p(c, K_DECODE);
             cudaError_t e = launch_decode_tc(D, q, k, v, t, kk, B, 0, out, c->stream, c->tmaps, pdl_ok(c));
             if (e != cudaSuccess) return fail(c, INFLLM_ECUDA, "decode launch (store, sinks, window): %s", cudaGetErrorString(e));
@@ -430,10 +412,6 @@ infllm_status decode_impl(infllm_ctx* c, const void* q, const void* k, const voi
 infllm_status zero_state(infllm_ctx* c) {
     CK(cudaMemsetAsync(c->D.Y, 0, sizeof(float) * (size_t)((c->D.T_max / c->D.gblk) + 2) * c->D.Hkv * c->D.d, c->stream));
     CK(cudaMemsetAsync(c->D.counters, 0, sizeof(unsigned) * 4 * c->D.Hkv, c->stream));
-    CK(cudaMemsetAsync(c->D.dflags, 0, sizeof(int) * 2 * c->D.Hkv, c->stream));
-    CK(cudaMemsetAsync(c->D.uflags, 0, sizeof(unsigned long long) * c->D.Hkv * std::max(1, c->D.topk), c->stream));
-    CK(cudaMemsetAsync(c->D.dq, 0, sizeof(unsigned long long), c->stream));
-    c->dq_base = 0;
     CK(cudaMemsetAsync(c->sel_base, 0xff, sizeof(int32_t) * 2 * (size_t)c->D.Hkv * std::max(1, c->D.topk), c->stream));
     c->tokens = 0;
     c->units_done = 0;
@@ -514,9 +492,6 @@ infllm_status create_impl(infllm_ctx* c) {
     AL(D.qbar_part, sizeof(float) * 2 * (size_t)D.Hkv * D.qtiles_max * D.d);  // two buffers
     AL(D.cand, sizeof(uint64_t) * (size_t)D.Hkv * D.score_splits_max * 32);
     AL(D.counters, sizeof(unsigned) * 4 * D.Hkv);
-    AL(D.dflags, sizeof(int) * 2 * D.Hkv);
-    AL(D.uflags, sizeof(unsigned long long) * D.Hkv * std::max(1, D.topk));
-    AL(D.dq, sizeof(unsigned long long));
     AL(D.Qm, (size_t)D.Hkv * 3 * D.qrows_max * D.d * c->elt);  // three slots
     AL(D.Qw, (size_t)D.Hkv * 3 * D.qrows_max * D.d * c->elt);
     AL(D.cs_chunk, sizeof(float2) * (size_t)g.max_chunk * D.half);
@@ -562,7 +537,6 @@ infllm_status create_impl(infllm_ctx* c) {
     *c->err_host = 0;
     CK(cudaHostGetDevicePointer((void**)&D.err, c->err_host, 0));
     c->use_tc = false;
-    c->step_coop = getenv("INFLLM_DECODE_CHAIN") == nullptr;
     if (g.dtype == INFLLM_BF16) {
         if (!attend_tc_supported(D))
             return fail(c, INFLLM_EINVAL, "bf16 needs the tensor-core attention: head_dim 64 or 128, "

@@ -37,9 +37,6 @@ struct Dev {
     uint64_t* cand;       // [Hkv][score_splits_max][32] top-k candidate lists
     unsigned* counters;   // [4][Hkv] arrival counters (last CTA done): unit selection, CUDA-core decode merge,
                           // tile decode part 0 and part 1
-    int* dflags;          // [2][Hkv] decode-step flags (step tags): selection final, sinks and window merged
-    unsigned long long* uflags;  // [Hkv][topk] decode-step slot flags: (step tag << 32) | selected unit id
-    unsigned long long* dq;  // decode-step work counter (monotonic; the host keeps each step's base)
     // rotated, packed queries of a chunk: [Hkv][3][qrows_max][d] (three slots, so later chunks'
     // queries can be packed while an earlier chunk's attention runs)
     void* Qm;             // R(W) q  (sink / memory frame)
@@ -91,24 +88,6 @@ enum ErrBits : int {
 };
 
 __device__ __forceinline__ void set_err(const Dev& D, int bit) { atomicOr(D.err, bit); }
-
-// Release store / acquire load of a GPU-scope flag (kernels that hand a result to other CTAs).
-__device__ __forceinline__ void st_release(int* p, int v) {
-    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-__device__ __forceinline__ int ld_acquire(const int* p) {
-    int v;
-    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-__device__ __forceinline__ void st_release64(unsigned long long* p, unsigned long long v) {
-    asm volatile("st.release.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
-__device__ __forceinline__ unsigned long long ld_acquire64(const unsigned long long* p) {
-    unsigned long long v;
-    asm volatile("ld.acquire.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-    return v;
-}
 
 // ---- element conversions --------------------------------------------------------------
 template <typename T> __device__ __forceinline__ float to_f(T x);

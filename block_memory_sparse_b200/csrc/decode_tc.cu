@@ -154,11 +154,22 @@ __device__ void merge_partials(const Dev& D, int hk, int ns, SlotOf slot_of, flo
             }
         }
         __syncthreads();
+        // the batch's weighted sum for every q head at once: one independent chain per head, so the
+        // slots' loads and multiply-adds of different heads overlap
+        float acc[MAXG];
+#pragma unroll
+        for (int h = 0; h < MAXG; ++h) acc[h] = 0.f;
+#pragma unroll 2
+        for (int sl = 0; sl < nr; ++sl) {
+            const float* srow = sbuf + sl * sf + 4 + tid;
+#pragma unroll
+            for (int h = 0; h < MAXG; ++h)
+                if (h < G) acc[h] = fmaf(wts[h][sl], srow[h * PST], acc[h]);
+        }
 #pragma unroll
         for (int h = 0; h < MAXG; ++h) {
             if (h >= G) continue;
-            float o = 0.f;
-            for (int sl = 0; sl < nr; ++sl) o = fmaf(wts[h][sl], sbuf[sl * sf + h * PST + 4 + tid], o);
+            const float o = acc[h];
             const float mb = stat[h][0], lb = stat[h][1];
             if (mb == -INFINITY) continue;
             if (mb > M[h]) {  // rescale the running totals to the larger max
@@ -451,381 +462,9 @@ __global__ void __launch_bounds__(DTHREADS, 1) k_decode_attn(const __grid_consta
     if (part == 0) pdl_hold();
 }
 
-// ---- one decode step in one cooperative launch ------------------------------------------------
-
-// Per-step arguments of k_decode_step.
-struct StepArgs {
-    const __nv_bfloat16* q;
-    const __nv_bfloat16* k;
-    const __nv_bfloat16* v;
-    __nv_bfloat16* out;
-    int64_t t, B;
-    unsigned long long qbase;  // value of the context's work counter when this step's unit tiles start
-    int kk, nm, nst, nwt, nut;  // selected units, eligible units, sink / window / unit tiles per head
-    int mode, tag;              // scoring operand; this step's flag value (> every earlier step's)
-    // Static partition of the scoring rows (units of all heads, head-major: N = Hkv nm) over the first
-    // gs CTAs.  weighted: CTA c < nw_cta also loads a window tile worth wr rows, so the ranges balance
-    // rows + window rows: range start = floor(c T / gs) - wr min(c, nw_cta), T = N + nw_cta wr;
-    // otherwise start = floor(c N / gs).
-    int64_t N, T;
-    int gs, weighted, wr, nw_cta;
-};
-
-// Start of CTA c's scoring range (flat unit index; N for c >= gs).  Non-decreasing in c, and strictly
-// increasing over [0, gs] (the host checks the weighted split's rows per CTA exceed a window tile's).
-__host__ __device__ __forceinline__ int64_t score_f0(const StepArgs& A, int c) {
-    if (c >= A.gs) return A.N;
-    if (A.weighted) {
-        const int64_t r = (int64_t)c * A.T / A.gs - (int64_t)A.wr * (c < A.nw_cta ? c : A.nw_cta);
-        return r < 0 ? 0 : (r > A.N ? A.N : r);
-    }
-    return (int64_t)c * A.N / A.gs;
-}
-// The CTA whose scoring range holds flat unit f (0 <= f < N): the largest c < gs with score_f0(c) <= f.
-__host__ __device__ __forceinline__ int score_owner(const StepArgs& A, int64_t f) {
-    int lo = 0, hi = A.gs - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (score_f0(A, mid) <= f) lo = mid;
-        else hi = mid - 1;
-    }
-    return lo;
-}
-
-// Bounded wait (one thread) for a flag another CTA of this grid sets to `tag` with a release store.
-__device__ __forceinline__ bool wait_flag(const Dev& D, const int* flag, int tag) {
-    if (ld_acquire(flag) == tag) return true;
-    const long long t0 = clock64();
-    while (ld_acquire(flag) != tag) {
-        if (clock64() - t0 > (1ll << 32)) {  // ~2 s: something is broken; give up cleanly
-            set_err(D, ERR_TIMEOUT);
-            return false;
-        }
-        __nanosleep(100);
-    }
-    return true;
-}
-
-// Scoring rows stream through a ring of SSTAGES bulk copies of SBYTES each, in the K and V tiles'
-// shared memory; each stage has its own mbarrier after the tile barrier.  The rest of the tiles'
-// space stages the candidate lists of a head's selection (LSTAGE lists at a time).
-constexpr int SSTAGES = 3;
-constexpr uint32_t SBYTES = 16384;
-constexpr int OFF_LSTAGE = OFF_K + SSTAGES * (int)SBYTES;
-constexpr int LSTAGE = (int)((2 * DTILE - SSTAGES * SBYTES) / 256);
-static_assert(LSTAGE >= 32, "no room to stage the candidate lists");
-constexpr int OFF_SBAR = OFF_MISC + 16;
-static_assert(16 + SSTAGES * 8 <= 64, "stage barriers overflow their slot");
-// after the (cos, sin) table: the scoring query R(W) (sum of the group's q heads) of every KV head
-constexpr int OFF_QB = OFF_CS + (DHD / 2) * 8;
-__host__ __device__ constexpr int step_smem(int hkv) { return OFF_QB + hkv * DHD * 4 + 1024; }
-
-// Scoring rows of flat unit f (head f / nm, unit f % nm) in the pool of the step's score mode.
-template <int ROWB>
-__device__ __forceinline__ const uint8_t* score_row(const Dev& D, const StepArgs& A, int64_t f) {
-    const uint8_t* pool = A.mode == OP_REPS ? (const uint8_t*)D.rep_keys
-                          : A.mode == OP_REPSUM ? (const uint8_t*)D.repsum
-                                                : (const uint8_t*)D.meankey;
-    return pool + ((f / A.nm) * D.units_max + f % A.nm) * ROWB;
-}
-// Units in the chunk that starts at flat unit f of a range ending at f1: at most a stage, and never
-// across a head boundary (the heads' rows are not contiguous in the pool).
-template <int ROWB>
-__device__ __forceinline__ int chunk_units(const StepArgs& A, int64_t f, int64_t f1) {
-    constexpr int UPS = (int)SBYTES / ROWB;
-    const int64_t seg_end = min(f1, (f / A.nm + 1) * A.nm);
-    return (int)min((int64_t)UPS, seg_end - f);
-}
-
-// Unit scores of this CTA's scoring range [f0, f1) of flat units (rows of ROWB bytes of E elements),
-// streamed through the ring: thread 0 keeps SSTAGES bulk copies in flight from the first chunk to
-// the last, across head boundaries.  The CTA's four warps score each stage from shared memory: a
-// warp takes 4 units per step for 512- and 1024-byte rows, 8 units for 256-byte rows (consecutive
-// lanes read consecutive 16 bytes), reduces each unit's dot product with the head's scoring query by
-// a transpose-reduce and keeps a top-32 list.  At the end of each head's part of the range the CTA's
-// list is published (part index = this CTA minus the head's first scoring CTA); the head's last CTA
-// to publish selects the head's units and publishes them slot by slot.  `sph` holds the stage
-// barriers' parities.  Returns false (error word set, copies in flight waited for) if a stage never
-// arrived.
-template <typename E, int ROWB>
-__device__ bool score_range(const Dev& D, const StepArgs& A, int64_t f0, int64_t f1, uint8_t* sm, uint32_t& sph) {
-    auto lists = reinterpret_cast<uint64_t(*)[32]>(sm + OFF_Q);  // [4][32]
-    uint64_t* sbar = reinterpret_cast<uint64_t*>(sm + OFF_SBAR);
-    constexpr int V = 16 / sizeof(E);
-    constexpr int HALFROW = ROWB == 256;
-    constexpr int CPL = HALFROW ? 1 : ROWB / 512;
-    constexpr int UB = HALFROW ? 8 : 4;  // units per warp step
-    constexpr int GRP = 32 / (HALFROW ? 8 : 4);
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    int64_t fi = f0;  // thread 0: next flat unit to put in flight
-    int ki = 0;       // thread 0: chunks put in flight
-    auto issue_next = [&]() {
-        if (fi >= f1) return;
-        const int n = chunk_units<ROWB>(A, fi, f1);
-        uint64_t* bar = &sbar[ki % SSTAGES];
-        ptx::mbar_expect_tx(bar, (uint32_t)(n * ROWB));
-        ptx::bulk_load(sm + OFF_K + (ki % SSTAGES) * SBYTES, score_row<ROWB>(D, A, fi), (uint32_t)(n * ROWB), bar);
-        fi += n;
-        ++ki;
-    };
-    // the ring overwrites shared memory that the generic proxy wrote (a tile's partial sums, a merge's
-    // copies); their use is over past the barrier
-    ptx::fence_proxy_async_smem();
-    __syncthreads();
-    if (tid == 0)
-        for (int c = 0; c < SSTAGES; ++c) issue_next();
-    const int half = lane >> 4, piece = lane & 15;
-    float qr[V];
-    int hk = -1;
-    uint64_t list = 0, cand = 0;
-    int it = 0;
-    int k = 0;
-    for (int64_t fc = f0; fc < f1; ++k) {
-        if (fc / A.nm != hk) {  // a new head's part of the range: its scoring query
-            hk = (int)(fc / A.nm);
-            const int i0 = ((HALFROW ? piece : lane) * V) % DHD;
-            const float* qb = reinterpret_cast<const float*>(sm + OFF_QB) + hk * DHD;
-#pragma unroll
-            for (int x = 0; x < V; ++x) qr[x] = qb[i0 + x];
-        }
-        const int st = k % SSTAGES;
-        const bool ok = __syncthreads_and(ptx::mbar_wait(&sbar[st], (sph >> st) & 1u));
-        if (!ok) {  // the stage never landed: wait (bounded) for the copies in flight, then give up
-            if (tid == 0) {
-                set_err(D, ERR_TIMEOUT);
-                for (int k2 = k + 1; k2 < ki; ++k2)  // at most SSTAGES - 1, each in its own stage
-                    ptx::mbar_wait(&sbar[k2 % SSTAGES], (sph >> (k2 % SSTAGES)) & 1u, 1ll << 28);
-            }
-            __syncthreads();
-            return false;
-        }
-        sph ^= 1u << st;
-        const uint4* base = reinterpret_cast<const uint4*>(sm + OFF_K + st * SBYTES);
-        const int u0c = (int)(fc % A.nm), nu = chunk_units<ROWB>(A, fc, f1);
-        for (int g = warp; g * UB < nu; g += 4, ++it) {  // warp-uniform
-            uint4 raw[4][CPL];
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int cc = 0; cc < CPL; ++cc) {
-                    const int u = HALFROW ? g * UB + 2 * i + half : g * UB + i;
-                    raw[i][cc] = u < nu ? (HALFROW ? base[u * 16 + piece] : base[u * 32 * CPL + cc * 32 + lane])
-                                        : make_uint4(0, 0, 0, 0);
-                }
-            float acc[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                float a = 0.f;
-#pragma unroll
-                for (int cc = 0; cc < CPL; ++cc) {
-                    if (sizeof(E) == 2) {
-                        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw[i][cc]);
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float2 f = __bfloat1622float2(h2[e]);
-                            a += f.x * qr[2 * e] + f.y * qr[2 * e + 1];
-                        }
-                    } else {
-                        const float* f = reinterpret_cast<const float*>(&raw[i][cc]);
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) a += f[e] * qr[e];
-                    }
-                }
-                acc[i] = a;
-            }
-            // halving steps then a butterfly: full rows -- masks 16, 8 then 4, 2, 1 (lane l: unit l / 8);
-            // half rows -- masks 8, 4 then 2, 1 inside each half (lane l: unit 2 ((l / 4) % 4) + l / 16)
-#pragma unroll
-            for (int m = HALFROW ? 8 : 16, nv = 4; nv > 1; m >>= 1, nv >>= 1) {
-                const bool upper = (lane & m) != 0;
-#pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    if (i < nv / 2) {
-                        const float send = upper ? acc[i] : acc[i + nv / 2];
-                        const float keep = upper ? acc[i + nv / 2] : acc[i];
-                        acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
-                    }
-                }
-            }
-#pragma unroll
-            for (int m = HALFROW ? 2 : 4; m >= 1; m >>= 1) acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], m);
-            const int jl = HALFROW ? g * UB + 2 * ((lane >> 2) & 3) + half : g * UB + lane / 8;
-            const int sub = HALFROW ? (lane & 3) : (lane & 7);
-            const float sc = acc[0] * D.inv_sqrt_d;
-            if (jl < nu) {
-                const int j = u0c + jl;
-                if (sub == 0) D.uscore[(int64_t)hk * D.units_max + j] = sc;
-                if (sub == it % GRP) cand = make_key(sc, (uint32_t)j);
-            }
-            if (it % GRP == GRP - 1) {
-                list = warp_topk_insert(list, cand);
-                cand = 0;
-            }
-        }
-        __syncthreads();  // every warp is done with stage st
-        if (tid == 0) issue_next();
-        fc += nu;
-        if (fc == f1 || fc % A.nm == 0) {  // the end of this head's part: publish the CTA's list
-            if (__any_sync(0xffffffffu, cand != 0)) list = warp_topk_insert(list, cand);
-            lists[warp][lane] = list;
-            for (int stride = 1; stride < 4; stride *= 2) {
-                __syncthreads();
-                if ((warp % (2 * stride)) == 0 && warp + stride < 4)
-                    lists[warp][lane] = warp_merge_desc(lists[warp][lane], lists[warp + stride][lane]);
-            }
-            __syncthreads();
-            const int c_first = score_owner(A, (int64_t)hk * A.nm);
-            const int c_last = score_owner(A, (int64_t)(hk + 1) * A.nm - 1);
-            publish_and_select(D, hk, (int)blockIdx.x - c_first, A.nm, c_last - c_first + 1, lists, 4, D.uflags,
-                               (unsigned)A.tag, reinterpret_cast<uint64_t*>(sm + OFF_LSTAGE), LSTAGE);
-            list = cand = 0;
-            it = 0;
-        }
-    }
-    return true;
-}
-
-// Bounded wait (one thread) for selected slot `slot` of KV head hk: returns the unit id, or -1 (error
-// word set) if the slot is not published within ~2 s.
-__device__ __forceinline__ int wait_slot(const Dev& D, int hk, int slot, unsigned tag) {
-    const unsigned long long* f = D.uflags + hk * D.topk + slot;
-    unsigned long long v = ld_acquire64(f);
-    if ((unsigned)(v >> 32) != tag) {
-        const long long t0 = clock64();
-        while ((unsigned)((v = ld_acquire64(f)) >> 32) != tag) {
-            if (clock64() - t0 > (1ll << 32)) {
-                set_err(D, ERR_TIMEOUT);
-                return -1;
-            }
-            __nanosleep(64);
-        }
-    }
-    return (int)(uint32_t)v;
-}
-
-// One tile of the step's working context into its partial slot; the head's last tile of its part
-// (arrival counter, re-armed by it) returns true.
-__device__ __forceinline__ bool tile_and_count(const TcMaps& maps, const Dev& D, const StepArgs& A, int hk, int ti,
-                                               int part, const DTile& T, uint8_t* sm, uint32_t& phase, int* sflag) {
-    tile_partial(maps, D, A.q, A.k, A.v, A.t, hk, ti, T, part == 0 && A.t >= T.y0 && A.t < T.y0 + T.nv, sm, phase);
-    __threadfence();
-    __syncthreads();
-    unsigned* ctr = D.counters + (2 + part) * D.Hkv + hk;
-    const int nblocks = part == 0 ? A.nst + A.nwt : A.nut;
-    if (threadIdx.x == 0) {
-        *sflag = atomicAdd(ctr, 1u) == (unsigned)(nblocks - 1);
-        if (*sflag) *ctr = 0u;  // re-armed for the next step (every arrival of this step is in)
-    }
-    __syncthreads();
-    const bool last = *sflag != 0;
-    if (last) __threadfence();
-    return last;
-}
-
-// The merged sinks and window of KV head hk (its last window tile's CTA): into the merged slot,
-// published on the head's window flag, or straight into the output when no unit is selected.
-__device__ __forceinline__ void window_merge(const Dev& D, const StepArgs& A, int hk, uint8_t* sm) {
-    merge_part(D, hk, 0, A.nst, A.nut, A.nwt, A.kk, sm, A.out);
-    if (A.kk > 0) {
-        __threadfence();
-        __syncthreads();
-        if (threadIdx.x == 0) st_release(D.dflags + D.Hkv + hk, A.tag);
-    }
-    __syncthreads();
-}
-
-// A whole decode step in one cooperative launch (every CTA resident at once).  CTA c, in order:
-//   1. window items c, c + grid, ...: the sink and window tiles of every KV head (the tile holding
-//      token t stores it first); the head's last one merges them -- after its scoring (step 3), when
-//      the grid covers every window tile, so that the merge's round trips do not delay its range;
-//   2. its static range of the scoring rows (score_range): the unit scores, its lists, and for each
-//      head the selection by the head's last CTA, published slot by slot with the unit ids;
-//   3. the deferred window merges, published on the head's window flag;
-//   4. unit tiles claimed from the context's counter: each waits (bounded) for its slot's flag; the
-//      head's last one waits (bounded) for the window flag and merges everything into the output.
-// Steps 1-3 wait for nothing, and the unit tiles wait only for them, so every wait ends.  The scoring
-// ranges are balanced by rows plus window-tile rows (StepArgs), so all CTAs stream until about the
-// same time and every byte is requested early.
-template <typename E, int ROWB>
-__global__ void __launch_bounds__(DTHREADS, 3) k_decode_step(const __grid_constant__ TcMaps maps, Dev D, StepArgs A) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + OFF_MISC);
-    float2* cs_t = reinterpret_cast<float2*>(sm + OFF_CS);
-    float* qball = reinterpret_cast<float*>(sm + OFF_QB);
-    __shared__ int next_s, flag_s;
-    const int tid = threadIdx.x, c = blockIdx.x, grid = gridDim.x;
-    const int per_w = A.nst + A.nwt;
-    const int NW = per_w * D.Hkv, NU = A.nut * D.Hkv;
-    if (tid == 0) {
-        ptx::mbar_init(bar, 1);
-        for (int s = 0; s < SSTAGES; ++s) ptx::mbar_init(reinterpret_cast<uint64_t*>(sm + OFF_SBAR) + s, 1);
-        ptx::mbar_fence_init();
-    }
-    for (int i = tid; i < DHD / 2; i += DTHREADS) cs_t[i] = cs_abs(D.cs_abs3, D.half, A.t, i);
-    for (int x = tid; x < D.Hkv * (DHD / 2); x += DTHREADS) {  // R(W) of the summed group query, per KV head
-        const int hk = x / (DHD / 2), i = x % (DHD / 2);
-        float a = 0.f, b = 0.f;
-        for (int h = 0; h < D.G; ++h) {
-            a += __bfloat162float(A.q[(hk * D.G + h) * DHD + i]);
-            b += __bfloat162float(A.q[(hk * D.G + h) * DHD + i + DHD / 2]);
-        }
-        const float2 cw = D.cs_W[i];
-        qball[hk * DHD + i] = a * cw.x - b * cw.y;
-        qball[hk * DHD + i + DHD / 2] = b * cw.x + a * cw.y;
-    }
-    __syncthreads();
-    uint32_t phase = 0, sph = 0;
-    int deferred = -1;  // KV head whose window merge waits for step 3
-    // 1. window tiles
-    for (int w = c; w < NW; w += grid) {
-        const int hk = w / per_w, wi = w % per_w;
-        const int ti = wi < A.nst ? wi : wi + A.nut;
-        const DTile T = decode_tile(D, hk, ti, A.t, A.kk, A.B);
-        if (tile_and_count(maps, D, A, hk, ti, 0, T, sm, phase, &flag_s)) {
-            if (grid >= NW && A.kk > 0) deferred = hk;
-            else window_merge(D, A, hk, sm);
-        }
-    }
-    // 2. scoring range
-    if (A.kk > 0) {
-        const int64_t f0 = score_f0(A, c), f1 = score_f0(A, c + 1);
-        if (f0 < f1 && !score_range<E, ROWB>(D, A, f0, f1, sm, sph)) return;  // error word set
-    }
-    // 3. deferred window merge
-    if (deferred >= 0) window_merge(D, A, deferred, sm);
-    // 4. unit tiles
-    if (tid == 32) next_s = (int)(atomicAdd(D.dq, 1ull) - A.qbase);
-    __syncthreads();
-    const int tpu = (D.U + DK - 1) / DK;
-    for (;;) {
-        const int item = next_s;
-        __syncthreads();
-        if (item >= NU) break;
-        if (tid == 32) next_s = (int)(atomicAdd(D.dq, 1ull) - A.qbase);  // the next claim overlaps this item
-        const int hk = item / A.nut, ui = item % A.nut;
-        const int ti = A.nst + ui, pt = ui % tpu;
-        if (tid == 0) flag_s = wait_slot(D, hk, ui / tpu, (unsigned)A.tag);  // the slot's unit
-        __syncthreads();
-        const int id = flag_s;
-        DTile T{1, 0, 0};
-        if (id >= 0 && (int64_t)D.S + (int64_t)(id + 1) * D.U <= A.B)
-            T = DTile{1, (int64_t)D.S + (int64_t)id * D.U + (int64_t)pt * DK, min(DK, D.U - pt * DK)};
-        else if (id >= 0 && tid == 0)
-            set_err(D, ERR_SEL_RANGE);
-        if (!tile_and_count(maps, D, A, hk, ti, 1, T, sm, phase, &flag_s)) continue;
-        if (tid == 0) flag_s = wait_flag(D, D.dflags + D.Hkv + hk, A.tag);  // the merged sinks and window
-        __syncthreads();
-        merge_part(D, hk, 1, A.nst, A.nut, A.nwt, A.kk, sm, A.out);
-        __syncthreads();
-    }
-}
-
 }  // namespace
 
-constexpr int STEP_HKV_MAX = 64;  // KV heads the one-launch step keeps scoring queries for
-
-bool decode_tc_supported(const Dev& D) { return D.d == DHD && D.G <= MAXG && D.topk <= 32 && D.Hkv <= STEP_HKV_MAX; }
+bool decode_tc_supported(const Dev& D) { return D.d == DHD && D.G <= MAXG && D.topk <= 32; }
 
 cudaError_t launch_decode_tc(const Dev& D, const void* q, const void* k, const void* v, int64_t t, int kk, int64_t B,
                              int part, void* out, cudaStream_t st, const void* tmaps, bool pdl) {
@@ -841,95 +480,6 @@ cudaError_t launch_decode_tc(const Dev& D, const void* q, const void* k, const v
     return launch_k(k_decode_attn, dim3(tiles, D.Hkv), dim3(DTHREADS), DSMEM, st, pdl,
                     *reinterpret_cast<const TcMaps*>(tmaps), D, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
                     (const __nv_bfloat16*)v, t, kk, B, part, (__nv_bfloat16*)out);
-}
-
-template <typename E, int ROWB>
-static cudaError_t launch_step(const Dev& D, const StepArgs& A, int grid, cudaStream_t st, const void* tmaps) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(DTHREADS);
-    cfg.dynamicSmemBytes = step_smem(D.Hkv);
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeCooperative;
-    attr[0].val.cooperative = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_decode_step<E, ROWB>, *reinterpret_cast<const TcMaps*>(tmaps), D, A);
-}
-
-// Resident CTAs of k_decode_step<E, ROWB> on the current device (the cooperative grid size).
-template <typename E, int ROWB>
-static int step_grid(const Dev& D, cudaError_t* err) {
-    static std::atomic<unsigned long long> attr_done{0};
-    *err = smem_limit_once(k_decode_step<E, ROWB>, step_smem(STEP_HKV_MAX), attr_done);
-    if (*err != cudaSuccess) return 0;
-    int dev = 0, sms = 0, per_sm = 0;
-    if ((*err = cudaGetDevice(&dev)) != cudaSuccess) return 0;
-    if ((*err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return 0;
-    if ((*err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_decode_step<E, ROWB>, DTHREADS,
-                                                              step_smem(D.Hkv))) !=
-        cudaSuccess)
-        return 0;
-    return per_sm * sms;
-}
-
-cudaError_t launch_decode_step(const Dev& D, const void* q, const void* k, const void* v, int64_t t, int kk, int64_t B,
-                               int nm, int score_mode, int tag, unsigned long long qbase, void* out, cudaStream_t st,
-                               const void* tmaps, unsigned long long* consumed) {
-    StepArgs A;
-    A.q = (const __nv_bfloat16*)q;
-    A.k = (const __nv_bfloat16*)k;
-    A.v = (const __nv_bfloat16*)v;
-    A.out = (__nv_bfloat16*)out;
-    A.t = t;
-    A.B = B;
-    A.qbase = qbase;
-    A.kk = kk;
-    A.nm = nm;
-    A.nst = (int)((std::min<int64_t>(D.S, t + 1) + DK - 1) / DK);
-    A.nwt = (int)((t - B + 1 + DK - 1) / DK);
-    A.nut = kk * ((D.U + DK - 1) / DK);
-    A.mode = score_mode;
-    A.tag = tag;
-    if (A.nst + A.nut + A.nwt + 1 > D.dec_splits_max) return cudaErrorInvalidValue;  // + the merged slot
-    const int row_bytes = score_mode == OP_REPS ? D.r * D.d * 2 : score_mode == OP_REPSUM ? D.d * 4 : D.d * 2;
-    cudaError_t err = cudaSuccess;
-    int grid = 0;
-    switch (row_bytes) {
-        case 1024: grid = step_grid<__nv_bfloat16, 1024>(D, &err); break;
-        case 512: grid = score_mode == OP_REPSUM ? step_grid<float, 512>(D, &err) : step_grid<__nv_bfloat16, 512>(D, &err); break;
-        case 256: grid = step_grid<__nv_bfloat16, 256>(D, &err); break;
-        default: return cudaErrorInvalidValue;
-    }
-    if (err != cudaSuccess) return err;
-    if (grid <= 0) return cudaErrorInvalidConfiguration;
-    // static split of the scoring rows (flat units, head-major) over the grid
-    const int NW = (A.nst + A.nwt) * D.Hkv;
-    A.N = kk > 0 ? (int64_t)D.Hkv * nm : 0;
-    A.wr = (int)(2 * DTILE / row_bytes);  // a window tile's bytes, in scoring rows
-    A.nw_cta = std::min(NW, grid);
-    A.T = A.N + (int64_t)A.nw_cta * A.wr;
-    A.weighted = grid > NW && A.T / grid >= A.wr + 1;  // then every range is at least one row
-    A.gs = A.weighted ? grid : (int)std::max<int64_t>(1, std::min<int64_t>(grid, A.N / 16));  // plain: >= 16 rows each
-    if (A.N > 0) {
-        // every head's parts must fit its candidate-list slots: fewer, longer ranges until they do
-        for (;;) {
-            int worst = 0;
-            for (int h = 0; h < D.Hkv; ++h)
-                worst = std::max(worst, score_owner(A, (int64_t)(h + 1) * nm - 1) - score_owner(A, (int64_t)h * nm) + 1);
-            if (worst <= D.score_splits_max) break;
-            A.weighted = 0;
-            A.gs = std::max(1, A.gs / 2);
-        }
-    }
-    *consumed = (unsigned long long)A.nut * D.Hkv + (unsigned long long)grid;  // every CTA's last claim overshoots once
-    switch (row_bytes) {
-        case 1024: return launch_step<__nv_bfloat16, 1024>(D, A, grid, st, tmaps);
-        case 512: return score_mode == OP_REPSUM ? launch_step<float, 512>(D, A, grid, st, tmaps)
-                                                 : launch_step<__nv_bfloat16, 512>(D, A, grid, st, tmaps);
-        default: return launch_step<__nv_bfloat16, 256>(D, A, grid, st, tmaps);
-    }
 }
 
 }  // namespace infllm

@@ -53,10 +53,5 @@ int decode_split_keys(int elt_bytes);
 bool decode_tc_supported(const Dev& D);
 cudaError_t launch_decode_tc(const Dev& D, const void* q, const void* k, const void* v, int64_t t, int kk, int64_t B,
                              int part, void* out, cudaStream_t st, const void* tmaps, bool pdl);
-// The whole decode step in one cooperative launch (k_decode_step); *consumed receives how far the
-// step advances the context's work counter.
-cudaError_t launch_decode_step(const Dev& D, const void* q, const void* k, const void* v, int64_t t, int kk, int64_t B,
-                               int nm, int score_mode, int tag, unsigned long long qbase, void* out, cudaStream_t st,
-                               const void* tmaps, unsigned long long* consumed);
 
 }  // namespace infllm

@@ -1,4 +1,4 @@
-// Thin inline-PTX wrappers for sm_100a: mbarriers, TMA tile and bulk loads, tcgen05 (TMEM alloc, MMA,
+// Thin inline-PTX wrappers for sm_100a: mbarriers, TMA tile loads, tcgen05 (TMEM alloc, MMA,
 // commit, TMEM loads/stores) and UMMA descriptors.  Every wait is bounded.
 #pragma once
 
@@ -48,13 +48,6 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
         "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];"
         ::"r"(smem_u32(dst)), "l"((uint64_t)map), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
         : "memory");
-}
-// Untiled bulk copy global -> this CTA's shared memory (no multicast), completing on `bar` with
-// `bytes` transaction bytes.  Both addresses 16-byte aligned; `bytes` a multiple of 16.
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                 ::"r"(smem_u32(dst)), "l"((uint64_t)src), "r"(bytes), "r"(smem_u32(bar))
-                 : "memory");
 }
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)map) : "memory");

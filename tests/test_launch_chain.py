@@ -167,23 +167,24 @@ class Schedule:
         self.chain = False
         t = self.tokens
         if self.tc_decode and self.G <= 8:
-            # representatives of a newly evicted unit, then the whole step in one cooperative launch
-            # (launched without the chaining attribute: it starts once everything before has finished)
-            self.reps_to(self.n_mem(t))
+            # representatives of a newly evicted unit; part 0: the token's store, the sink and window
+            # tiles and their merge (early); the lookup alongside it (late after new representatives);
+            # part 1: the selected units' tiles and the final merge (late)
+            new_reps = self.reps_to(self.n_mem(t))
             L = self.nlook
             self.nlook += 1
             nm = self.n_mem(t)
+            kk = min(self.topk, nm)
             B = self.S + self.U * nm
-            reads = {("in", tag), self.selbuf(L)} | self.keys(0, t + 1) | {("rep", j) for j in range(nm)} | \
-                self.yblocks(t, t + 1)
-            writes = self.keys(t, t + 1) | self.yblocks(t, t + 1) | {("dpart", 0), ("dpart", 1), ("out", tag),
-                                                                    self.selbuf(L), ("uscore",), ("cand",)}
-            if self.plant == "decode_step_chained":
-                self.launch("decode_step", EARLY, reads, writes)
-            else:
-                self.launch("decode_step", NOPDL, reads, writes, attr=False)
+            w0 = self.keys(t, t + 1) | self.yblocks(t, t + 1) | {("dpart", 0)} | ({("out", tag)} if kk == 0 else set())
+            self.launch("decode_part0", EARLY, {("in", tag)} | self.keys(0, min(self.S, t + 1)) | self.keys(B, t + 1), w0)
             self.chain = True
             self.tokens = t + 1
+            if kk > 0:
+                wait_first = new_reps and self.plant != "decode_score_never_waits"
+                self.stage_select(L, nm, tag, wait_first)
+                self.launch("decode_part1", LATE, {("in", tag), self.selbuf(L), ("dpart", 0)} |
+                            self.keys(self.S, self.S + nm * self.U), {("dpart", 1), ("out", tag)})
             return
         self.pending_c0 = t
         self.stage_store(1, tag)
@@ -316,7 +317,7 @@ PLANTS = {
     "one_selection_buffer": ("attend", "score", "sel"),          # lookup c over the selection attend c-1 reads
     "attention_early": ("score", "attend", "sel"),               # attention before its selection is final
     "chunk1_chained_without_lookup": ("ysum", "reps", "Y"),      # chunk 1's representatives beside chunk 0's sums
-    "decode_step_chained": ("reps", "decode_step", "rep"),       # a decode step beside its new representatives
+    "decode_score_never_waits": ("reps", "score", "rep"),        # a decode lookup beside its new representatives
 }
 
 
