@@ -548,16 +548,20 @@ __global__ void __launch_bounds__(256) k_score_dec_half(Dev D, int mode, int n_m
     const uint4* base = score_operand<T>(D, mode, hk);
     const int half = lane >> 4, piece = lane & 15;
     const int slot = (lane >> 2) & 3;
-    // the first step's rows are requested before the query sum, which they do not need
-    uint4 raw[4];
-    auto load = [&](int u0) {
+    const int stride = nw * 8;
+    // two steps' rows in flight per warp (ping-pong buffers), the first two requested before the
+    // query sum, which they do not need
+    uint4 ra[4], rb[4];
+    auto load = [&](uint4 (&raw)[4], int u0) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int u = u0 + 2 * i + half;
             raw[i] = u < u_end ? __ldg(base + (int64_t)u * 16 + piece) : make_uint4(0, 0, 0, 0);
         }
     };
-    load(u_begin + warp * 8);
+    int u0 = u_begin + warp * 8;
+    load(ra, u0);
+    load(rb, u0 + stride);
     rotated_query_sum<T>(D, hk, 1, qraw, qb);
     __syncthreads();
     float qr[V];
@@ -568,8 +572,7 @@ __global__ void __launch_bounds__(256) k_score_dec_half(Dev D, int mode, int n_m
     }
     uint64_t list = 0, cand = 0;
     int it = 0;
-    for (int u0 = u_begin + warp * 8; u0 < u_end; u0 += nw * 8, ++it) {  // warp-uniform
-        if (it > 0) load(u0);
+    auto step = [&](const uint4 (&raw)[4], int s0) {  // one step: 8 units from s0 (warp-uniform)
         float acc[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[i] = dot16<E>(raw[i], qr);
@@ -587,7 +590,7 @@ __global__ void __launch_bounds__(256) k_score_dec_half(Dev D, int mode, int n_m
         }
         acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], 2);
         acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], 1);
-        const int j = u0 + 2 * slot + half;
+        const int j = s0 + 2 * slot + half;
         const float sc = acc[0] * D.inv_sqrt_d;
         if (j < u_end) {
             if ((lane & 3) == 0) D.uscore[(int64_t)hk * D.units_max + j] = sc;
@@ -596,6 +599,15 @@ __global__ void __launch_bounds__(256) k_score_dec_half(Dev D, int mode, int n_m
         if ((it & 3) == 3) {
             list = warp_topk_insert(list, cand);
             cand = 0;
+        }
+        ++it;
+    };
+    for (; u0 < u_end; u0 += 2 * stride) {  // warp-uniform
+        step(ra, u0);
+        load(ra, u0 + 2 * stride);
+        if (u0 + stride < u_end) {
+            step(rb, u0 + stride);
+            load(rb, u0 + 3 * stride);
         }
     }
     if (__any_sync(0xffffffffu, cand != 0)) list = warp_topk_insert(list, cand);
