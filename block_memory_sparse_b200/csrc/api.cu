@@ -412,6 +412,7 @@ infllm_status decode_impl(infllm_ctx* c, const void* q, const void* k, const voi
 infllm_status zero_state(infllm_ctx* c) {
     CK(cudaMemsetAsync(c->D.Y, 0, sizeof(float) * (size_t)((c->D.T_max / c->D.gblk) + 2) * c->D.Hkv * c->D.d, c->stream));
     CK(cudaMemsetAsync(c->D.counters, 0, sizeof(unsigned) * 4 * c->D.Hkv, c->stream));
+    CK(cudaMemsetAsync(c->D.simt_ctr, 0, sizeof(unsigned) * SIMT_PART_GROUPS, c->stream));
     CK(cudaMemsetAsync(c->sel_base, 0xff, sizeof(int32_t) * 2 * (size_t)c->D.Hkv * std::max(1, c->D.topk), c->stream));
     c->tokens = 0;
     c->units_done = 0;
@@ -492,6 +493,8 @@ infllm_status create_impl(infllm_ctx* c) {
     AL(D.qbar_part, sizeof(float) * 2 * (size_t)D.Hkv * D.qtiles_max * D.d);  // two buffers
     AL(D.cand, sizeof(uint64_t) * (size_t)D.Hkv * D.score_splits_max * 32);
     AL(D.counters, sizeof(unsigned) * 4 * D.Hkv);
+    AL(D.simt_part, sizeof(float) * (size_t)SIMT_PART_GROUPS * 8 * (D.d + 2));
+    AL(D.simt_ctr, sizeof(unsigned) * SIMT_PART_GROUPS);
     AL(D.Qm, (size_t)D.Hkv * 3 * D.qrows_max * D.d * c->elt);  // three slots
     AL(D.Qw, (size_t)D.Hkv * 3 * D.qrows_max * D.d * c->elt);
     AL(D.cs_chunk, sizeof(float2) * (size_t)g.max_chunk * D.half);

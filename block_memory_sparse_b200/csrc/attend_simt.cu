@@ -9,6 +9,8 @@
 // true relative distance (query R(t) q, key R(n) k).
 #include <math.h>
 
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -17,9 +19,14 @@ namespace infllm {
 constexpr int SIMT_ROWS = 8;   // packed query rows per CTA (one per warp)
 constexpr int SIMT_KT = 32;    // keys per smem tile (one per lane)
 
+// Grid (row CTAs, Hkv, nsplit).  With nsplit > 1 (a small chunk that would leave most SMs idle),
+// split sp takes every nsplit-th 32-key tile of the working context, writes its rows' partial
+// softmax (m, l, unnormalised o) to D.simt_part, and the CTA that finishes a row group's last split
+// (arrival counter, no CTA waits for another) merges the nsplit partials: the log-sum-exp
+// combination of disjoint key sets, in split order.
 template <typename T>
 __global__ void __launch_bounds__(256) k_attn_simt(Dev D, int64_t c0, int n, int kk, int64_t B, int par,
-                                                   T* __restrict__ out) {
+                                                   T* __restrict__ out, int nsplit) {
     extern __shared__ float sm[];
     pdl_wait();  // late kernel: selection, packed queries and keys are complete past this point
     pdl_trigger();
@@ -53,8 +60,10 @@ __global__ void __launch_bounds__(256) k_attn_simt(Dev D, int64_t c0, int n, int
     }
     float m = -INFINITY, l = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
     const int ndim = d / 32;
-    if (t_hi < 0) return;  // whole CTA is padding (uniform)
+    if (t_hi < 0) return;  // whole CTA is padding (uniform; every split of it returns here)
     const int nseg = 2 + kk;
+    const int sp = blockIdx.z;
+    int g = 0;  // tiles of the working context seen so far (all splits walk the same sequence)
     for (int sg = 0; sg < nseg; ++sg) {
         int64_t base, len;
         bool win = false, causal = false;
@@ -79,6 +88,7 @@ __global__ void __launch_bounds__(256) k_attn_simt(Dev D, int64_t c0, int n, int
         const T* Ks = (const T*)(win ? D.Krot : D.Kraw) + ((int64_t)hk * D.T_max + base) * d;
         const T* Vs = (const T*)D.V + ((int64_t)hk * D.T_max + base) * d;
         for (int64_t k0 = 0; k0 < len; k0 += SIMT_KT) {
+            if (g++ % nsplit != sp) continue;  // another split's tile (CTA-uniform)
             const int nk = (int)((len - k0) < SIMT_KT ? (len - k0) : SIMT_KT);
             __syncthreads();
             for (int idx = threadIdx.x; idx < SIMT_KT * d; idx += blockDim.x) {
@@ -113,11 +123,47 @@ __global__ void __launch_bounds__(256) k_attn_simt(Dev D, int64_t c0, int n, int
             m = m_new;
         }
     }
-    if (valid) {
-        T* o = out + ((int64_t)tl * D.Hq + hk * D.G + hg) * d;
-        const float inv = 1.f / l;
-        for (int c = 0; c < ndim; ++c) o[lane + 32 * c] = from_f<T>(acc[c] * inv);
+    if (nsplit == 1) {
+        if (valid) {
+            T* o = out + ((int64_t)tl * D.Hq + hk * D.G + hg) * d;
+            const float inv = 1.f / l;
+            for (int c = 0; c < ndim; ++c) o[lane + 32 * c] = from_f<T>(acc[c] * inv);
+        }
+        return;
     }
+    // this split's partial of the row (m, l, o) -> slot [row group][split][row]
+    const int grp = hk * gridDim.x + blockIdx.x;
+    float* part = D.simt_part + ((int64_t)grp * nsplit * SIMT_ROWS) * (d + 2);
+    float* mine = part + ((int64_t)sp * SIMT_ROWS + warp) * (d + 2);
+    if (lane == 0) {
+        mine[0] = m;
+        mine[1] = l;
+    }
+    for (int c = 0; c < ndim; ++c) mine[2 + lane + 32 * c] = acc[c];
+    __threadfence();
+    __syncthreads();
+    __shared__ int last;
+    if (threadIdx.x == 0) last = atomicAdd(D.simt_ctr + grp, 1u) == (unsigned)(nsplit - 1);
+    __syncthreads();
+    if (!last) return;
+    __threadfence();
+    if (valid) {
+        float M = -INFINITY;
+        for (int x = 0; x < nsplit; ++x) M = fmaxf(M, __ldcg(part + ((int64_t)x * SIMT_ROWS + warp) * (d + 2)));
+        float L = 0.f, o[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int x = 0; x < nsplit; ++x) {
+            const float* px = part + ((int64_t)x * SIMT_ROWS + warp) * (d + 2);
+            const float mx = __ldcg(px);
+            if (mx == -INFINITY) continue;  // no attended key in this split
+            const float f = expf(mx - M);
+            L = fmaf(f, __ldcg(px + 1), L);
+            for (int c = 0; c < ndim; ++c) o[c] = fmaf(f, __ldcg(px + 2 + lane + 32 * c), o[c]);
+        }
+        T* orow = out + ((int64_t)tl * D.Hq + hk * D.G + hg) * d;
+        const float inv = 1.f / L;
+        for (int c = 0; c < ndim; ++c) orow[lane + 32 * c] = from_f<T>(o[c] * inv);
+    }
+    if (threadIdx.x == 0) D.simt_ctr[grp] = 0u;  // re-armed for the next launch
 }
 
 template <typename T>
@@ -126,13 +172,18 @@ cudaError_t launch_attend_simt(const Dev& D, int64_t c0, int n, int kk, int64_t 
     if (n <= 0) return cudaSuccess;
     const int tiles = (n + D.qt - 1) / D.qt;
     const int rows = tiles * D.qt * D.G;
-    dim3 grid((rows + SIMT_ROWS - 1) / SIMT_ROWS, D.Hkv);
+    const int ctas = (rows + SIMT_ROWS - 1) / SIMT_ROWS;
+    // split the keys over up to SIMT_MAX_SPLIT CTAs per row group while the grid stays under
+    // SIMT_PART_GROUPS CTAs (the partial slots and counters allocated at create)
+    const int groups = ctas * D.Hkv;
+    const int nsplit = groups >= SIMT_PART_GROUPS / 2 ? 1 : std::min(SIMT_MAX_SPLIT, SIMT_PART_GROUPS / groups);
+    dim3 grid(ctas, D.Hkv, nsplit);
     const size_t smem = (size_t)(2 * SIMT_ROWS * D.d + SIMT_KT * (D.d + 1) + SIMT_KT * D.d) * sizeof(float);
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(k_attn_simt<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
-    return launch_k(k_attn_simt<T>, grid, dim3(256), smem, st, pdl, D, c0, n, kk, B, par, (T*)out);
+    return launch_k(k_attn_simt<T>, grid, dim3(256), smem, st, pdl, D, c0, n, kk, B, par, (T*)out, nsplit);
 }
 
 template cudaError_t launch_attend_simt<float>(const Dev&, int64_t, int, int, int64_t, int, void*, cudaStream_t, bool);

@@ -11,6 +11,11 @@ namespace infllm {
 
 // Everything a kernel needs to know about the layer and the context's device buffers.
 // Passed by value to every kernel.
+// Split of the CUDA-core chunk attention over keys: at most SIMT_MAX_SPLIT splits, and
+// (row groups x splits) <= SIMT_PART_GROUPS, the CTAs whose partials the context keeps room for.
+constexpr int SIMT_MAX_SPLIT = 16;
+constexpr int SIMT_PART_GROUPS = 296;
+
 struct Dev {
     // shape
     int Hq, Hkv, G, d, half;
@@ -52,6 +57,10 @@ struct Dev {
     // (cos, sin)(x 2^(11 L) theta_i) in fp64 for L < 3, x < 2048: exp(i t theta) for any
     // t < 2^33 is the product of three entries (t's 11-bit digits)
     const double2* cs_abs3;  // [3][2048][half]
+    // CUDA-core chunk attention split over keys: partials [groups][splits][8 rows][d + 2] (m, l, o) and
+    // one arrival counter per row group (SIMT_PART_GROUPS x 8 rows of slots in all)
+    float* simt_part;
+    unsigned* simt_ctr;
     // decode partials: [Hkv][dec_splits_max][G][d + 4] (the CUDA-core decode uses [G][d + 2] of a slot)
     float* dec_part;
     int dec_splits_max;
