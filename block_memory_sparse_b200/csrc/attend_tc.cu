@@ -8,22 +8,24 @@
 // One CTA per (128 packed query rows, KV head): the rows are G q heads x 128/G consecutive
 // queries of one KV group, so every K/V tile is read once per group.  Warp roles:
 //   warp 0      TMA producer: the two query tiles once, then K and V tiles (2-stage rings)
-//   warp 1      MMA issuer:   S_i = Q K_i^T into TMEM (double buffered, Q and K from shared
-//                             memory); O_h += P_i[:, half h] V_i[half h] with P read from TMEM
-//   warps 2..9  softmax:      two threads per row (warps w and w + 4 share a TMEM lane quarter
-//                             and split the tile's 128 columns in halves).  Each half runs its own
-//                             online softmax over its columns of every tile -- its own running
-//                             max, sum and accumulator O_h -- so the two never wait for each
-//                             other inside the loop; O_h is rescaled lazily (only when the half's
-//                             max grows by > 2^8).  P_i goes as bf16 into the TMEM columns of S_i.
-//                             After the last tile the halves exchange (max, sum) once through
-//                             shared memory and each thread stores 64 outputs of the merged row.
-// Splitting a row's keys in two and merging the partial softmaxes at the end is exact (up to
-// rounding): it is the log-sum-exp combination of two disjoint key sets.  Each softmax warp writes
-// its half of P_i over the first 32 columns of its own half of S_i (it has read them; the partner
-// warp never reads them), so S_i and P_i share a buffer, double buffered: the exponentials of tile
-// i overlap the PV product of tile i - 1, and QK of tile i + 2 (same buffer) is issued after
-// PV(i) -- the tensor pipe executes one thread's MMAs in issue order.
+//   warp 1      MMA issuer:   S_i = Q K_i^T into S buffer i & 1 (Q and K from shared memory);
+//                             O_{i & 1} += P_i V_i with P read from TMEM
+//   warps 2..9  softmax:      two groups of four warps (one warp per TMEM lane quarter, one thread
+//                             per row): group g takes the KV tiles i with i & 1 == g, all 128
+//                             columns of each.  Each group runs its own online softmax over its
+//                             tiles -- its own running max, sum and accumulator O_g -- so the two
+//                             never wait for each other inside the loop and work on different
+//                             tiles at once; O_g is rescaled lazily (only when the group's max
+//                             grows by > 2^8).  P_i goes as bf16 over the first 64 columns of S_i.
+//                             After the last tile the groups exchange (max, sum) once through
+//                             shared memory and each thread stores HD / 2 outputs of the merged row.
+// Splitting a row's keys into two sets and merging the partial softmaxes at the end is exact (up
+// to rounding): it is the log-sum-exp combination of two disjoint key sets.  S_i and P_i share a
+// buffer, double buffered: the exponentials of tile i overlap QK of tile i + 1 and the PV product
+// of tile i - 1, and QK of tile i + 2 (same buffer) is issued after PV(i) -- the tensor pipe
+// executes one thread's MMAs in issue order.  The MMA-issuing thread keeps pace with the tensor
+// pipe (its queue is short), so its loop holds no lookups: the K and V ring slots are released by
+// the same two barriers that announce S_i and PV(i), and the query tile is chosen by tile index.
 // Sinks and memory tiles use R(W) q with raw keys; window tiles use R(t) q with R(n) k.
 #include <cuda.h>
 #include <math.h>
@@ -42,7 +44,8 @@ constexpr int BN = 128;  // keys per tile
 constexpr int NTHREADS = 320;  // producer warp, MMA warp, 8 softmax warps
 constexpr int NSOFT = 256;     // softmax threads
 constexpr uint32_t SWB = BN * 128;  // one 64-column swizzle block of a tile (128 rows x 128 B)
-constexpr int NSTAGE = 2;           // K and V ring depth
+constexpr int NSTAGE = 2;           // K and V ring depth (= the S buffers: the ring reuses their barriers)
+static_assert(NSTAGE == 2, "the K / V slots are released by the S / PV barriers of the two tile parities");
 constexpr int MAX_SEL = 4096;       // selected unit ids of this KV head kept in shared memory
 
 // Shared-memory layout for head dim HD (64 or 128): a tile is HD / 64 swizzle blocks.
@@ -69,9 +72,11 @@ constexpr float RESCALE_LOG2 = 8.0f;
 constexpr int ERR_TIMEOUT = 16;
 
 struct Bars {
-    // pfull and pvdone alternate by tile parity: P(i) is released on pfull[i & 1] and PV(i) completes on
-    // pvdone[i & 1], so that neither consumer can fall two phases behind one barrier (parity aliasing)
-    uint64_t q, kfull[NSTAGE], kempty[NSTAGE], vfull[NSTAGE], vempty[NSTAGE], sfull[2], pfull[2], pvdone[2];
+    // sfull, pfull and pvdone alternate by tile parity: S(i) lands on sfull[i & 1], P(i) is released on
+    // pfull[i & 1] and PV(i) completes on pvdone[i & 1], so that no consumer can fall two phases behind
+    // one barrier (parity aliasing)
+    // K / V slot i % NSTAGE is free again once QK(i) / PV(i) is complete: sfull / pvdone, as NSTAGE == 2
+    uint64_t q, kfull[NSTAGE], vfull[NSTAGE], sfull[2], pfull[2], pvdone[2];
     uint32_t tmem;
     int abort;
 };
@@ -93,7 +98,7 @@ struct Plan {
         if (i < nst) return {0, (int64_t)i * BN, min(BN, S_eff - i * BN)};
         i -= nst;
         if (i < nut) {
-            const int u = i / tpu, part = i % tpu;
+            const int u = tpu == 1 ? i : i / tpu, part = tpu == 1 ? 0 : i % tpu;
             const int j = sel[u];
             if (j < 0) return {1, 0, 0};
             return {1, (int64_t)D.S + (int64_t)j * D.U + (int64_t)part * BN, min(BN, D.U - part * BN)};
@@ -143,12 +148,14 @@ __device__ void producer(const TcMaps& maps, const Plan& P, const Dev& D, uint8_
     for (int i = 0; i < P.NT; ++i) {
         const int s = i % NSTAGE;
         const uint32_t use = (uint32_t)(i / NSTAGE);
-        if (i >= NSTAGE && !wait_bar(&bars->kempty[s], (use - 1) & 1, bars, D)) break;
+        // K slot s held tile i - 2: free once QK(i - 2) is complete, which sfull[s] announces
+        if (i >= NSTAGE && !wait_bar(&bars->sfull[s], (use - 1) & 1, bars, D)) break;
         const TileInfo T = P.tile(D, i);
         const CUtensorMap* km = T.kind == 2 ? &maps.krot : &maps.kraw;
         ptx::mbar_expect_tx(&bars->kfull[s], Y::TILE);
         load_tile<HD>(sm + Y::OFF_K + s * Y::TILE, km, &bars->kfull[s], (int)T.y0, P.hk);
-        if (i >= NSTAGE && !wait_bar(&bars->vempty[s], (use - 1) & 1, bars, D)) {
+        // V slot s: free once PV(i - 2) is complete (pvdone[s])
+        if (i >= NSTAGE && !wait_bar(&bars->pvdone[s], (use - 1) & 1, bars, D)) {
             issued = i + 1;
             break;
         }
@@ -182,7 +189,7 @@ __device__ void mma_issuer(const Plan& P, const Dev& D, uint8_t* sm, Bars* bars,
             const int s = i % NSTAGE, b = i & 1;
             if (!wait_bar(&bars->kfull[s], (uint32_t)(i / NSTAGE) & 1, bars, D)) return;
             ptx::tc_fence_after();
-            const uint32_t qa = P.tile(D, i).kind == 2 ? qw : qm;
+            const uint32_t qa = i >= P.nst + P.nut ? qw : qm;
             const uint32_t ka = kb + s * Y::TILE;
 #pragma unroll
             for (int ks = 0; ks < HD / 16; ++ks) {  // 16 of the head dim: swizzle block ks / 4, 32 B each
@@ -191,7 +198,6 @@ __device__ void mma_issuer(const Plan& P, const Dev& D, uint8_t* sm, Bars* bars,
                               IDESC_QK, ks > 0 ? 1u : 0u);
             }
             ptx::mma_commit(&bars->sfull[b]);
-            ptx::mma_commit(&bars->kempty[s]);
         }
         if (i >= 1) {
             const int j = i - 1, sj = j % NSTAGE, bj = j & 1;
@@ -201,12 +207,10 @@ __device__ void mma_issuer(const Plan& P, const Dev& D, uint8_t* sm, Bars* bars,
             const uint32_t va = vb + sj * Y::TILE;
 #pragma unroll
             for (int ks = 0; ks < BN / 16; ++ks)  // keys 16 ks ..: half h = ks / 4 of P_j into O_h
-                ptx::mma_bf16_ts(tmem + TM_O + (uint32_t)(ks >> 2) * HD,
-                                 tmem + bj * BN + (uint32_t)(ks >> 2) * 64 + (uint32_t)(ks & 3) * 8,
+                ptx::mma_bf16_ts(tmem + TM_O + (uint32_t)bj * HD, tmem + bj * BN + (uint32_t)ks * 8,
                                  ptx::sdesc_sw128(va + (uint32_t)ks * 2048, SWB, 1024), IDESC_PV,
-                                 (j > 0 || (ks & 3) > 0) ? 1u : 0u);
+                                 (j > 1 || ks > 0) ? 1u : 0u);
             ptx::mma_commit(&bars->pvdone[j & 1]);
-            ptx::mma_commit(&bars->vempty[sj]);
         }
     }
 }
@@ -222,125 +226,124 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
-// PV completions are consumed strictly in order, PV(x) as phase x >> 1 of pvdone[x & 1], and never
-// two phases late on one barrier: a parity wait on an mbarrier that has completed two phases past
-// the awaited one would wait for a third.  Tile i consumes PV(i - 2) before it releases P_i, and
-// PV(i) is issued only after that release, so at most PV(i - 1) can be complete past it.
+// PV completions of one softmax group: the x-th PV product of group g (tile g + 2x) completes phase x
+// of pvdone[g].  Consumed strictly in order and never two phases late: the group consumes its
+// previous PV before it releases its next P, and that PV is issued only after the release.
 struct PvTrack {
-    int seen = 0;  // PV products known complete: tiles [0, seen)
-    __device__ __forceinline__ bool upto(int j, Bars* bars, const Dev& D) {
-        while (seen <= j) {
-            if (!warp_wait(&bars->pvdone[seen & 1], (uint32_t)(seen >> 1) & 1, bars, D)) return false;
+    int seen = 0;  // this group's PV products known complete: its first `seen` tiles
+    __device__ __forceinline__ bool upto(int x, uint64_t* bar, Bars* bars, const Dev& D) {
+        while (seen <= x) {
+            if (!warp_wait(bar, (uint32_t)seen & 1, bars, D)) return false;
             ++seen;
         }
         return true;
     }
 };
 
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 template <int HD>
 __device__ void softmax_role(const Plan& P, const Dev& D, Bars* bars, float* lsum, float* mref, uint32_t tmem,
                              int64_t c0, int n, __nv_bfloat16* __restrict__ out, int warp, int lane) {
-    const int quarter = warp & 3;        // TMEM lanes this warp may access
-    const int half = (warp - 2) >> 2;    // columns [64 half, 64 half + 64) of every tile are this thread's
+    const int quarter = warp & 3;       // TMEM lanes this warp may access
+    const int grp = (warp - 2) >> 2;    // KV tiles i with i & 1 == grp are this thread's
     const int row = quarter * 32 + lane;
     const uint32_t tl_addr = tmem + ((uint32_t)(quarter * 32) << 16);
-    const uint32_t o_addr = tl_addr + TM_O + (uint32_t)half * HD;  // this thread's row of O_half
+    const uint32_t sbase = tl_addr + (uint32_t)grp * BN;       // S_i / P_i of this group's tiles
+    const uint32_t o_addr = tl_addr + TM_O + (uint32_t)grp * HD;  // this thread's row of O_grp
     const int hg = row / D.qt, tl = P.a * D.qt + row % D.qt;
     const bool valid = tl < n;
     const int64_t t = c0 + tl;
     const float sc = D.inv_sqrt_d * LOG2E;  // logits in log2 units: s * sc
-    // This half's own online softmax: reference max (log2 units), sum, and O_half; the two
-    // halves of a row meet once, after the last tile.
     float m_used = -INFINITY, l = 0.f;
-    float s[64];
     PvTrack pv;
+    uint64_t* pvbar = &bars->pvdone[grp];
     bool ok = true;
-    for (int i = 0; i < P.NT; ++i) {
-        const int b = i & 1;
-        if (!warp_wait(&bars->sfull[b], (uint32_t)(i >> 1) & 1, bars, D)) {
+    for (int i = grp; i < P.NT; i += 2) {
+        const int x = i >> 1;  // this group's tile count before tile i
+        if (!warp_wait(&bars->sfull[grp], (uint32_t)x & 1, bars, D)) {
             ok = false;
             break;
         }
         ptx::tc_fence_after();
-        const uint32_t sbase = tl_addr + b * BN;
-        ptx::tmem_ld32(sbase + half * 64, s);
-        ptx::tmem_ld32(sbase + half * 64 + 32, s + 32);
+        float s[128];
+        ptx::tmem_ld32(sbase, s);
+        ptx::tmem_ld32(sbase + 32, s + 32);
+        ptx::tmem_ld32(sbase + 64, s + 64);
+        ptx::tmem_ld32(sbase + 96, s + 96);
         ptx::tmem_wait_ld();
-        // columns [0, lim) of this tile are attended by this row (causal limit on sinks and window)
         const TileInfo T = P.tile(D, i);
         int lim = T.nv;
         if (T.kind != 1) {
             const int64_t c = t - T.y0 + 1;
             lim = c < (int64_t)lim ? (int)(c < 0 ? 0 : c) : lim;
         }
-        const int own = lim - half * 64;  // valid columns of this half
-        float mq[8];                       // independent partial maxima (short dependency chains)
+        float mq[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) mq[e] = -INFINITY;
-        if (__all_sync(0xffffffffu, own >= 64)) {
+        if (!__all_sync(0xffffffffu, lim >= BN)) {
 #pragma unroll
-            for (int c = 0; c < 64; ++c) mq[c & 7] = fmaxf(mq[c & 7], s[c]);
-        } else {
-#pragma unroll
-            for (int c = 0; c < 64; ++c) {
-                s[c] = c < own ? s[c] : -INFINITY;
-                mq[c & 7] = fmaxf(mq[c & 7], s[c]);
-            }
+            for (int c = 0; c < 128; ++c) s[c] = c < lim ? s[c] : -INFINITY;
         }
+#pragma unroll
+        for (int c = 0; c < 128; c += 2) mq[(c >> 1) & 7] = max3(mq[(c >> 1) & 7], s[c], s[c + 1]);
         const float mx = fmaxf(fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])), fmaxf(fmaxf(mq[4], mq[5]), fmaxf(mq[6], mq[7])));
         const float mt = mx * sc;
         const bool need = mt > m_used + RESCALE_LOG2;
         const float m_new = need ? mt : m_used;
-        if (i >= 1 && __any_sync(0xffffffffu, need)) {  // O_half must hold every earlier product first
-            if (!pv.upto(i - 1, bars, D)) {
-                ok = false;
-                break;
-            }
-            ptx::tc_fence_after();
-            const float f = need ? ex2(m_used - m_new) : 1.f;
-            l *= f;
-#pragma unroll
-            for (int c4 = 0; c4 < HD / 32; ++c4) {
-                float o[32];
-                ptx::tmem_ld32(o_addr + c4 * 32, o);
-                ptx::tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 32; ++e) o[e] *= f;
-                ptx::tmem_st32(o_addr + c4 * 32, o);
-            }
-        }
+        const float f = need ? ex2(m_used - m_new) : 1.f;  // rescale of this group's O and sum
         m_used = m_new;
         const float nref = m_used == -INFINITY ? 0.f : -m_used;
         float rs[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) rs[e] = 0.f;
-        uint32_t w[32];  // this half's 64 keys as 32 columns of packed bf16 pairs
+        uint32_t w[64];  // the tile's 128 keys as 64 columns of packed bf16 pairs
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
+        for (int e = 0; e < 64; ++e) {
             const float p0 = ex2(fmaf(s[2 * e], sc, nref)), p1 = ex2(fmaf(s[2 * e + 1], sc, nref));
             rs[(2 * e) & 7] += p0;
             rs[(2 * e + 1) & 7] += p1;
             __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
             w[e] = *reinterpret_cast<uint32_t*>(&h);
         }
-        ptx::tmem_st32(sbase + half * 64, reinterpret_cast<const float*>(w));  // over this half's own S columns
-        l += ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
-        ptx::tmem_wait_st();
-        // consume PV(i - 2) before P_i is released (PV(i) is issued only after the arrival below);
-        // PV(i - 1) may still run while this row goes on to tile i + 1
-        if (i >= 2 && !pv.upto(i - 2, bars, D)) {
-            ok = false;
-            break;
+        ptx::tmem_st32(sbase, reinterpret_cast<const float*>(w));  // over columns [0, 64) of S_i, read above
+        ptx::tmem_st32(sbase + 32, reinterpret_cast<const float*>(w + 32));
+        l = fmaf(l, f, ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7])));
+        // O_grp holds this group's earlier products (and P_i may be released) once PV of its previous
+        // tile is complete; a growing maximum rescales O_grp here, before PV(i) adds to it
+        if (x >= 1) {
+            if (!pv.upto(x - 1, pvbar, bars, D)) {
+                ok = false;
+                break;
+            }
+            if (__any_sync(0xffffffffu, need)) {
+                ptx::tc_fence_after();
+#pragma unroll
+                for (int c4 = 0; c4 < HD / 32; ++c4) {
+                    float o[32];
+                    ptx::tmem_ld32(o_addr + c4 * 32, o);
+                    ptx::tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) o[e] *= f;
+                    ptx::tmem_st32(o_addr + c4 * 32, o);
+                }
+            }
         }
+        ptx::tmem_wait_st();
         ptx::tc_fence_before();
-        ptx::mbar_arrive(&bars->pfull[i & 1]);
+        ptx::mbar_arrive(&bars->pfull[grp]);
     }
-    ok = ok && pv.upto(P.NT - 1, bars, D);
-    // the two halves of the row meet: O = (2^(m_0 - M) O_0 + 2^(m_1 - M) O_1) / (same weights on
-    // l_0, l_1), M = max(m_0, m_1); each of the pair stores HD / 2 outputs of the row.  Every
-    // softmax thread reaches this barrier: all waits above are bounded.
-    lsum[half * 128 + row] = l;
-    mref[half * 128 + row] = m_used;
+    const int mine = P.NT > grp ? (P.NT - grp + 1) >> 1 : 0;  // tiles of this group
+    ok = ok && (mine == 0 || pv.upto(mine - 1, pvbar, bars, D));
+    // the two groups of a row meet: O = (2^(m_0 - M) O_0 + 2^(m_1 - M) O_1) / (same weights on
+    // l_0, l_1), M = max(m_0, m_1); a group without tiles has m = -inf, weight 0 and an O that was
+    // never written (selected away, not multiplied).  Each of the pair stores HD / 2 outputs.
+    lsum[grp * 128 + row] = l;
+    mref[grp * 128 + row] = m_used;
     asm volatile("bar.sync 1, %0;" ::"n"(NSOFT) : "memory");
     if (!__all_sync(0xffffffffu, ok)) return;
     ptx::tc_fence_after();
@@ -349,13 +352,14 @@ __device__ void softmax_role(const Plan& P, const Dev& D, Bars* bars, float* lsu
     const float f0 = m0 == -INFINITY ? 0.f : ex2(m0 - M), f1 = m1 == -INFINITY ? 0.f : ex2(m1 - M);
     const float inv = 1.f / (lsum[row] * f0 + lsum[128 + row] * f1);
     const float g0 = f0 * inv, g1 = f1 * inv;
+    const bool use0 = f0 != 0.f, use1 = f1 != 0.f;
     constexpr int OWN = HD / 2;
-    __nv_bfloat16* orow = out + ((int64_t)tl * D.Hq + P.hk * D.G + hg) * HD + half * OWN;
+    __nv_bfloat16* orow = out + ((int64_t)tl * D.Hq + P.hk * D.G + hg) * HD + grp * OWN;
 #pragma unroll 1
     for (int c4 = 0; c4 < OWN / 32; ++c4) {
         float o0[32], o1[32];
-        ptx::tmem_ld32(tl_addr + TM_O + half * OWN + c4 * 32, o0);
-        ptx::tmem_ld32(tl_addr + TM_O + HD + half * OWN + c4 * 32, o1);
+        ptx::tmem_ld32(tl_addr + TM_O + grp * OWN + c4 * 32, o0);
+        ptx::tmem_ld32(tl_addr + TM_O + HD + grp * OWN + c4 * 32, o1);
         ptx::tmem_wait_ld();
         if (valid) {
 #pragma unroll
@@ -364,8 +368,9 @@ __device__ void softmax_role(const Plan& P, const Dev& D, Bars* bars, float* lsu
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     const int k = e * 8 + 2 * q;
-                    __nv_bfloat162 h = __floats2bfloat162_rn(fmaf(o0[k], g0, o1[k] * g1),
-                                                             fmaf(o0[k + 1], g0, o1[k + 1] * g1));
+                    const float a0 = use0 ? o0[k] * g0 : 0.f, a1 = use0 ? o0[k + 1] * g0 : 0.f;
+                    const float b0 = use1 ? o1[k] * g1 : 0.f, b1 = use1 ? o1[k + 1] * g1 : 0.f;
+                    __nv_bfloat162 h = __floats2bfloat162_rn(a0 + b0, a1 + b1);
                     w4[q] = *reinterpret_cast<uint32_t*>(&h);
                 }
                 *reinterpret_cast<uint4*>(orow + c4 * 32 + e * 8) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
@@ -408,13 +413,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         ptx::mbar_init(&bars->q, 1);
         for (int s = 0; s < NSTAGE; ++s) {
             ptx::mbar_init(&bars->kfull[s], 1);
-            ptx::mbar_init(&bars->kempty[s], 1);
             ptx::mbar_init(&bars->vfull[s], 1);
-            ptx::mbar_init(&bars->vempty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             ptx::mbar_init(&bars->sfull[b], 1);
-            ptx::mbar_init(&bars->pfull[b], NSOFT);
+            ptx::mbar_init(&bars->pfull[b], NSOFT / 2);  // the threads of group b
             ptx::mbar_init(&bars->pvdone[b], 1);
         }
         bars->abort = 0;

@@ -3,23 +3,24 @@
 No compute-sanitizer run of this kernel exists, so its synchronisation is checked on a model
 instead: the roles of `k_attn_tc` (attend_tc.cu) as coroutines that a seeded scheduler
 interleaves at random, with exact mbarrier parity semantics.
-- TMA producer: two query tiles, then K and V tiles through 2-stage rings.
-- MMA issuer: QK(i) into S buffer i & 1, then PV(i - 1) after P(i - 1) is released.
+- TMA producer: two query tiles, then K and V tiles through 2-stage rings. Slot s is refilled
+  with tile i once QK(i - 2) / PV(i - 2) is complete, seen on the S / PV barriers of parity s
+  (there are no separate slot-release barriers).
+- MMA issuer: QK(i) into S buffer i & 1, then PV(i - 1) into O_{(i - 1) & 1} after P(i - 1) is
+  released.
 - Tensor pipe: executes one thread's MMAs in issue order; each commit arrives when every
   earlier MMA is done.
 - TMA engine: lands copies in any order.
-- Two softmax threads: the two column halves of a row, each with its own online softmax. A
-  half may rescale its accumulator O_h (only after PV(i - 1) is complete) and writes its half
-  of P(i) over its half of S(i); it releases P(i) once PV(i - 2) is complete, so PV(i - 1) can
-  run while it works on the next tile.  P releases and PV completions alternate between two
-  barriers each (by tile parity), which keeps every consumer within one phase of its barrier.
+- Two softmax groups: group g takes the tiles i with i & 1 == g, reads all of S(i), writes P(i)
+  over it and keeps its own online softmax and accumulator O_g. A group may rescale O_g only
+  after its previous PV is complete, and releases P(i) only after that PV is complete (so the
+  PV barrier of its parity is never two phases ahead of it).
 
 Every data hand-off is asserted where it happens:
 - a ring slot is refilled only after the MMA that read it has executed;
-- S(i) is read only once QK(i) has written it, and is not overwritten before both halves are
-  done;
-- PV(j) reads both halves of P(j), and never a stale one;
-- O_h is read or rescaled only when no PV that writes it is pending;
+- S(i) is read only once QK(i) has written it, and is not overwritten before its group read it;
+- PV(j) reads P(j), and never a stale one;
+- O_g is read or rescaled only when no PV that writes it is pending;
 - a parity wait never runs two or more phases behind its barrier, where parity aliases;
 - no interleaving deadlocks (bounded step count).
 A planted protocol mistake must fail the same checks (last test).
@@ -58,17 +59,19 @@ class Bar:
 
 def run(NT, seed, plant=None):
     rnd = random.Random(seed)
-    bars = {"q": Bar("q", 1), "pfull0": Bar("pfull0", 2), "pfull1": Bar("pfull1", 2), "pvdone0": Bar("pvdone0", 1), "pvdone1": Bar("pvdone1", 1),
-            "sfull0": Bar("sfull0", 1), "sfull1": Bar("sfull1", 1)}
+    bars = {"q": Bar("q", 1)}
+    for g in (0, 1):
+        for x in ("sfull", "pfull", "pvdone"):
+            bars[f"{x}{g}"] = Bar(f"{x}{g}", 1)  # pfull: one arrival stands for the group's threads
     for s in range(NSTAGE):
-        for x in ("kfull", "kempty", "vfull", "vempty"):
+        for x in ("kfull", "vfull"):
             bars[f"{x}{s}"] = Bar(f"{x}{s}", 1)
-    kslot = [None] * NSTAGE   # tile whose K occupies the slot (None: empty)
+    kslot = [None] * NSTAGE   # tile whose K occupies the slot
     vslot = [None] * NSTAGE
     kread = [-1] * NSTAGE     # last tile whose QK has executed on that slot
     vread = [-1] * NSTAGE
-    S = [None, None]          # per buffer: (tile, set of halves that have read it)
-    P = [dict(), dict()]      # per buffer: half -> tile of the P half stored there
+    S = [None, None]          # per buffer: [tile, read by its group?]
+    P = [None, None]          # per buffer: tile of the P stored there, or ("used", tile)
     pv_done = []              # PV tiles executed, in order
     pipe = []                 # issued, not yet executed tensor-pipe ops
     tma = []                  # copies in flight
@@ -82,12 +85,12 @@ def run(NT, seed, plant=None):
         tma.append(("q", None, None))
         for i in range(NT):
             s, use = i % NSTAGE, i // NSTAGE
-            if i >= NSTAGE:
-                yield from wait(f"kempty{s}", use - 1)
+            if i >= NSTAGE and plant != "k_slot_not_released":
+                yield from wait(f"sfull{s}", use - 1)
             tma.append(("k", s, i))
             yield
             if i >= NSTAGE:
-                yield from wait(f"vempty{s}", use - 1)
+                yield from wait(f"pvdone{s}", use - 1)
             tma.append(("v", s, i))
             yield
 
@@ -116,14 +119,14 @@ def run(NT, seed, plant=None):
             if i < NT:
                 s, use = i % NSTAGE, i // NSTAGE
                 yield from wait(f"kfull{s}", use)
-                pipe.extend([("qk", i), ("commit", f"sfull{i & 1}"), ("commit", f"kempty{s}")])
+                pipe.extend([("qk", i), ("commit", f"sfull{i & 1}")])
                 yield
             if i >= 1:
                 j = i - 1
                 yield from wait(f"pfull{j & 1}", j >> 1)
                 if plant != "pv_skips_v_wait":
                     yield from wait(f"vfull{j % NSTAGE}", j // NSTAGE)
-                pipe.extend([("pv", j), ("commit", f"pvdone{j & 1}"), ("commit", f"vempty{j % NSTAGE}")])
+                pipe.extend([("pv", j), ("commit", f"pvdone{j & 1}")])
                 yield
 
     def tensor_pipe():
@@ -135,51 +138,50 @@ def run(NT, seed, plant=None):
                     assert q_landed[0]
                     assert kslot[s] == x, f"QK({x}) read K slot {s} holding {kslot[s]}"
                     if S[b] is not None:
-                        assert S[b][1] == {0, 1}, f"QK({x}) overwrote S({S[b][0]}) before both halves read it"
-                        assert all(v == ("used", x - 2) for v in P[b].values()), f"QK({x}) overwrote P: {P[b]}"
-                    S[b] = (x, set())
-                    P[b] = {}
+                        assert S[b][1], f"QK({x}) overwrote S({S[b][0]}) before its group read it"
+                        assert P[b] == ("used", x - 2), f"QK({x}) overwrote P: {P[b]}"
+                    S[b] = [x, False]
+                    P[b] = None
                     kread[s] = x
                 elif op == "pv":
                     b, s = x & 1, x % NSTAGE
                     assert vslot[s] == x, f"PV({x}) read V slot {s} holding {vslot[s]}"
-                    assert P[b] == {0: x, 1: x}, f"PV({x}) read P {P[b]}"
-                    P[b] = {h: ("used", x) for h in (0, 1)}
+                    assert P[b] == x, f"PV({x}) read P {P[b]}"
+                    P[b] = ("used", x)
                     vread[s] = x
                     pv_done.append(x)
                 else:
                     bars[x].arrive()
             yield
 
-    def softmax(h):
-        seen = [0]  # PV completions consumed: tiles [0, seen)
+    def softmax(g):
+        seen = [0]  # this group's PV products known complete
 
-        def upto(j):  # PV(x) completes phase x >> 1 of pvdone[x & 1]
-            while seen[0] <= j:
-                yield from wait(f"pvdone{seen[0] & 1}", seen[0] >> 1)
+        def upto(x):  # the x-th PV of group g (tile g + 2x) completes phase x of pvdone[g]
+            while seen[0] <= x:
+                yield from wait(f"pvdone{g}", seen[0])
                 seen[0] += 1
 
-        for i in range(NT):
-            b = i & 1
-            yield from wait(f"sfull{b}", i >> 1)
-            assert S[b] is not None and S[b][0] == i, f"half {h} read S buffer {b} = {S[b]} for tile {i}"
+        for i in range(g, NT, 2):
+            x = i >> 1
+            yield from wait(f"sfull{g}", x)
+            assert S[g] is not None and S[g][0] == i, f"group {g} read S buffer {g} = {S[g]} for tile {i}"
+            S[g][1] = True
             yield
-            if i >= 1 and rnd.random() < 0.3:  # the half's running max grew: rescale O_h
-                if plant != "rescale_without_pv_wait":
-                    yield from upto(i - 1)
-                assert pv_done == list(range(i)), f"half {h} rescaled O at tile {i} with PVs done {pv_done}"
-            S[b][1].add(h)
-            P[b][h] = i  # over this half's own S columns (it has read them; the partner never does)
+            P[g] = i  # over S(i), which this group has read
             yield
-            # PV(i - 2) is consumed before P(i) is released: PV(i) is issued only after the release, so
-            # the barrier is then at most one phase ahead of this consumer (no parity aliasing), and
-            # PV(i - 1) may still run while this half works on tile i + 1
-            if i >= 2 and plant != "release_without_pv_wait":
-                yield from upto(i - 2)
-            bars[f"pfull{i & 1}"].arrive()
+            if x >= 1:
+                if plant not in ("rescale_without_pv_wait", "release_without_pv_wait"):
+                    yield from upto(x - 1)
+                if rnd.random() < 0.3 or plant == "rescale_without_pv_wait":  # the group's max grew
+                    mine = [j for j in pv_done if j % 2 == g]
+                    assert mine == list(range(g, i, 2)), f"group {g} rescaled O at tile {i} with PVs done {pv_done}"
+            bars[f"pfull{g}"].arrive()
             yield
-        yield from upto(NT - 1)
-        assert pv_done == list(range(NT)), f"half {h} read O with PVs done {pv_done}"
+        mine = len(range(g, NT, 2))
+        if mine:
+            yield from upto(mine - 1)
+        assert [j for j in pv_done if j % 2 == g] == list(range(g, NT, 2)), f"group {g} read O with PVs done {pv_done}"
 
     actors = [producer(), mma(), softmax(0), softmax(1)]
     engines = [tma_engine(), tensor_pipe()]
@@ -205,7 +207,8 @@ def test_protocol_random_interleavings(NT):
         run(NT, seed)
 
 
-@pytest.mark.parametrize("plant", ["pv_skips_v_wait", "rescale_without_pv_wait", "release_without_pv_wait"])
+@pytest.mark.parametrize("plant", ["pv_skips_v_wait", "rescale_without_pv_wait", "release_without_pv_wait",
+                                   "k_slot_not_released"])
 def test_planted_protocol_mistakes_are_caught(plant):
     """Each planted mistake drops one wait of the protocol; some interleaving must trip a check."""
     caught = 0
@@ -218,13 +221,15 @@ def test_planted_protocol_mistakes_are_caught(plant):
 
 
 def test_model_matches_kernel_source():
-    """The model's ring depth and barrier arrival counts are the kernel's: two K/V stages, one
-    arrival (the TMA transaction) for the query tiles, every softmax thread for P, one commit
-    for each of the tensor-pipe barriers."""
+    """The model's ring depth and barrier arrival counts are the kernel's: two K/V stages released
+    through the S and PV barriers, one arrival (the TMA transaction) for the query tiles, the
+    threads of one softmax group for P, one commit for each of the tensor-pipe barriers."""
     src = open(KERNEL).read()
     assert int(re.search(r"constexpr int NSTAGE = (\d+);", src).group(1)) == NSTAGE
-    for init in ("mbar_init(&bars->q, 1)", "mbar_init(&bars->pfull[b], NSOFT)", "mbar_init(&bars->pvdone[b], 1)",
-                 "mbar_init(&bars->sfull[b], 1)", "mbar_init(&bars->kfull[s], 1)", "mbar_init(&bars->vempty[s], 1)"):
+    for init in ("mbar_init(&bars->q, 1)", "mbar_init(&bars->pfull[b], NSOFT / 2)", "mbar_init(&bars->pvdone[b], 1)",
+                 "mbar_init(&bars->sfull[b], 1)", "mbar_init(&bars->kfull[s], 1)", "mbar_init(&bars->vfull[s], 1)",
+                 "wait_bar(&bars->sfull[s], (use - 1) & 1", "wait_bar(&bars->pvdone[s], (use - 1) & 1"):
         assert init in src, init
-    # the two halves of a row never wait for each other inside the tile loop (no exchange barrier)
-    assert "bars->mx" not in src
+    # no separate slot-release barriers, and the two groups never exchange inside the tile loop
+    for gone in ("kempty", "vempty", "bars->mx"):
+        assert gone not in src, gone
