@@ -307,8 +307,8 @@ __device__ void softmax_role(const Plan& P, const Dev& D, Bars* bars, float* lsu
             const float p0 = ex2(fmaf(s[2 * e], sc, nref)), p1 = ex2(fmaf(s[2 * e + 1], sc, nref));
             rs[(2 * e) & 7] += p0;
             rs[(2 * e + 1) & 7] += p1;
-            __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
-            w[e] = *reinterpret_cast<uint32_t*>(&h);
+            // bf16 pair on the integer pipe: round half up (+0x8000), keep the two high halves
+            w[e] = __byte_perm(__float_as_uint(p0) + 0x8000u, __float_as_uint(p1) + 0x8000u, 0x7632);
         }
         ptx::tmem_st32(sbase, reinterpret_cast<const float*>(w));  // over columns [0, 64) of S_i, read above
         ptx::tmem_st32(sbase + 32, reinterpret_cast<const float*>(w + 32));
