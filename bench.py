@@ -86,6 +86,7 @@ class ClockSampler:
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.rows = []
+        self.skip = 0
         self.proc = None
         self.thread = None
 
@@ -96,6 +97,12 @@ class ClockSampler:
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
+            # nvidia-smi takes a while to start: wait (bounded) for its first sample, so that sampling is
+            # live when the timed region begins; only the samples after this one are summarised
+            t0 = time.time()
+            while not self.rows and time.time() - t0 < 5.0 and self.proc.poll() is None:
+                time.sleep(0.01)
+            self.skip = len(self.rows)
         except Exception:
             self.proc = None
         return self
@@ -106,6 +113,10 @@ class ClockSampler:
 
     def __exit__(self, *a):
         if self.proc:
+            # a region shorter than the sampling period still gets the sample that ends it
+            t0 = time.time()
+            while len(self.rows) <= self.skip and time.time() - t0 < 0.5 and self.proc.poll() is None:
+                time.sleep(0.01)
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
@@ -115,15 +126,16 @@ class ClockSampler:
             self.thread.join(timeout=2)
 
     def summary(self):
-        if not self.rows:
+        rows = self.rows[self.skip:] or self.rows
+        if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
-        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in self.rows for i in range(4) if len(r) > 5 + i and r[5 + i] == "Active"})
+        reasons = sorted({names[i] for r in rows for i in range(4) if len(r) > 5 + i and r[5 + i] == "Active"})
         load = [s for s in sm if s > 0.5 * (max(sm) if sm else 1)]
         return {"sm_mhz": float(np.median(load)) if load else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(self.rows)}
+                "reasons": reasons, "samples": len(rows)}
 
 
 # ------------------------------------------------------------------------------------------------
