@@ -21,7 +21,8 @@ Every data hand-off is asserted where it happens:
 - S(i) is read only once QK(i) has written it, and is not overwritten before its group read it;
 - PV(j) reads P(j), and never a stale one;
 - O_g is read or rescaled only when no PV that writes it is pending;
-- a parity wait never runs two or more phases behind its barrier, where parity aliases;
+- a parity wait never runs two or more phases behind its barrier, where parity aliases, nor
+  starts before the previous phase completed, where it would pass early;
 - no interleaving deadlocks (bounded step count).
 A planted protocol mistake must fail the same checks (last test).
 """
@@ -40,7 +41,8 @@ KERNEL = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))
 
 class Bar:
     """mbarrier: `count` arrivals complete a phase; a parity wait for phase j is true once phase j
-    has completed, and is ambiguous (aliases) if two or more phases completed past it."""
+    has completed. It aliases if two or more phases completed past it (it would wait for a third),
+    and it passes early if phase j - 1 has not completed yet (phase j - 2 has j's parity)."""
 
     def __init__(self, name, count):
         self.name, self.count, self.arrived, self.phase = name, count, 0, 0
@@ -54,6 +56,7 @@ class Bar:
 
     def done(self, j):
         assert self.phase < j + 2, f"{self.name}: parity wait for phase {j} after {self.phase} completed phases"
+        assert self.phase >= j, f"{self.name}: parity wait for phase {j} with only {self.phase} completed (passes early)"
         return self.phase > j
 
 
