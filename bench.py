@@ -192,13 +192,18 @@ ATTN_PROFILE = os.path.join(ROOT, "profiles", "k_attn_tc_mistral_128k.md")
 ATTN_SOURCE = os.path.join(ROOT, "block_memory_sparse_b200", "csrc", "attend_tc.cu")
 
 
-def attn_device_hash():
+def attn_device_hash(src=None):
     """sha256 of the attention kernel's device code: attend_tc.cu up to its host-side part (the
-    tensor-map encoding and the launcher), which does not change what the kernel moves."""
+    tensor-map encoding and the launcher), which does not change what the kernel moves, with
+    comments and trailing blanks removed (editing a comment does not change the kernel)."""
     import hashlib
-    src = open(ATTN_SOURCE, "rb").read()
-    cut = src.find(b"typedef CUresult (*EncodeTiledFn)")
-    return hashlib.sha256(src if cut < 0 else src[:cut]).hexdigest()
+    import re
+    src = open(ATTN_SOURCE).read() if src is None else src
+    cut = src.find("typedef CUresult (*EncodeTiledFn)")
+    code = src if cut < 0 else src[:cut]
+    code = re.sub(r"/\*.*?\*/", "", code, flags=re.S)
+    code = "\n".join(line.split("//", 1)[0].rstrip() for line in code.splitlines())
+    return hashlib.sha256(code.encode()).hexdigest()
 
 
 def attn_traffic():

@@ -57,8 +57,8 @@ struct Lay {
     static constexpr int OFF_K = OFF_QW + (int)TILE;
     static constexpr int OFF_V = OFF_K + NSTAGE * (int)TILE;
     static constexpr int OFF_BAR = OFF_V + NSTAGE * (int)TILE;
-    static constexpr int OFF_LSUM = OFF_BAR + 256;           // [2 halves][128] row sums
-    static constexpr int OFF_MREF = OFF_LSUM + 2 * 128 * 4;  // [2 halves][128] reference maxima (log2 units)
+    static constexpr int OFF_LSUM = OFF_BAR + 256;           // [2 groups][128] row sums
+    static constexpr int OFF_MREF = OFF_LSUM + 2 * 128 * 4;  // [2 groups][128] reference maxima (log2 units)
     static constexpr int OFF_SEL = OFF_MREF + 2 * 128 * 4;   // selected unit ids of this KV head
     static constexpr int SMEM_BYTES = OFF_SEL + MAX_SEL * 4 + 1024;  // + alignment slack
 };
@@ -66,7 +66,7 @@ static_assert(Lay<128>::SMEM_BYTES <= 227 * 1024, "shared-memory layout exceeds 
 
 // TMEM columns: S0 / P0 [0,128), S1 / P1 [128,256), O_0 [256, 256 + HD), O_1 [256 + HD, 256 + 2 HD)
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t TM_O = 256;  // O_h: the products with the keys of column half h of every tile
+constexpr uint32_t TM_O = 256;  // O_g: the products with the KV tiles of parity g
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float RESCALE_LOG2 = 8.0f;
 constexpr int ERR_TIMEOUT = 16;
@@ -206,7 +206,7 @@ __device__ void mma_issuer(const Plan& P, const Dev& D, uint8_t* sm, Bars* bars,
             ptx::tc_fence_after();
             const uint32_t va = vb + sj * Y::TILE;
 #pragma unroll
-            for (int ks = 0; ks < BN / 16; ++ks)  // keys 16 ks ..: half h = ks / 4 of P_j into O_h
+            for (int ks = 0; ks < BN / 16; ++ks)  // keys 16 ks .. 16 ks + 15 of P_j, into O_{j & 1}
                 ptx::mma_bf16_ts(tmem + TM_O + (uint32_t)bj * HD, tmem + bj * BN + (uint32_t)ks * 8,
                                  ptx::sdesc_sw128(va + (uint32_t)ks * 2048, SWB, 1024), IDESC_PV,
                                  (j > 1 || ks > 0) ? 1u : 0u);
