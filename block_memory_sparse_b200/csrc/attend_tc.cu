@@ -26,6 +26,8 @@
 // executes one thread's MMAs in issue order.  The MMA-issuing thread keeps pace with the tensor
 // pipe (its queue is short), so its loop holds no lookups: the K and V ring slots are released by
 // the same two barriers that announce S_i and PV(i), and the query tile is chosen by tile index.
+// Likewise each softmax group does what does not need S_i (the tile's column limit, consuming its
+// previous PV) while QK(i) runs, so that only the max, the exponentials and the store follow S_i.
 // Sinks and memory tiles use R(W) q with raw keys; window tiles use R(t) q with R(n) k.
 #include <cuda.h>
 #include <math.h>
@@ -265,6 +267,21 @@ __device__ void softmax_role(const Plan& P, const Dev& D, Bars* bars, float* lsu
     bool ok = true;
     for (int i = grp; i < P.NT; i += 2) {
         const int x = i >> 1;  // this group's tile count before tile i
+        // columns [0, lim) of this tile are attended by this row (causal limit on sinks and window);
+        // known before S(i) lands
+        const TileInfo T = P.tile(D, i);
+        int lim = T.nv;
+        if (T.kind != 1) {
+            const int64_t c = t - T.y0 + 1;
+            lim = c < (int64_t)lim ? (int)(c < 0 ? 0 : c) : lim;
+        }
+        const bool full = __all_sync(0xffffffffu, lim >= BN);
+        // O_grp holds this group's earlier products (and P_i may be released) once PV of its previous
+        // tile is complete; PV(i - 2) was issued before QK(i), so it is complete before S(i) lands
+        if (x >= 1 && !pv.upto(x - 1, pvbar, bars, D)) {
+            ok = false;
+            break;
+        }
         if (!warp_wait(&bars->sfull[grp], (uint32_t)x & 1, bars, D)) {
             ok = false;
             break;
@@ -276,16 +293,10 @@ __device__ void softmax_role(const Plan& P, const Dev& D, Bars* bars, float* lsu
         ptx::tmem_ld32(sbase + 64, s + 64);
         ptx::tmem_ld32(sbase + 96, s + 96);
         ptx::tmem_wait_ld();
-        const TileInfo T = P.tile(D, i);
-        int lim = T.nv;
-        if (T.kind != 1) {
-            const int64_t c = t - T.y0 + 1;
-            lim = c < (int64_t)lim ? (int)(c < 0 ? 0 : c) : lim;
-        }
         float mq[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) mq[e] = -INFINITY;
-        if (!__all_sync(0xffffffffu, lim >= BN)) {
+        if (!full) {
 #pragma unroll
             for (int c = 0; c < 128; ++c) s[c] = c < lim ? s[c] : -INFINITY;
         }
@@ -313,24 +324,17 @@ __device__ void softmax_role(const Plan& P, const Dev& D, Bars* bars, float* lsu
         ptx::tmem_st32(sbase, reinterpret_cast<const float*>(w));  // over columns [0, 64) of S_i, read above
         ptx::tmem_st32(sbase + 32, reinterpret_cast<const float*>(w + 32));
         l = fmaf(l, f, ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7])));
-        // O_grp holds this group's earlier products (and P_i may be released) once PV of its previous
-        // tile is complete; a growing maximum rescales O_grp here, before PV(i) adds to it
-        if (x >= 1) {
-            if (!pv.upto(x - 1, pvbar, bars, D)) {
-                ok = false;
-                break;
-            }
-            if (__any_sync(0xffffffffu, need)) {
-                ptx::tc_fence_after();
+        // a growing maximum rescales O_grp here, before PV(i) adds to it
+        if (x >= 1 && __any_sync(0xffffffffu, need)) {
+            ptx::tc_fence_after();
 #pragma unroll
-                for (int c4 = 0; c4 < HD / 32; ++c4) {
-                    float o[32];
-                    ptx::tmem_ld32(o_addr + c4 * 32, o);
-                    ptx::tmem_wait_ld();
+            for (int c4 = 0; c4 < HD / 32; ++c4) {
+                float o[32];
+                ptx::tmem_ld32(o_addr + c4 * 32, o);
+                ptx::tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) o[e] *= f;
-                    ptx::tmem_st32(o_addr + c4 * 32, o);
-                }
+                for (int e = 0; e < 32; ++e) o[e] *= f;
+                ptx::tmem_st32(o_addr + c4 * 32, o);
             }
         }
         ptx::tmem_wait_st();

@@ -12,9 +12,9 @@ interleaves at random, with exact mbarrier parity semantics.
   earlier MMA is done.
 - TMA engine: lands copies in any order.
 - Two softmax groups: group g takes the tiles i with i & 1 == g, reads all of S(i), writes P(i)
-  over it and keeps its own online softmax and accumulator O_g. A group may rescale O_g only
-  after its previous PV is complete, and releases P(i) only after that PV is complete (so the
-  PV barrier of its parity is never two phases ahead of it).
+  over it and keeps its own online softmax and accumulator O_g. Before it waits for S(i) it
+  consumes its previous PV, so it rescales O_g and releases P(i) only after that PV is complete
+  (and the PV barrier of its parity is never two phases ahead of it).
 
 Every data hand-off is asserted where it happens:
 - a ring slot is refilled only after the MMA that read it has executed;
@@ -167,6 +167,10 @@ def run(NT, seed, plant=None):
 
         for i in range(g, NT, 2):
             x = i >> 1
+            # the group's previous PV is consumed before the wait for S(i) (it completes first anyway:
+            # PV(i - 2) was issued before QK(i)); rescaling O_g and releasing P(i) both follow it
+            if x >= 1 and plant not in ("rescale_without_pv_wait", "release_without_pv_wait"):
+                yield from upto(x - 1)
             yield from wait(f"sfull{g}", x)
             assert S[g] is not None and S[g][0] == i, f"group {g} read S buffer {g} = {S[g]} for tile {i}"
             S[g][1] = True
@@ -174,8 +178,6 @@ def run(NT, seed, plant=None):
             P[g] = i  # over S(i), which this group has read
             yield
             if x >= 1:
-                if plant not in ("rescale_without_pv_wait", "release_without_pv_wait"):
-                    yield from upto(x - 1)
                 if rnd.random() < 0.3 or plant == "rescale_without_pv_wait":  # the group's max grew
                     mine = [j for j in pv_done if j % 2 == g]
                     assert mine == list(range(g, i, 2)), f"group {g} rescaled O at tile {i} with PVs done {pv_done}"
