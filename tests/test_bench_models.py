@@ -47,3 +47,20 @@ def test_decode_bytes_counts_keys_and_the_scoring_operand(mode):
         per_unit = w.n_reps * w.head_dim * elt if mode == "reps" else w.head_dim * 4
         want = nm * w.n_kv_heads * per_unit + keys * w.n_kv_heads * w.head_dim * elt * 2
         assert bench.decode_bytes(w, t, mode) == want, t
+
+
+def test_attention_traffic_key_ignores_comments_only():
+    """The captured DRAM traffic is keyed to the attention kernel's device code: editing a comment
+    keeps the key, changing a statement or anything before the host-side part changes it, and the
+    host-side part (tensor maps, launcher) does not enter it."""
+    src = open(bench.ATTN_SOURCE).read()
+    cut = src.index("typedef CUresult (*EncodeTiledFn)")
+    base = bench.attn_device_hash(src)
+    line = "constexpr int BN = 128;  // keys per tile"
+    assert line in src
+    assert bench.attn_device_hash(src.replace(line, "constexpr int BN = 128;  // keys in one tile")) == base
+    assert bench.attn_device_hash(src.replace("// Exact attention", "/* a block comment */\n// Exact attention", 1)) == base
+    assert bench.attn_device_hash(src.replace(line, "constexpr int BN = 64;  // keys per tile")) != base
+    assert bench.attn_device_hash(src[:cut] + src[cut:].replace("return", "return ", 1)) == base
+    # the committed profile's key matches the committed kernel, so the bench reports its traffic
+    assert bench.attn_traffic() is not None
