@@ -195,14 +195,14 @@ ATTN_SOURCE = os.path.join(ROOT, "block_memory_sparse_b200", "csrc", "attend_tc.
 def attn_device_hash(src=None):
     """sha256 of the attention kernel's device code: attend_tc.cu up to its host-side part (the
     tensor-map encoding and the launcher), which does not change what the kernel moves, with
-    comments and trailing blanks removed (editing a comment does not change the kernel)."""
+    comments, trailing blanks and empty lines removed (editing a comment does not change the kernel)."""
     import hashlib
     import re
     src = open(ATTN_SOURCE).read() if src is None else src
     cut = src.find("typedef CUresult (*EncodeTiledFn)")
     code = src if cut < 0 else src[:cut]
     code = re.sub(r"/\*.*?\*/", "", code, flags=re.S)
-    code = "\n".join(line.split("//", 1)[0].rstrip() for line in code.splitlines())
+    code = "\n".join(x for x in (line.split("//", 1)[0].rstrip() for line in code.splitlines()) if x)
     return hashlib.sha256(code.encode()).hexdigest()
 
 
