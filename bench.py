@@ -378,7 +378,7 @@ def run_ours(args, rank, world):
            "roofline": fields["roofline"], "gpu_launches": fields["gpu_launches"], "clocks": fields["clocks"],
            "time_split_ms_per_step": fields["time_split_ms_per_step"]}
     if not args.no_e2e and plan is None:
-        res["e2e"] = run_e2e(args, w, layer, q_h, k_h, v_h, torch, device, stream, world)
+        res["e2e"] = run_e2e(args, w, layer, q_h, k_h, v_h, torch, device, stream, world, args.e2e_group)
     layer.close()
     del q_h, k_h, v_h
     torch.cuda.empty_cache()
@@ -403,7 +403,7 @@ def run_ours(args, rank, world):
     return res
 
 
-def run_e2e(args, w, layer, q_h, k_h, v_h, torch, device, stream, world, group_chunks=8):
+def run_e2e(args, w, layer, q_h, k_h, v_h, torch, device, stream, world, group_chunks=32):
     """Same prompt through the public API with inputs in pinned host memory and the output read
     back to host: host<->device copies are inside the timed region.  The prompt goes in groups
     of `group_chunks` chunks (one infllm_prefill call each); the copies run on two side streams
@@ -612,6 +612,8 @@ def main():
     ap.add_argument("--decode-units", type=int, default=0, help="memory units of the decode workload (0: 8192)")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-group", type=int, default=32,
+                    help="chunks per host<->device copy group of the e2e arm (32 measured best of 4-64)")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-others", action="store_true", help="skip the other prefill workloads")
     ap.add_argument("--parallel", choices=["replicas", "kv"], default="replicas",
